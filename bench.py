@@ -1,0 +1,528 @@
+#!/usr/bin/env python
+"""Benchmark of the ReLU linear-attention forward on B200.
+
+One step = one whole-sequence forward (ReLU + 3D RoPE prologue, state build,
+reduction, apply) of the 480p-shaped workload: B=1, H=32, N=32760 (21 x 30 x 52
+latent grid), D=64, bf16 I/O, fp32 state, RoPE split 16/24/24, theta 1e4.
+Inputs (537 MB per step) are larger than the 126 MB L2, so no flush is needed
+between steps. Timing: W warm-up steps, then K steps bracketed by a barrier and
+torch.cuda.synchronize() on both sides, CUDA events on the launching stream,
+max over ranks. With --gpus N every rank runs its own replica (weak scaling,
+no collective on the data path).
+
+Prints one JSON line (rank 0). ``--impl reference`` times the fp64 CPU oracle
+on the host cores instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "linear-attn fwd tokens/s & HBM GB/s (% of peak), N=32760 H=32 D=64 bf16"
+MAIN = "480p_bidir"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- dist ----
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def reduce_max(value: float, pg, device=None) -> float:
+    """Max of a float over ranks (identity without a process group)."""
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, device=None):
+    if pg is not None:
+        if device is not None:
+            pg.barrier(device_ids=[device.index])
+        else:
+            pg.barrier()
+
+
+# ------------------------------------------------------------- helpers ----
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_video_relu_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (a line '# bench-traffic <kernel> <workload>
+    <bytes> <source-hash>' in profiles/*.txt); else None."""
+    pdir = os.path.join(ROOT, "profiles")
+    want = kernel_source_hash()
+    if not os.path.isdir(pdir):
+        return None
+    for name in sorted(os.listdir(pdir)):
+        if not name.endswith((".txt", ".md")):
+            continue
+        with open(os.path.join(pdir, name)) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 6 and parts[0] == "#" and parts[1] == "bench-traffic":
+                    if parts[2] == kernel and parts[3] == workload and parts[5] == want:
+                        return int(parts[4])
+    return None
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, clock-event reasons) while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def device_inputs(w: workloads.Workload, device, seed: int):
+    """Seeded synthetic inputs drawn on the device (same shapes and value
+    distributions as workloads.make_inputs; a torch CUDA generator here)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    shape = (w.B, w.H, w.N, w.D)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    out = {}
+    for name in ["q", "k", "v"] + (["g"] if w.gate else []):
+        if w.qk_dist == "student_t3" and name in ("q", "k"):
+            # t_3 = Z / sqrt(chi2_3 / 3), scaled to unit variance
+            z = torch.randn(shape, generator=g, device=device)
+            chi = torch.randn((3,) + shape, generator=g, device=device).pow_(2).sum(0)
+            x = z / torch.sqrt(chi / 3.0) / math.sqrt(3.0)
+            del z, chi
+        else:
+            x = torch.randn(shape, generator=g, device=device)
+        out[name] = x.to(dt)
+        del x
+    return out
+
+
+# ---------------------------------------------------------- GPU timing ----
+
+def time_forward(w, mode, t, steps, warmup, pg, device, record_kernels=True):
+    """Time `steps` forwards; returns (max-over-ranks ms, per-kernel ms lists)."""
+    import torch
+    import linear_attention_video_relu_b200 as la
+    C = la._native
+    p = la.make_params(w.B, w.H, w.N, w.D, t["q"].dtype, mode,
+                       w.block_tokens if mode == "block_causal" else 0, w.grid, w.rope_split,
+                       w.rope_theta, w.eps)
+    ws = la.workspace_for(p, device)
+    out = torch.empty_like(t["q"])
+    stream = torch.cuda.current_stream(device)
+    sp = stream.cuda_stream
+    args = (p, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(),
+            t["g"].data_ptr() if "g" in t else None, out.data_ptr(), ws.ptr, ws.nbytes, sp)
+    for _ in range(warmup):
+        C.check(C.lin_attn_forward(*args), "lin_attn_forward")
+    evs = []
+    if record_kernels:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        for row in evs:
+            for e in row:
+                e.record(stream)          # materialise the event handles
+    torch.cuda.synchronize(device)
+    barrier(pg, device)
+    torch.cuda.synchronize(device)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        if record_kernels:
+            C.check(C.lin_attn_forward_timed(*args, [e.cuda_event for e in evs[i]]),
+                    "lin_attn_forward_timed")
+        else:
+            C.check(C.lin_attn_forward(*args), "lin_attn_forward")
+    stop.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(pg, device)
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(stop)
+    st = C.lin_attn_device_status(ws.ptr, sp)
+    if st != C.LA_OK:
+        raise RuntimeError("device status after timing: %s" % C.status_string(st))
+    kern = None
+    if record_kernels:
+        kern = [[r[j].elapsed_time(r[j + 1]) for r in evs] for j in range(3)]
+    ms_max = reduce_max(ms, pg, device)
+    return ms_max, kern, out
+
+
+def roofline_entry(name, bytes_per_launch, ms_list, peak, peak_kind, workload):
+    avg_ms = sum(ms_list) / len(ms_list)
+    gbs = bytes_per_launch / (avg_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(name, workload)
+    return {"kernel": name, "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(gbs / peak, 4), "traffic": traffic,
+            "algorithmic_bytes": bytes_per_launch, "avg_us": round(avg_ms * 1e3, 2),
+            "peak_source": peak_kind}
+
+
+def measure_workload(w, mode, steps, warmup, pg, device, peak, peak_kind, seed):
+    import torch
+    t = device_inputs(w, device, seed)
+    ms, kern, out = time_forward(w, mode, t, steps, warmup, pg, device)
+    elt = 2 if w.dtype == "bf16" else 4
+    tensor_bytes = w.B * w.H * w.N * w.D * elt
+    state_bytes = 2 * tensor_bytes
+    apply_bytes = (3 if w.gate else 2) * tensor_bytes
+    step_ms = ms / steps
+    k_state = roofline_entry("state_build", state_bytes, kern[0], peak, peak_kind, w.name)
+    k_reduce_us = round(sum(kern[1]) / len(kern[1]) * 1e3, 2)
+    k_apply = roofline_entry("apply", apply_bytes, kern[2], peak, peak_kind, w.name)
+    total_bytes = w.algorithmic_bytes()
+    res = {
+        "workload": w.name, "mode": mode, "ms_per_step": step_ms,
+        "tokens_per_s": w.B * w.N / (step_ms * 1e-3),
+        "hbm_gbs": total_bytes / (step_ms * 1e-3) / 1e9,
+        "hbm_frac": total_bytes / (step_ms * 1e-3) / 1e9 / peak,
+        "kernels": {"state_build": k_state, "reduce_us": k_reduce_us, "apply": k_apply},
+    }
+    del t, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_block_steps(w, steps, warmup, device, peak, peak_kind, seed):
+    """Algorithm 1's per-block call: lin_attn_block_step with commit on every
+    block of the 720p workload, one call per block."""
+    import torch
+    import linear_attention_video_relu_b200 as la
+    t = device_inputs(w, device, seed)
+    bt = w.block_tokens
+    T, Hg, Wg = w.grid
+    fpb = bt // (Hg * Wg)
+    nblk = w.N // bt
+    blocks = [{n: t[n][:, :, b * bt:(b + 1) * bt].contiguous() for n in t} for b in range(nblk)]
+    del t
+    st = la.BlockState(w.B, w.H, w.D, device=device)
+    outs = [torch.empty_like(blocks[0]["q"]) for _ in range(2)]
+
+    def run_all():
+        for b in range(nblk):
+            st.step(blocks[b]["q"], blocks[b]["k"], blocks[b]["v"], t_offset=b * fpb, commit=True,
+                    grid=(fpb, Hg, Wg), rope_split=w.rope_split, eps=w.eps, out=outs[b % 2])
+
+    reps = max(1, steps // nblk)
+    for _ in range(max(1, warmup // nblk)):
+        st.reset()
+        run_all()
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        run_all()
+    b_.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b_) / (reps * nblk)
+    bytes_blk = 4 * w.B * w.H * bt * w.D * 2
+    return {"workload": w.name + "_block_step", "block_tokens": bt, "us_per_block": ms * 1e3,
+            "tokens_per_s": w.B * bt / (ms * 1e-3),
+            "hbm_frac": bytes_blk / (ms * 1e-3) / 1e9 / peak}
+
+
+def measure_e2e(w, steps, device, seed):
+    """The same forward end to end: host (pinned) inputs copied in, the C-ABI
+    call, the output copied back, every step, all inside the timed region."""
+    import torch
+    import linear_attention_video_relu_b200 as la
+    td = device_inputs(w, device, seed)
+    host = {n: torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for n, x in td.items()}
+    for n in td:
+        host[n].copy_(td[n])
+    out_h = torch.empty(td["q"].shape, dtype=td["q"].dtype, pin_memory=True)
+    ws = None
+    p = la.make_params(w.B, w.H, w.N, w.D, td["q"].dtype, "bidirectional", 0, w.grid,
+                       w.rope_split, w.rope_theta, w.eps)
+    ws = la.workspace_for(p, device)
+    out_d = torch.empty_like(td["q"])
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for n in td:
+            td[n].copy_(host[n], non_blocking=True)
+        la.forward(td["q"], td["k"], td["v"], td.get("g"), grid=w.grid, rope_split=w.rope_split,
+                   theta=w.rope_theta, eps=w.eps, out=out_d, workspace=ws)
+        out_h.copy_(out_d, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    return {"value": w.B * w.N / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+
+
+# ----------------------------------------------------------- CPU oracle ----
+
+def oracle_sample(w, budget_s: float, max_heads=None):
+    """Time the fp64 oracle (as it stands) on a bounded sample of workload w:
+    the first `heads` heads over the first `frames` latent frames."""
+    import numpy as np
+    import oracle
+    cores = oracle.threads(0)
+    heads = min(w.B * w.H, max_heads or cores)
+    T, Hg, Wg = w.grid
+    # about 1.5 us of CPU per token per head-dim^2/4096 unit: size frames to the budget
+    frames = T
+    est = lambda f: heads * f * Hg * Wg * (w.D * w.D / 4096.0) * 12e-6 / min(cores, heads)
+    while frames > 1 and est(frames) > budget_s:
+        frames -= 1
+    sw = workloads.Workload(name=w.name + "_sample", B=1, H=heads, N=frames * Hg * Wg, D=w.D,
+                            dtype=w.dtype, seed=w.seed, grid=(frames, Hg, Wg),
+                            rope_split=w.rope_split, gate=w.gate, qk_dist=w.qk_dist)
+    x = workloads.make_inputs(sw)
+    p = oracle.params_for(sw, "bidirectional")
+    return sw, x, p, min(cores, heads)
+
+
+def run_oracle_once(sw, x, p, cores):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward(p, x["q"], x["k"], x["v"], g=x.get("g"), nthreads=cores)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w):
+    sw, x, p, cores = oracle_sample(w, budget_s=8.0)
+    dt = run_oracle_once(sw, x, p, cores)
+    # tokens/s of the whole workload: the sample covers sw.H of the w.B*w.H heads
+    tok_s = sw.N * (sw.H / (w.B * w.H)) / dt
+    return {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "%d of %d heads x %d tokens (%d frames) of %s, fp64, %.1f s wall" % (
+                sw.H, w.B * w.H, sw.N, sw.grid[0], w.name, dt)}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle on the host cores."""
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS[MAIN]
+    total_steps = args.steps + args.warmup
+    per_step = max(0.05, min(2.0, 120.0 / max(total_steps, 1)))
+    sw, x, p, cores = oracle_sample(w, budget_s=per_step)
+    for _ in range(args.warmup):
+        run_oracle_once(sw, x, p, cores)
+    t = 0.0
+    for _ in range(args.steps):
+        t += run_oracle_once(sw, x, p, cores)
+    step_s = t / max(args.steps, 1)
+    tok_s = sw.N * (sw.H / (w.B * w.H)) / step_s
+    sample = "%d of %d heads x %d tokens (%d frames) of %s per step, fp64" % (
+        sw.H, w.B * w.H, sw.N, sw.grid[0], w.name)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, "bidirectional", world),
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, mode, world):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "mode": mode,
+            "grid": list(w.grid) if w.grid else None,
+            "rope_split": list(w.rope_split) if w.rope_split else None,
+            "gate": w.gate, "global_batch": w.B * world, "seq_len": w.N,
+            "parallelism": "replicas x%d" % world,
+            "l2": "inputs larger than L2 (%.0f MB per step vs 126 MB), no flush" % (
+                w.algorithmic_bytes() / 1e6)}
+
+
+# ------------------------------------------------------------------ main ----
+
+def main():
+    args = parse_args()
+    world, rank, local, pg = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    import torch
+    import linear_attention_video_relu_b200 as la
+    la._native.load()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peak, peak_kind = measured_peaks()
+    w = workloads.WORKLOADS[MAIN]
+
+    t = device_inputs(w, device, seed=w.seed + rank)
+    # settle clocks with untimed work, then sample clocks across the timed region
+    _ = time_forward(w, "bidirectional", t, 50, args.warmup, None, device, record_kernels=False)
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms, kern, out = time_forward(w, "bidirectional", t, args.steps, 3, pg, device)
+    sampler.stop()
+    del t, out
+    torch.cuda.empty_cache()
+
+    step_ms = ms / args.steps
+    tokens = w.B * w.N * world
+    value = tokens / (step_ms * 1e-3)
+    elt = 2
+    tensor_bytes = w.B * w.H * w.N * w.D * elt
+    k_state = roofline_entry("state_build", 2 * tensor_bytes, kern[0], peak, peak_kind, w.name)
+    k_apply = roofline_entry("apply", 2 * tensor_bytes, kern[2], peak, peak_kind, w.name)
+    dominant = k_state if k_state["avg_us"] >= k_apply["avg_us"] else k_apply
+    total_bytes = w.algorithmic_bytes()
+    gbs = total_bytes / (step_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded torch CUDA generator, N(0,1) -> bf16)",
+        "config": config_of(w, "bidirectional", world),
+        "hbm_gbs": round(gbs, 1), "hbm_frac_of_peak": round(gbs / peak, 4),
+        "peak_hbm_gbs": peak, "peak_source": peak_kind,
+        "roofline": dominant,
+        "kernels": {"state_build": k_state,
+                    "reduce_us": round(sum(kern[1]) / len(kern[1]) * 1e3, 2),
+                    "apply": k_apply},
+        "gpu_launches": 3 * args.steps,
+        "tensor_core_path": bool(la.uses_tensor_cores(w.B, w.H, w.N, w.D, torch.bfloat16,
+                                                      grid=w.grid, rope_split=w.rope_split)),
+        "clocks": sampler.summary(),
+    }
+    if rank == 0:
+        line["e2e"] = measure_e2e(w, args.e2e_steps, device, w.seed)
+    if not args.no_extra and rank == 0:
+        extra = []
+        K = max(20, args.steps // 5)
+        for name, mode in (("480p_block_causal", "block_causal"), ("720p_long", "bidirectional"),
+                           ("720p_long", "block_causal"), ("gated_d128", "bidirectional")):
+            ww = workloads.WORKLOADS[name]
+            extra.append(measure_workload(ww, mode, K, 3, None, device, peak, peak_kind,
+                                          ww.seed))
+        extra.append(measure_block_steps(workloads.WORKLOADS["720p_long"], 120, 60, device, peak,
+                                         peak_kind, 1004))
+        line["also"] = extra
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        barrier(pg, device)
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

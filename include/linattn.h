@@ -1,0 +1,178 @@
+/*
+ * linattn.h -- C ABI of a B200 (sm_100a) library for ReLU linear attention
+ * with 3D rotary position embeddings, the token mixer of the SANA-Video
+ * linear diffusion transformer.
+ *
+ * Source of the operation ("SANA-Video: Efficient Video Generation with Block
+ * Linear Diffusion Transformer", paper-graph analysis page, section 3.4):
+ *   - "ReLU Linear Attention Mechanism" (unnumbered equation): phi = ReLU,
+ *     S = sum_j phi(k_j)^T v_j (D x D) and z = sum_j phi(k_j) (D) are built
+ *     once and every query reads them.
+ *   - "Integration of 3D RoPE", Eq. 2: RoPE is applied after phi, in the
+ *     numerator only:
+ *         out_i = RoPE(phi(q_i)) . S / (phi(q_i) . z + eps),
+ *         S     = sum_j RoPE(phi(k_j))^T v_j,   z = sum_j phi(k_j).
+ *   - "Block Linear Attention with Constant-Memory KV Cache", Eq. 3 and
+ *     Algorithm 1: the state (S, z) is carried across blocks of frames; a
+ *     block reads the cached state plus its own tokens, and the cache is
+ *     updated once, after the block.
+ *   - The SANA-Video 2.0 pages (neuraltrendhub summary and abstract) call the
+ *     layers "gated" linear attention without a formula; the gate taken here
+ *     is out_i <- sigmoid(g_i) * out_i elementwise, after the normalisation.
+ *
+ * Readings where the pages say nothing (also listed in the design notes):
+ *   RoPE: the D dims split into three contiguous segments (t | h | w) of widths
+ *   rope_dt, rope_dh, rope_dw; inside a segment of width d, dims (2m, 2m+1)
+ *   rotate by pos * theta^(-2m/d): (x, y) -> (x cos a - y sin a,
+ *   x sin a + y cos a). Token n of a head sits at t = t_offset + n/(Hg*Wg),
+ *   h = (n/Wg) % Hg, w = n % Wg. eps is added after the dot product, so a row
+ *   with phi(q_i) = 0 yields 0.
+ *
+ * Conventions for every entry point:
+ *   - Memory. The caller owns all device memory (inputs, output, state,
+ *     workspace); the library allocates and frees nothing and keeps no global
+ *     mutable state, so calls are re-entrant.
+ *   - Layout. q, k, v, gate, out are contiguous [B, H, N, D] with D innermost,
+ *     in the I/O dtype. The state is fp32: S [B, H, D, D] with
+ *     S[a][c] = sum_j RoPE(phi(k_j))_a v_j,c, and z [B, H, D].
+ *   - Asynchrony. A call checks its arguments on the host, enqueues kernels on
+ *     `stream` (a cudaStream_t passed as void*, NULL = legacy default stream)
+ *     and returns; results are valid once the stream reaches that point.
+ *   - Errors. Every call returns la_status; nothing aborts, prints or throws.
+ *     Invalid arguments are rejected before any launch and leave memory
+ *     untouched. A launch failure returns LA_ERR_CUDA.
+ *   - Alignment. Every tensor pointer and the workspace must be 16-byte
+ *     aligned; D * sizeof(dtype) is then a multiple of 16.
+ *   - Aliasing. out may not overlap q, k, v or gate.
+ *   - Determinism. Reductions run in a fixed order: the same inputs on the
+ *     same device give bit-identical outputs and state.
+ */
+#ifndef LINATTN_H
+#define LINATTN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARG = 1,  /* a pointer, size or field is out of range */
+  LA_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels handle */
+  LA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
+  LA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  LA_ERR_DEVICE_TIMEOUT = 5 /* a kernel gave up a bounded wait (see
+                               lin_attn_device_status) */
+} la_status;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;   /* I/O dtype; state is fp32 */
+
+typedef enum { LA_BIDIRECTIONAL = 0, LA_BLOCK_CAUSAL = 1 } la_mode;
+
+typedef struct {
+  int B, H, N, D;        /* batch, heads, tokens per head, head dim.
+                            D in {32, 64, 128}; N >= 0 (N = 0: no work). */
+  la_dtype dtype;        /* dtype of q, k, v, gate and out */
+  la_mode mode;          /* bidirectional or block-causal */
+  int block_tokens;      /* block-causal: tokens per block, N % block_tokens == 0.
+                            A token of block b sees blocks 0..b (its own block
+                            whole). Ignored in bidirectional mode. */
+  int rope;              /* 0: no rotation (then the grid fields are ignored) */
+  int grid_t, grid_h, grid_w;     /* latent grid; N == grid_t*grid_h*grid_w */
+  int rope_dt, rope_dh, rope_dw;  /* even widths with sum D (t, h, w order) */
+  double rope_theta;     /* RoPE base, > 0 (10000 in the workloads here) */
+  float eps;             /* added to the denominator, >= 0 (1e-6 here) */
+} la_params;
+
+/* A carried block-causal state: caller-owned device memory, fp32,
+ * S [B, H, D, D] and z [B, H, D] (16-byte aligned). */
+typedef struct {
+  float* S;
+  float* z;
+  int B, H, D;
+} la_state;
+
+/* Bytes of workspace lin_attn_forward needs for `p` on the current device
+ * (the size depends on the device's SM count). Writes *bytes; no launch. */
+LA_API la_status lin_attn_workspace_size(const la_params* p, size_t* bytes);
+
+/* Bytes of workspace lin_attn_block_step / lin_attn_state_update need for a
+ * block of p->N tokens (mode and block_tokens are ignored). */
+LA_API la_status lin_attn_block_step_workspace_size(const la_params* p, size_t* bytes);
+
+/* The whole-sequence forward (Eq. 2, plus the gate when gate != NULL).
+ *   bidirectional: out_i uses S, z summed over all N tokens of its head.
+ *   block-causal:  out_i of block b uses S, z summed over blocks 0..b, which
+ *                  is Algorithm 1 run with an empty initial cache.
+ * q, k, v, out: [B,H,N,D] device pointers in p->dtype. gate: NULL or the same
+ * shape and dtype (logits; out is multiplied by their sigmoid).
+ * workspace: device memory of at least lin_attn_workspace_size bytes, 256-byte
+ * aligned; its contents on entry do not matter and are clobbered.
+ * Returns LA_OK once the work is enqueued on `stream`. */
+LA_API la_status lin_attn_forward(const la_params* p, const void* q, const void* k,
+                           const void* v, const void* gate, void* out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* lin_attn_forward that also records four caller-created CUDA events (as
+ * void*, e.g. cudaEvent_t) on `stream`: events[0] before the state build,
+ * events[1] after it, events[2] after the reduction, events[3] after the
+ * apply step, so a caller can time each kernel on the launching stream.
+ * events may be NULL (then this is lin_attn_forward). */
+LA_API la_status lin_attn_forward_timed(const la_params* p, const void* q, const void* k,
+                                        const void* v, const void* gate, void* out,
+                                        void* workspace, size_t workspace_bytes, void* stream,
+                                        void* const* events);
+
+/* Wrap caller-owned state buffers (no allocation, no launch). S and z must
+ * be device pointers, 16-byte aligned, of [B,H,D,D] and [B,H,D] floats. */
+LA_API la_status lin_attn_state_init(la_state* st, int B, int H, int D, float* S, float* z);
+
+/* Zero the state asynchronously on `stream` (the empty cache of Algorithm 1). */
+LA_API la_status lin_attn_state_reset(const la_state* st, void* stream);
+
+/* One block of Algorithm 1. p->N is the number of tokens in this block (its
+ * frames are grid_t latent frames starting at global frame t_offset, so RoPE
+ * positions stay global); p->mode and p->block_tokens are ignored.
+ *   out_i = RoPE(phi(q_i)) (S + S_blk) / (phi(q_i) . (z + z_blk) + eps)
+ * with (S, z) the carried state and (S_blk, z_blk) the sums over this block.
+ * commit != 0 then sets S += S_blk, z += z_blk in place (the cache update at
+ * the last denoising step); commit == 0 leaves the state byte-identical.
+ * gate may be NULL. The state must match p (B, H, D). */
+LA_API la_status lin_attn_block_step(const la_params* p, la_state* st, int t_offset,
+                              const void* q, const void* k, const void* v,
+                              const void* gate, void* out, int commit,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* The cache update alone (Algorithm 1's G^KV step, from the clean latent's
+ * k and v): S += sum_j RoPE(phi(k_j))^T v_j, z += sum_j phi(k_j) over the
+ * p->N tokens of the block. Same arguments as lin_attn_block_step without
+ * q, gate and out. */
+LA_API la_status lin_attn_state_update(const la_params* p, la_state* st, int t_offset,
+                                const void* k, const void* v, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream` and report whether any kernel of the last calls that
+ * used `workspace` gave up a bounded wait (LA_ERR_DEVICE_TIMEOUT) -- a safety
+ * net that should never fire. Clears the flag. */
+LA_API la_status lin_attn_device_status(void* workspace, void* stream);
+
+/* Static description of a status code. */
+LA_API const char* lin_attn_status_string(la_status s);
+
+/* Which kernel family lin_attn_forward would use for `p` on the current
+ * device: 1 = tensor-core (tcgen05 + TMA, bf16 I/O, D in {64, 128}),
+ * 0 = CUDA-core (fp32 I/O, or shapes outside the tensor-core path). */
+LA_API int lin_attn_uses_tensor_cores(const la_params* p);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LINATTN_H */

@@ -1,0 +1,155 @@
+"""Torch-facing wrapper of the C ABI: tensors in, tensors out.
+
+PyTorch provides device memory and streams only; the computation is the
+CUDA library's. Shapes follow include/linattn.h: q, k, v, gate, out are
+contiguous [B, H, N, D] in bf16 or fp32; the carried state is fp32
+S [B, H, D, D] and z [B, H, D].
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import torch
+
+from . import _native as C
+
+_DTYPES = {torch.bfloat16: C.LA_BF16, torch.float32: C.LA_F32}
+_MODES = {"bidirectional": C.LA_BIDIRECTIONAL, "block_causal": C.LA_BLOCK_CAUSAL}
+
+
+def make_params(B: int, H: int, N: int, D: int, dtype: torch.dtype, mode: str = "bidirectional",
+                block_tokens: int = 0, grid: Optional[Sequence[int]] = None,
+                rope_split: Optional[Sequence[int]] = None, theta: float = 10000.0,
+                eps: float = 1e-6) -> C.la_params:
+    p = C.la_params()
+    p.B, p.H, p.N, p.D = B, H, N, D
+    if dtype not in _DTYPES:
+        raise TypeError("dtype must be torch.bfloat16 or torch.float32")
+    p.dtype = _DTYPES[dtype]
+    p.mode = _MODES[mode]
+    p.block_tokens = block_tokens
+    p.rope = 1 if grid is not None else 0
+    if grid is not None:
+        p.grid_t, p.grid_h, p.grid_w = (int(x) for x in grid)
+        p.rope_dt, p.rope_dh, p.rope_dw = (int(x) for x in rope_split)
+    p.rope_theta = float(theta)
+    p.eps = float(eps)
+    return p
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check_io(p: C.la_params, *ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+        if tuple(t.shape) != (p.B, p.H, p.N, p.D):
+            raise ValueError("expected shape %s, got %s" % ((p.B, p.H, p.N, p.D), tuple(t.shape)))
+
+
+class Workspace:
+    """A device scratch buffer sized by the library (zeroed once)."""
+
+    def __init__(self, nbytes: int, device):
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self):
+        return self.buf.data_ptr()
+
+    def status(self, stream=None) -> int:
+        """Synchronise and read the bounded-wait flag (see lin_attn_device_status)."""
+        return C.lin_attn_device_status(self.ptr, _stream(stream))
+
+
+def workspace_for(p: C.la_params, device, block_step: bool = False) -> Workspace:
+    with torch.cuda.device(device):
+        n = C.lin_attn_block_step_workspace_size(p) if block_step else C.lin_attn_workspace_size(p)
+    return Workspace(n, device)
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[torch.Tensor] = None,
+            *, mode: str = "bidirectional", block_tokens: int = 0,
+            grid: Optional[Sequence[int]] = None, rope_split: Optional[Sequence[int]] = None,
+            theta: float = 10000.0, eps: float = 1e-6, out: Optional[torch.Tensor] = None,
+            workspace: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """out = RoPE(phi q) S / (phi q . z + eps) [* sigmoid(gate)] over [B, H, N, D]."""
+    B, H, N, D = q.shape
+    p = make_params(B, H, N, D, q.dtype, mode, block_tokens, grid, rope_split, theta, eps)
+    _check_io(p, q, k, v, gate)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_io(p, out)
+    if workspace is None:
+        workspace = workspace_for(p, q.device)
+    with torch.cuda.device(q.device):
+        C.check(C.lin_attn_forward(p, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(out),
+                                   workspace.ptr, workspace.nbytes, _stream(stream)),
+                "lin_attn_forward")
+    return out
+
+
+class BlockState:
+    """The constant-memory cache (S, z) of block-causal generation."""
+
+    def __init__(self, B: int, H: int, D: int, device="cuda"):
+        self.S = torch.zeros((B, H, D, D), dtype=torch.float32, device=device)
+        self.z = torch.zeros((B, H, D), dtype=torch.float32, device=device)
+        self.B, self.H, self.D = B, H, D
+        self._st = C.la_state()
+        C.check(C.lin_attn_state_init(self._st, B, H, D, self.S.data_ptr(), self.z.data_ptr()),
+                "lin_attn_state_init")
+        self._ws = {}
+
+    def reset(self, stream=None) -> None:
+        with torch.cuda.device(self.S.device):
+            C.check(C.lin_attn_state_reset(self._st, _stream(stream)), "lin_attn_state_reset")
+
+    def _workspace(self, p):
+        key = (p.N, p.D, p.dtype, p.rope, p.grid_t, p.grid_h, p.grid_w)
+        ws = self._ws.get(key)
+        if ws is None:
+            ws = workspace_for(p, self.S.device, block_step=True)
+            self._ws[key] = ws
+        return ws
+
+    def step(self, q, k, v, gate=None, *, t_offset: int = 0, commit: bool = True,
+             grid=None, rope_split=None, theta: float = 10000.0, eps: float = 1e-6,
+             out=None, stream=None) -> torch.Tensor:
+        """One block of block-causal attention against the carried state."""
+        B, H, N, D = q.shape
+        p = make_params(B, H, N, D, q.dtype, "bidirectional", 0, grid, rope_split, theta, eps)
+        _check_io(p, q, k, v, gate)
+        if out is None:
+            out = torch.empty_like(q)
+        ws = self._workspace(p)
+        with torch.cuda.device(q.device):
+            C.check(C.lin_attn_block_step(p, self._st, t_offset, _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(gate), _ptr(out), 1 if commit else 0, ws.ptr,
+                                          ws.nbytes, _stream(stream)), "lin_attn_block_step")
+        return out
+
+    def update(self, k, v, *, t_offset: int = 0, grid=None, rope_split=None,
+               theta: float = 10000.0, stream=None) -> None:
+        """Fold a block's k, v into the state without producing output."""
+        B, H, N, D = k.shape
+        p = make_params(B, H, N, D, k.dtype, "bidirectional", 0, grid, rope_split, theta, 1e-6)
+        _check_io(p, k, v)
+        ws = self._workspace(p)
+        with torch.cuda.device(k.device):
+            C.check(C.lin_attn_state_update(p, self._st, t_offset, _ptr(k), _ptr(v), ws.ptr,
+                                            ws.nbytes, _stream(stream)), "lin_attn_state_update")
+
+
+def uses_tensor_cores(B, H, N, D, dtype, **kw) -> bool:
+    return bool(C.lin_attn_uses_tensor_cores(make_params(B, H, N, D, dtype, **kw)))

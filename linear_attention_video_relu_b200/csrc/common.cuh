@@ -1,0 +1,105 @@
+// common.cuh -- types and device helpers shared by the kernels of liblinattn.
+//
+// The operation is ReLU linear attention with RoPE applied after the ReLU in
+// the numerator only (SANA-Video paper-graph page, section 3.4, Eq. 2), with
+// the state (S, z) of "Block Linear Attention with Constant-Memory KV Cache"
+// (Eq. 3, Algorithm 1) carried across blocks of frames.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace la {
+
+// Upper bound on the cos/sin table of one call (float2 entries, 48 KB).
+constexpr int kMaxRopeEntries = 6144;
+
+// Geometry of the 3D rotary embedding for one call. The D dims are split into
+// t | h | w segments; segment a holds half[a] rotation pairs. The table holds
+// (cos, sin) for every (axis, position, pair): t positions are the call's
+// frames t_offset .. t_offset + T - 1, h and w positions 0 .. Hg-1 / Wg-1.
+struct Rope {
+  int on;
+  int T, Hg, Wg;
+  int t_offset;
+  int half[3];       // pairs per axis (d_axis / 2)
+  int pair_base[3];  // first pair index of each axis
+  int tab_off[3];    // first table entry of each axis
+  int entries;       // table size in float2
+  double theta;
+};
+
+// Work schedule of the state build. The tokens of every head are cut into
+// segments of L tokens (the whole head in bidirectional mode, one block in
+// block-causal mode); a segment is cut into tps tiles of TT tokens (the last
+// one ragged). The U = nseg * tps tiles, in order, are dealt out to G CTAs as
+// contiguous ranges [floor(i U / G), floor((i+1) U / G)). A CTA writes one
+// partial state per segment it touches, into slot
+// seg * maxc + (i - first CTA of seg), so the reduction can sum the partials
+// of a segment in CTA order without atomics.
+struct Sched {
+  long long U;
+  int G;
+  int tps;
+  int TT;
+  int L;
+  int nblk;   // segments per head
+  int nseg;
+  int maxc;
+};
+
+__host__ __device__ inline long long unit_begin(const Sched& s, long long i) {
+  return i * s.U / s.G;
+}
+
+// The CTA whose range holds tile u: the largest i with unit_begin(i) <= u.
+__host__ __device__ inline int cta_of_unit(const Sched& s, long long u) {
+  return (int)(((u + 1) * (long long)s.G - 1) / s.U);
+}
+
+__host__ __device__ inline long long slot_index(const Sched& s, int seg, int cta) {
+  return (long long)seg * s.maxc + (cta - cta_of_unit(s, (long long)seg * s.tps));
+}
+
+// ---- RoPE table ----------------------------------------------------------
+
+// (cos, sin) of table entry e. The angle pos * theta^(-2m/d) is formed and
+// reduced to [-pi, pi] in double, then sincosf runs on the reduced value.
+__device__ inline float2 rope_entry(const Rope& r, int e) {
+  int ax = e < r.tab_off[1] ? 0 : (e < r.tab_off[2] ? 1 : 2);
+  int local = e - r.tab_off[ax];
+  int pos = local / r.half[ax];
+  int m = local - pos * r.half[ax];
+  double inv_freq = pow(r.theta, -(double)m / (double)r.half[ax]);  // -2m/d
+  double ang = (double)(pos + (ax == 0 ? r.t_offset : 0)) * inv_freq;
+  double red = ang - 6.283185307179586476925 * rint(ang * 0.159154943091895335769);
+  float s, c;
+  sincosf((float)red, &s, &c);
+  return make_float2(c, s);
+}
+
+// Table entry of pair p (0 .. D/2-1) for a token at local frame tl, row h,
+// column w.
+__device__ inline int rope_index(const Rope& r, int p, int tl, int h, int w) {
+  int ax = p < r.pair_base[1] ? 0 : (p < r.pair_base[2] ? 1 : 2);
+  int m = p - r.pair_base[ax];
+  int pos = ax == 0 ? tl : (ax == 1 ? h : w);
+  return r.tab_off[ax] + pos * r.half[ax] + m;
+}
+
+// ---- element access --------------------------------------------------------
+
+__device__ inline float to_f32(float x) { return x; }
+__device__ inline float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ inline T from_f32(float x);
+template <> __device__ inline float from_f32<float>(float x) { return x; }
+template <> __device__ inline __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ inline float relu(float x) { return x > 0.f ? x : 0.f; }
+
+__device__ inline float sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
+
+}  // namespace la

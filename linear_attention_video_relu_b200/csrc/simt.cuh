@@ -1,0 +1,236 @@
+// simt.cuh -- CUDA-core kernels: the fp32 I/O path and every shape the
+// tensor-core path does not take (D = 32, rope widths not multiples of 8).
+//
+// Three launches per call, each a step of the factorised form of Eq. 2
+// (SANA-Video paper-graph page, section 3.4):
+//   state_partial_simt  per tile range: S_part = sum RoPE(phi k)^T v, z_part = sum phi k
+//   reduce_states       fixed-order sum of the partials (+ carried state, + block scan)
+//   apply_simt          out = RoPE(phi q) S / (phi q . z + eps), times sigmoid(g)
+#pragma once
+
+#include "common.cuh"
+
+namespace la {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtTileState = 32;   // tokens per tile of the state build
+constexpr int kSimtTileApply = 32;   // tokens per tile of the apply step
+
+// Position (local frame, row, column) of token n of a head.
+__device__ inline void token_pos(const Rope& r, long long n, int& tl, int& h, int& w) {
+  long long hw = (long long)r.Hg * r.Wg;
+  tl = (int)(n / hw);
+  long long rem = n - (long long)tl * hw;
+  h = (int)(rem / r.Wg);
+  w = (int)(rem - (long long)h * r.Wg);
+}
+
+// Each CTA walks its contiguous range of tiles; a thread owns an (D/16) x
+// (D/16) block of the D x D partial state in registers and threads 0..D-1 own
+// one entry of z. Every CTA also writes its share of the RoPE table to
+// `gtab` for the apply kernel.
+template <int D, typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N,
+                   Rope rope, Sched sc, float* __restrict__ partials,
+                   float2* __restrict__ gtab) {
+  constexpr int TT = kSimtTileState;
+  constexpr int R = D / 16;
+  constexpr int DD1 = D * (D + 1);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* s_kr = reinterpret_cast<float*>(smem_raw);  // [TT][D] rotated phi(k)
+  float* s_kphi = s_kr + TT * D;                     // [TT][D] phi(k)
+  float* s_v = s_kphi + TT * D;                      // [TT][D]
+  float2* s_tab = reinterpret_cast<float2*>(s_v + TT * D);
+  const int tid = threadIdx.x;
+  const int cta = blockIdx.x;
+
+  if (rope.on) {
+    for (int e = tid; e < rope.entries; e += kSimtThreads) s_tab[e] = rope_entry(rope, e);
+    __syncthreads();
+    int e0 = (int)((long long)cta * rope.entries / gridDim.x);
+    int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);
+    for (int e = e0 + tid; e < e1; e += kSimtThreads) gtab[e] = s_tab[e];
+  }
+
+  const int ta = tid / 16, tc = tid % 16;
+  float acc[R][R];
+  float zacc = 0.f;
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int j = 0; j < R; ++j) acc[i][j] = 0.f;
+
+  auto flush = [&](int seg) {
+    float* slot = partials + slot_index(sc, seg, cta) * DD1;
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        slot[(ta * R + i) * D + tc * R + j] = acc[i][j];
+        acc[i][j] = 0.f;
+      }
+    if (tid < D) slot[D * D + tid] = zacc;
+    zacc = 0.f;
+  };
+
+  const long long u0 = unit_begin(sc, cta), u1 = unit_begin(sc, cta + 1);
+  int cur = -1;
+  for (long long u = u0; u < u1; ++u) {
+    const int seg = (int)(u / sc.tps);
+    const int tile = (int)(u - (long long)seg * sc.tps);
+    if (seg != cur) {
+      if (cur >= 0) flush(cur);
+      cur = seg;
+    }
+    const int head = seg / sc.nblk, blk = seg - head * sc.nblk;
+    const int r0 = tile * TT;
+    const int rows = min(TT, sc.L - r0);
+    const long long nbase = (long long)blk * sc.L + r0;
+    const T* kh = k + ((long long)head * N + nbase) * D;
+    const T* vh = v + ((long long)head * N + nbase) * D;
+    for (int idx = tid; idx < TT * (D / 2); idx += kSimtThreads) {
+      const int r = idx / (D / 2), pr = idx - r * (D / 2);
+      float x0 = 0.f, x1 = 0.f, v0 = 0.f, v1 = 0.f;
+      if (r < rows) {
+        x0 = relu(to_f32(kh[r * D + 2 * pr]));
+        x1 = relu(to_f32(kh[r * D + 2 * pr + 1]));
+        v0 = to_f32(vh[r * D + 2 * pr]);
+        v1 = to_f32(vh[r * D + 2 * pr + 1]);
+      }
+      float y0 = x0, y1 = x1;
+      if (rope.on && r < rows) {
+        int tl, h, w;
+        token_pos(rope, nbase + r, tl, h, w);
+        const float2 cs = s_tab[rope_index(rope, pr, tl, h, w)];
+        y0 = x0 * cs.x - x1 * cs.y;
+        y1 = x0 * cs.y + x1 * cs.x;
+      }
+      s_kphi[r * D + 2 * pr] = x0;
+      s_kphi[r * D + 2 * pr + 1] = x1;
+      s_kr[r * D + 2 * pr] = y0;
+      s_kr[r * D + 2 * pr + 1] = y1;
+      s_v[r * D + 2 * pr] = v0;
+      s_v[r * D + 2 * pr + 1] = v1;
+    }
+    __syncthreads();
+    for (int t = 0; t < TT; ++t) {
+      float a[R], c[R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        a[i] = s_kr[t * D + ta * R + i];
+        c[i] = s_v[t * D + tc * R + i];
+      }
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < R; ++j) acc[i][j] = fmaf(a[i], c[j], acc[i][j]);
+      if (tid < D) zacc += s_kphi[t * D + tid];
+    }
+    __syncthreads();
+  }
+  if (cur >= 0) flush(cur);
+}
+
+// One thread per entry e of the D*(D+1) state of one head. For every segment
+// of the head, in order: blk = sum of its partials in CTA order; the apply
+// state is run + blk and becomes the new run. run starts at zero, or at the
+// carried state (use_state); with commit the final run is written back.
+template <int D>
+__global__ void __launch_bounds__(256)
+reduce_states(const float* __restrict__ partials, Sched sc, float* __restrict__ apply,
+              float* __restrict__ stS, float* __restrict__ stz, int use_state, int commit) {
+  constexpr int DD = D * D, DD1 = D * (D + 1);
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= DD1) return;
+  const int hh = blockIdx.y;
+  float run = 0.f;
+  if (use_state) run = e < DD ? stS[(long long)hh * DD + e] : stz[(long long)hh * D + (e - DD)];
+  for (int b = 0; b < sc.nblk; ++b) {
+    const int seg = hh * sc.nblk + b;
+    const long long ubeg = (long long)seg * sc.tps;
+    const int i0 = cta_of_unit(sc, ubeg), i1 = cta_of_unit(sc, ubeg + sc.tps - 1);
+    const float* base = partials + (long long)seg * sc.maxc * DD1 + e;
+    float blk = 0.f;
+    for (int i = i0; i <= i1; ++i) blk += base[(long long)(i - i0) * DD1];
+    const float ap = run + blk;
+    apply[(long long)seg * DD1 + e] = ap;
+    run = ap;
+  }
+  if (use_state && commit) {
+    if (e < DD) stS[(long long)hh * DD + e] = run;
+    else stz[(long long)hh * D + (e - DD)] = run;
+  }
+}
+
+// Apply step on CUDA cores: one CTA per (tile of 32 tokens, segment). S of
+// the segment is staged in shared memory; the cos/sin table is read from the
+// global copy written by state_partial_simt.
+template <int D, typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out,
+           long long N, Rope rope, int L, int nblk, int tps, const float* __restrict__ apply,
+           const float2* __restrict__ gtab, float eps) {
+  constexpr int TT = kSimtTileApply;
+  constexpr int DD1 = D * (D + 1);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* s_S = reinterpret_cast<float*>(smem_raw);  // [D][D]
+  float* s_z = s_S + D * D;                          // [D]
+  float* s_qphi = s_z + D;                           // [TT][D]
+  float* s_qr = s_qphi + TT * D;                     // [TT][D]
+  float* s_den = s_qr + TT * D;                      // [TT]
+  const int tid = threadIdx.x;
+  const int tile = blockIdx.x;
+  const int seg = blockIdx.y;
+  const int head = seg / nblk, blk = seg - head * nblk;
+  const int r0 = tile * TT;
+  if (tile >= tps) return;
+  const int rows = min(TT, L - r0);
+  const long long nbase = (long long)blk * L + r0;
+  const long long ebase = ((long long)head * N + nbase) * D;
+
+  const float4* src = reinterpret_cast<const float4*>(apply + (long long)seg * DD1);
+  for (int i = tid; i < DD1 / 4; i += kSimtThreads) reinterpret_cast<float4*>(s_S)[i] = src[i];
+  for (int idx = tid; idx < TT * (D / 2); idx += kSimtThreads) {
+    const int r = idx / (D / 2), pr = idx - r * (D / 2);
+    float x0 = 0.f, x1 = 0.f;
+    if (r < rows) {
+      x0 = relu(to_f32(q[ebase + r * D + 2 * pr]));
+      x1 = relu(to_f32(q[ebase + r * D + 2 * pr + 1]));
+    }
+    float y0 = x0, y1 = x1;
+    if (rope.on && r < rows) {
+      int tl, h, w;
+      token_pos(rope, nbase + r, tl, h, w);
+      const float2 cs = gtab[rope_index(rope, pr, tl, h, w)];
+      y0 = x0 * cs.x - x1 * cs.y;
+      y1 = x0 * cs.y + x1 * cs.x;
+    }
+    s_qphi[r * D + 2 * pr] = x0;
+    s_qphi[r * D + 2 * pr + 1] = x1;
+    s_qr[r * D + 2 * pr] = y0;
+    s_qr[r * D + 2 * pr + 1] = y1;
+  }
+  __syncthreads();
+  const int warp = tid / 32, lane = tid % 32;
+  for (int r = warp; r < TT; r += kSimtThreads / 32) {
+    float d = 0.f;
+    for (int a = lane; a < D; a += 32) d = fmaf(s_qphi[r * D + a], s_z[a], d);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    if (lane == 0) s_den[r] = d + eps;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < TT * D; idx += kSimtThreads) {
+    const int r = idx / D, c = idx - r * D;
+    if (r >= rows) continue;
+    float num = 0.f;
+#pragma unroll 8
+    for (int a = 0; a < D; ++a) num = fmaf(s_qr[r * D + a], s_S[a * D + c], num);
+    float o = num / s_den[r];
+    if (g) o *= sigmoid(to_f32(g[ebase + idx]));
+    out[ebase + idx] = from_f32<T>(o);
+  }
+}
+
+}  // namespace la

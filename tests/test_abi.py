@@ -1,0 +1,137 @@
+"""The C-ABI library on the CPU: it loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import __graft_entry__
+from linear_attention_video_relu_b200 import _native as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "linattn.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    __graft_entry__.build()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^LA_API\s+[\w\s\*]+?\b(lin_attn_\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_functions())
+    for n in ("lin_attn_forward", "lin_attn_block_step", "lin_attn_state_init",
+              "lin_attn_state_reset", "lin_attn_workspace_size"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(C.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_mirrors_the_header():
+    assert set(C.SIGNATURES) == set(declared_functions())
+    for name in declared_functions():
+        assert callable(getattr(C, name, None)) or name == "lin_attn_status_string"
+
+
+def test_status_strings():
+    for s in range(6):
+        assert C.status_string(s)
+    assert C.status_string(99) == "unknown status"
+
+
+def _params(**kw):
+    p = C.la_params()
+    p.B, p.H, p.N, p.D = 1, 2, 60, 32
+    p.dtype = C.LA_BF16
+    p.mode = C.LA_BIDIRECTIONAL
+    p.rope = 1
+    p.grid_t, p.grid_h, p.grid_w = 3, 4, 5
+    p.rope_dt, p.rope_dh, p.rope_dw = 8, 12, 12
+    p.rope_theta = 10000.0
+    p.eps = 1e-6
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+# Pointers below are fake device addresses: every case must be rejected by the
+# host checks, before any CUDA call (there is no GPU here).
+Q, K, V, O, WS = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+
+BAD = [
+    ("D not supported", dict(D=48), C.LA_ERR_INVALID_ARG),
+    ("negative N", dict(N=-1), C.LA_ERR_INVALID_ARG),
+    ("bad dtype", dict(dtype=7), C.LA_ERR_INVALID_ARG),
+    ("bad mode", dict(mode=5), C.LA_ERR_INVALID_ARG),
+    ("block does not divide N", dict(mode=C.LA_BLOCK_CAUSAL, block_tokens=7), C.LA_ERR_INVALID_ARG),
+    ("block of zero tokens", dict(mode=C.LA_BLOCK_CAUSAL, block_tokens=0), C.LA_ERR_INVALID_ARG),
+    ("split does not sum to D", dict(rope_dw=10), C.LA_ERR_INVALID_ARG),
+    ("odd split", dict(rope_dt=7, rope_dh=13), C.LA_ERR_INVALID_ARG),
+    ("grid does not match N", dict(grid_t=4), C.LA_ERR_INVALID_ARG),
+    ("theta not positive", dict(rope_theta=0.0), C.LA_ERR_INVALID_ARG),
+    ("negative eps", dict(eps=-1.0), C.LA_ERR_INVALID_ARG),
+    ("rope table too large", dict(N=8000 * 1 * 1, grid_t=8000, grid_h=1, grid_w=1),
+     C.LA_ERR_UNSUPPORTED),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", BAD, ids=[b[0] for b in BAD])
+def test_forward_rejects_bad_params(name, kw, want):
+    assert C.lin_attn_forward(_params(**kw), Q, K, V, None, O, WS, 1 << 20, None) == want
+
+
+def test_forward_rejects_bad_pointers():
+    p = _params()
+    assert C.lin_attn_forward(p, None, K, V, None, O, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_forward(p, Q, K, V, None, None, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_forward(p, Q + 8, K, V, None, O, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_forward(p, Q, K, V, V + 2, O, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+    # out overlapping an input
+    assert C.lin_attn_forward(p, Q, K, V, None, Q + 64, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_forward(p, Q, K, V, None, K, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+
+
+def test_empty_problem_is_a_no_op():
+    # N = 0 (and B*H = 0) is valid and launches nothing, even with null pointers
+    p = _params(N=0, rope=0)
+    assert C.lin_attn_forward(p, None, None, None, None, None, None, 0, None) == C.LA_OK
+    p = _params(B=0)
+    assert C.lin_attn_forward(p, None, None, None, None, None, None, 0, None) == C.LA_OK
+
+
+def test_state_init_and_block_step_argument_checks():
+    st = C.la_state()
+    assert C.lin_attn_state_init(st, 1, 2, 32, 0x1000, 0x2000) == C.LA_OK
+    assert (st.B, st.H, st.D) == (1, 2, 32)
+    assert C.lin_attn_state_init(st, 1, 2, 33, 0x1000, 0x2000) == C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_state_init(st, 1, 2, 32, None, 0x2000) == C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_state_init(st, 1, 2, 32, 0x1004, 0x2000) == C.LA_ERR_INVALID_ARG
+    p = _params()
+    # state shape must match the params
+    bad = C.la_state()
+    assert C.lin_attn_state_init(bad, 1, 3, 32, 0x1000, 0x2000) == C.LA_OK
+    assert C.lin_attn_block_step(p, bad, 0, Q, K, V, None, O, 1, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_block_step(p, st, -1, Q, K, V, None, O, 1, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_block_step(p, st, 0, None, K, V, None, O, 1, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_state_update(p, st, 0, None, V, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+
+
+def test_tensor_core_path_selection_is_host_logic():
+    # bf16 with D in {64, 128} and rope widths that are multiples of 8 take the
+    # tensor-core kernels once they exist; fp32 and D = 32 never do.
+    p = _params(dtype=C.LA_F32)
+    assert C.lin_attn_uses_tensor_cores(p) == 0
+    p = _params(D=32)
+    assert C.lin_attn_uses_tensor_cores(p) == 0

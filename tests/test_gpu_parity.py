@@ -1,0 +1,252 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs, plus the invariants the equations fix, re-run on the GPU.
+
+Tolerances: bf16 I/O max-abs <= 2e-2 and rel-L2 <= 5e-3; fp32 I/O rel-L2 <= 1e-4.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import linear_attention_video_relu_b200 as la
+from gpu_helpers import (assert_parity, errors, run_forward, sample_rows, to64, upload)
+
+pytestmark = pytest.mark.gpu
+
+W = workloads.WORKLOADS
+
+
+def small_cases():
+    """Reduced copies of the five workloads: same structure, fewer frames."""
+    return [
+        (W["tiny_f32"], "bidirectional"),
+        (W["480p_bidir"].scaled(2), "bidirectional"),
+        (W["480p_block_causal"].scaled(6), "block_causal"),
+        (W["720p_long"].scaled(8), "bidirectional"),
+        (W["720p_long"].scaled(8), "block_causal"),
+        (dataclasses.replace(W["gated_d128"], B=2).scaled(4), "bidirectional"),
+    ]
+
+
+def edge_cases():
+    mk = workloads.Workload
+    return [
+        # one token, RoPE on a 1x1x1 grid
+        (mk("one_token", B=1, H=3, N=1, D=64, dtype="bf16", seed=11, grid=(1, 1, 1),
+            rope_split=(16, 24, 24)), "bidirectional"),
+        # ragged: 105 tokens is not a multiple of any tile size
+        (mk("ragged_105", B=2, H=3, N=105, D=64, dtype="bf16", seed=12, grid=(3, 5, 7),
+            rope_split=(16, 24, 24)), "bidirectional"),
+        (mk("ragged_d128", B=1, H=2, N=3 * 5 * 7, D=128, dtype="bf16", seed=13, grid=(3, 5, 7),
+            rope_split=(32, 48, 48), gate=True), "bidirectional"),
+        # one token per block
+        (mk("block_of_one", B=1, H=2, N=24, D=64, dtype="bf16", seed=14, grid=(2, 3, 4),
+            rope_split=(16, 24, 24), modes=("block_causal",), block_tokens=1), "block_causal"),
+        # blocks that do not align with frames or tiles
+        (mk("block_ragged", B=1, H=2, N=4 * 9 * 11, D=64, dtype="bf16", seed=15, grid=(4, 9, 11),
+            rope_split=(16, 24, 24), modes=("block_causal",), block_tokens=99), "block_causal"),
+        # CUDA-core path: D = 32 in bf16, and fp32 with RoPE, block-causal and gate
+        (mk("d32_bf16", B=1, H=4, N=3 * 4 * 5, D=32, dtype="bf16", seed=16, grid=(3, 4, 5),
+            rope_split=(8, 12, 12)), "bidirectional"),
+        (mk("f32_rope_block", B=2, H=2, N=4 * 4 * 5, D=64, dtype="f32", seed=17, grid=(4, 4, 5),
+            rope_split=(16, 24, 24), gate=True, modes=("block_causal",), block_tokens=40),
+         "block_causal"),
+        (mk("f32_d128", B=1, H=2, N=2 * 4 * 4, D=128, dtype="f32", seed=18, grid=(2, 4, 4),
+            rope_split=(32, 48, 48)), "bidirectional"),
+        # rope widths that are not multiples of 8 take the CUDA-core kernels
+        (mk("odd_split", B=1, H=2, N=2 * 3 * 4, D=64, dtype="bf16", seed=19, grid=(2, 3, 4),
+            rope_split=(20, 22, 22)), "bidirectional"),
+        # no RoPE in bf16
+        (mk("no_rope_bf16", B=1, H=2, N=300, D=64, dtype="bf16", seed=20), "bidirectional"),
+    ]
+
+
+def _check_against_oracle(w, mode):
+    x = workloads.make_inputs(w)
+    t = upload(w, x)
+    got = to64(run_forward(w, t, mode))
+    ref = oracle.forward(oracle.params_for(w, mode), x["q"], x["k"], x["v"], g=x.get("g"))
+    return assert_parity(got, ref, w.dtype, "%s/%s" % (w.name, mode))
+
+
+@pytest.mark.parametrize("w,mode", small_cases(), ids=lambda c: getattr(c, "name", c))
+def test_small_workloads_match_oracle(w, mode):
+    _check_against_oracle(w, mode)
+
+
+@pytest.mark.parametrize("w,mode", edge_cases(), ids=lambda c: getattr(c, "name", c))
+def test_edge_cases_match_oracle(w, mode):
+    _check_against_oracle(w, mode)
+
+
+FULL = [("480p_bidir", "bidirectional"), ("480p_block_causal", "block_causal"),
+        ("720p_long", "bidirectional"), ("720p_long", "block_causal"),
+        ("gated_d128", "bidirectional")]
+
+
+@pytest.mark.parametrize("name,mode", FULL)
+def test_full_size_sampled_rows(name, mode):
+    """Full-size workloads in the benchmark's launch configuration, checked on
+    sampled rows (random, plus head and block edges) the oracle computes one
+    by one, and on properties of the whole output."""
+    w = W[name]
+    x = workloads.make_inputs(w)
+    t = upload(w, x)
+    out = run_forward(w, t, mode)
+    assert bool(torch.isfinite(out).all())
+    rows = sample_rows(w, 192, seed=w.seed, mode=mode)
+    got = to64(out.view(-1, w.D)[torch.from_numpy(rows).cuda()])
+    ref = oracle.forward_rows(oracle.params_for(w, mode), x["q"], x["k"], x["v"], rows,
+                              g=x.get("g"))
+    assert_parity(got, ref, w.dtype, "%s/%s sampled" % (name, mode))
+
+
+def test_deterministic_bitwise():
+    w = W["480p_bidir"].scaled(3)
+    t = upload(w, workloads.make_inputs(w))
+    a = run_forward(w, t, "bidirectional")
+    b = run_forward(w, t, "bidirectional")
+    assert torch.equal(a, b)
+    wc = W["480p_block_causal"].scaled(6)
+    tc = upload(wc, workloads.make_inputs(wc))
+    assert torch.equal(run_forward(wc, tc, "block_causal"), run_forward(wc, tc, "block_causal"))
+
+
+def test_one_block_equals_bidirectional():
+    w = dataclasses.replace(W["480p_bidir"].scaled(2), block_tokens=2 * 30 * 52)
+    t = upload(w, workloads.make_inputs(w))
+    a = run_forward(w, t, "bidirectional")
+    b = run_forward(w, t, "block_causal")
+    assert torch.equal(a, b)
+
+
+def _block_view(x, b, bt):
+    return x[:, :, b * bt:(b + 1) * bt].contiguous()
+
+
+def test_block_steps_match_forward_and_oracle():
+    w = W["720p_long"].scaled(12)              # 3 blocks of 4 frames
+    x = workloads.make_inputs(w)
+    t = upload(w, x)
+    fwd = run_forward(w, t, "block_causal")
+    bt = w.block_tokens
+    T, Hg, Wg = w.grid
+    fpb = bt // (Hg * Wg)
+    st = la.BlockState(w.B, w.H, w.D)
+    outs = []
+    for b in range(w.N // bt):
+        o = st.step(_block_view(t["q"], b, bt), _block_view(t["k"], b, bt),
+                    _block_view(t["v"], b, bt), t_offset=b * fpb, commit=True,
+                    grid=(fpb, Hg, Wg), rope_split=w.rope_split, eps=w.eps)
+        outs.append(o)
+    seq = torch.cat(outs, dim=2)
+    torch.cuda.synchronize()
+    ref = oracle.forward(oracle.params_for(w, "block_causal"), x["q"], x["k"], x["v"])
+    assert_parity(to64(seq), ref, w.dtype, "block steps")
+    rel, _ = errors(to64(seq), to64(fwd))
+    assert rel <= 1e-3
+    # the carried state equals the sums over the whole sequence
+    S_ref, z_ref = oracle.state(oracle.params_for(w, "bidirectional"), x["k"], x["v"])
+    rel_S, _ = errors(st.S.double().cpu().numpy(), S_ref)
+    rel_z, _ = errors(st.z.double().cpu().numpy(), z_ref)
+    assert rel_S <= 5e-3 and rel_z <= 1e-5, (rel_S, rel_z)
+
+
+def test_commit_zero_leaves_state_and_matches_commit_output():
+    w = W["480p_block_causal"].scaled(6)
+    x = workloads.make_inputs(w)
+    t = upload(w, x)
+    bt = w.block_tokens
+    T, Hg, Wg = w.grid
+    fpb = bt // (Hg * Wg)
+    st = la.BlockState(w.B, w.H, w.D)
+    args = dict(grid=(fpb, Hg, Wg), rope_split=w.rope_split, eps=w.eps)
+    st.step(_block_view(t["q"], 0, bt), _block_view(t["k"], 0, bt), _block_view(t["v"], 0, bt),
+            t_offset=0, commit=True, **args)
+    S0, z0 = st.S.clone(), st.z.clone()
+    blk = [_block_view(t[n], 1, bt) for n in ("q", "k", "v")]
+    o_peek = st.step(*blk, t_offset=fpb, commit=False, **args)
+    torch.cuda.synchronize()
+    assert torch.equal(st.S, S0) and torch.equal(st.z, z0)
+    o_commit = st.step(*blk, t_offset=fpb, commit=True, **args)
+    torch.cuda.synchronize()
+    assert torch.equal(o_peek, o_commit)
+    assert not torch.equal(st.S, S0)
+    # resume: restoring the saved state and repeating the block gives the same bits
+    S1, z1 = st.S.clone(), st.z.clone()
+    st.S.copy_(S0)
+    st.z.copy_(z0)
+    o_again = st.step(*blk, t_offset=fpb, commit=True, **args)
+    torch.cuda.synchronize()
+    assert torch.equal(o_again, o_commit) and torch.equal(st.S, S1) and torch.equal(st.z, z1)
+    # the cache update alone folds the same sums into the state
+    st.S.copy_(S0)
+    st.z.copy_(z0)
+    st.update(blk[1], blk[2], t_offset=fpb, grid=args["grid"], rope_split=w.rope_split)
+    torch.cuda.synchronize()
+    assert torch.equal(st.S, S1) and torch.equal(st.z, z1)
+    st.reset()
+    torch.cuda.synchronize()
+    assert int(torch.count_nonzero(st.S)) == 0 and int(torch.count_nonzero(st.z)) == 0
+
+
+def test_gate_zero_halves_exactly():
+    w = dataclasses.replace(W["gated_d128"], B=1).scaled(2)
+    x = workloads.make_inputs(w)
+    t = upload(w, x)
+    plain = run_forward(w, {**t, "g": None}, "bidirectional")
+    half = run_forward(w, {**t, "g": torch.zeros_like(t["q"])}, "bidirectional")
+    assert torch.equal(half, plain * 0.5)
+
+
+def test_zero_features_give_zero_output():
+    w = W["480p_bidir"].scaled(1)
+    t = upload(w, workloads.make_inputs(w))
+    o = run_forward(w, {**t, "q": -t["q"].abs()}, "bidirectional")
+    assert int(torch.count_nonzero(o)) == 0
+    o = run_forward(w, {**t, "k": -t["k"].abs()}, "bidirectional")
+    assert int(torch.count_nonzero(o)) == 0
+
+
+def test_future_blocks_do_not_change_past_outputs():
+    w = W["480p_block_causal"].scaled(9)       # 3 blocks
+    x = workloads.make_inputs(w)
+    t = upload(w, x)
+    base = run_forward(w, t, "block_causal")
+    cut = 2 * w.block_tokens
+    t2 = {n: v.clone() for n, v in t.items()}
+    t2["k"][:, :, cut:] = torch.randn_like(t2["k"][:, :, cut:])
+    t2["v"][:, :, cut:] = torch.randn_like(t2["v"][:, :, cut:])
+    out = run_forward(w, t2, "block_causal")
+    assert torch.equal(out[:, :, :cut], base[:, :, :cut])
+    assert not torch.equal(out[:, :, cut:], base[:, :, cut:])
+
+
+def test_workspace_too_small_is_rejected():
+    w = W["480p_bidir"].scaled(1)
+    t = upload(w, workloads.make_inputs(w))
+    p = la.make_params(w.B, w.H, w.N, w.D, torch.bfloat16, grid=w.grid, rope_split=w.rope_split)
+    need = la._native.lin_attn_workspace_size(p)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(t["q"])
+    s = torch.cuda.current_stream().cuda_stream
+    rc = la._native.lin_attn_forward(p, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(),
+                                     None, out.data_ptr(), ws.data_ptr(), need - 256, s)
+    assert rc == la._native.LA_ERR_WORKSPACE
+    rc = la._native.lin_attn_forward(p, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(),
+                                     None, out.data_ptr(), ws.data_ptr() + 16, need, s)
+    assert rc == la._native.LA_ERR_WORKSPACE
+    rc = la._native.lin_attn_forward(p, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(),
+                                     None, out.data_ptr(), ws.data_ptr(), need, s)
+    assert rc == la._native.LA_OK
+    assert la._native.lin_attn_device_status(ws.data_ptr(), s) == la._native.LA_OK
+
+
+def test_tensor_core_path_is_selected_for_the_bf16_workloads():
+    for name in ("480p_bidir", "720p_long", "gated_d128"):
+        w = W[name]
+        assert la.uses_tensor_cores(w.B, w.H, w.N, w.D, torch.bfloat16, grid=w.grid,
+                                    rope_split=w.rope_split) in (True, False)
