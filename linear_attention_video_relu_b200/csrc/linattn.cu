@@ -219,7 +219,7 @@ la_status run_simt(const Launch& L) {
       static_cast<const T*>(L.k), static_cast<const T*>(L.v), N, pl.rope, pl.sc, part, gtab);
   if ((st = last_error()) != LA_OK) return st;
   if ((st = mark(L, 1)) != LA_OK) return st;
-  dim3 g2((D * (D + 1) + 255) / 256, (unsigned)pl.heads);
+  dim3 g2((D * (D + 1) + 255) / 256, (unsigned)(pl.heads < 65535 ? pl.heads : 65535));
   reduce_states<D><<<g2, 256, 0, L.stream>>>(part, pl.sc, apply, L.stS, L.stz, L.use_state,
                                               L.commit);
   if ((st = last_error()) != LA_OK) return st;
@@ -229,10 +229,10 @@ la_status run_simt(const Launch& L) {
   size_t smem3 = ((size_t)D * (D + 1) + 2 * (size_t)TA * D + TA) * sizeof(float);
   st = set_smem(apply_simt<D, T>, smem3);
   if (st != LA_OK) return st;
-  dim3 g3(pl.apply_tps, pl.sc.nseg);
+  dim3 g3(pl.apply_tps, pl.sc.nseg < 65535 ? pl.sc.nseg : 65535);
   apply_simt<D, T><<<g3, kSimtThreads, smem3, L.stream>>>(
       static_cast<const T*>(L.q), static_cast<const T*>(L.g), static_cast<T*>(L.out), N,
-      pl.rope, pl.sc.L, pl.sc.nblk, pl.apply_tps, apply, gtab, L.p->eps);
+      pl.rope, pl.sc.L, pl.sc.nblk, pl.apply_tps, pl.sc.nseg, apply, gtab, L.p->eps);
   if ((st = last_error()) != LA_OK) return st;
   return mark(L, 3);
 }

@@ -143,7 +143,8 @@ reduce_states(const float* __restrict__ partials, Sched sc, float* __restrict__ 
   constexpr int DD = D * D, DD1 = D * (D + 1);
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= DD1) return;
-  const int hh = blockIdx.y;
+  const int heads = sc.nseg / sc.nblk;
+  for (int hh = blockIdx.y; hh < heads; hh += gridDim.y) {
   float run = 0.f;
   if (use_state) run = e < DD ? stS[(long long)hh * DD + e] : stz[(long long)hh * D + (e - DD)];
   for (int b = 0; b < sc.nblk; ++b) {
@@ -161,6 +162,7 @@ reduce_states(const float* __restrict__ partials, Sched sc, float* __restrict__ 
     if (e < DD) stS[(long long)hh * DD + e] = run;
     else stz[(long long)hh * D + (e - DD)] = run;
   }
+  }
 }
 
 // Apply step on CUDA cores: one CTA per (tile of 32 tokens, segment). S of
@@ -169,7 +171,8 @@ reduce_states(const float* __restrict__ partials, Sched sc, float* __restrict__ 
 template <int D, typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out,
-           long long N, Rope rope, int L, int nblk, int tps, const float* __restrict__ apply,
+           long long N, Rope rope, int L, int nblk, int tps, int nseg,
+           const float* __restrict__ apply,
            const float2* __restrict__ gtab, float eps) {
   constexpr int TT = kSimtTileApply;
   constexpr int DD1 = D * (D + 1);
@@ -181,10 +184,10 @@ apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out
   float* s_den = s_qr + TT * D;                      // [TT]
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
-  const int seg = blockIdx.y;
+  if (tile >= tps) return;
+  for (int seg = blockIdx.y; seg < nseg; seg += gridDim.y) {
   const int head = seg / nblk, blk = seg - head * nblk;
   const int r0 = tile * TT;
-  if (tile >= tps) return;
   const int rows = min(TT, L - r0);
   const long long nbase = (long long)blk * L + r0;
   const long long ebase = ((long long)head * N + nbase) * D;
@@ -230,6 +233,8 @@ apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out
     float o = num / s_den[r];
     if (g) o *= sigmoid(to_f32(g[ebase + idx]));
     out[ebase + idx] = from_f32<T>(o);
+  }
+  __syncthreads();
   }
 }
 
