@@ -130,6 +130,36 @@ LA_API la_status lin_attn_forward_timed(const la_params* p, const void* q, const
                                         void* workspace, size_t workspace_bytes, void* stream,
                                         void* const* events);
 
+/* Size of the fixed scratch area that lin_attn_forward_noalloc uses. */
+#define LA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* lin_attn_forward for callers that cannot allocate device memory for a
+ * workspace -- for example a plugin inside a host engine that owns all device
+ * memory through a pre-planned arena and forbids extra allocations, or a
+ * real-time generation loop that must never call cudaMalloc (which can
+ * synchronise the device). The paper has no counterpart: this is a packaging
+ * choice of the library, not a step of the method.
+ *
+ * Instead of a caller workspace it uses one file-scope device array of
+ * LA_NOALLOC_SCRATCH_BYTES (32 MiB) inside the library. Every GPU on which the
+ * library is loaded holds that array until the process exits. The call itself
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - Set-up: the first call on a device (with that device current) looks up
+ *     the array's device address once; make that first call before any stream
+ *     capture.
+ *   - Limit: a problem whose workspace (lin_attn_workspace_size) exceeds
+ *     LA_NOALLOC_SCRATCH_BYTES is rejected with LA_ERR_WORKSPACE before any
+ *     launch.
+ *   - Sharing: all calls on a device share the one array, and it keeps the
+ *     last call's contents (the call clears what must start at zero). Calls
+ *     that overlap on the GPU -- on different streams, or from different host
+ *     threads without ordering -- race on it and give wrong results; order them
+ *     on one stream.
+ * Arguments and results are those of lin_attn_forward without the workspace. */
+LA_API la_status lin_attn_forward_noalloc(const la_params* p, const void* q, const void* k,
+                                          const void* v, const void* gate, void* out,
+                                          void* stream);
+
 /* Wrap caller-owned state buffers (no allocation, no launch). S and z must
  * be device pointers, 16-byte aligned, of [B,H,D,D] and [B,H,D] floats. */
 LA_API la_status lin_attn_state_init(la_state* st, int B, int H, int D, float* S, float* z);

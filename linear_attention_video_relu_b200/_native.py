@@ -51,6 +51,7 @@ SIGNATURES = {
     "lin_attn_forward": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, ctypes.c_size_t, _V]),
     "lin_attn_forward_timed": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, ctypes.c_size_t, _V,
                                               ctypes.POINTER(ctypes.c_void_p)]),
+    "lin_attn_forward_noalloc": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
     "lin_attn_state_init": (ctypes.c_int, [_ST, ctypes.c_int, ctypes.c_int, ctypes.c_int, _V, _V]),
     "lin_attn_state_reset": (ctypes.c_int, [_ST, _V]),
     "lin_attn_block_step": (ctypes.c_int, [_P, _ST, ctypes.c_int, _V, _V, _V, _V, _V, ctypes.c_int,
@@ -121,6 +122,10 @@ def lin_attn_forward_timed(p, q, k, v, gate, out, workspace, workspace_bytes, st
         ev = (ctypes.c_void_p * 4)(*events)
     return load().lin_attn_forward_timed(ctypes.byref(p), q, k, v, gate, out, workspace,
                                          workspace_bytes, stream, ev)
+
+
+def lin_attn_forward_noalloc(p, q, k, v, gate, out, stream) -> int:
+    return load().lin_attn_forward_noalloc(ctypes.byref(p), q, k, v, gate, out, stream)
 
 
 def lin_attn_state_init(st: la_state, B, H, D, S, z) -> int:

@@ -14,6 +14,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "simt.cuh"
 #include "tc.cuh"
@@ -330,6 +332,34 @@ la_status block_common(const la_params* p, la_state* st, int t_offset, const voi
   return run(L);
 }
 
+// ---- fixed scratch for lin_attn_forward_noalloc ----------------------------
+//
+// The one device array behind lin_attn_forward_noalloc. In host code its name
+// is only a stand-in for the symbol: the device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_noalloc_once[kMaxDevices];
+void* g_noalloc_ptr[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices];
+
+la_status noalloc_scratch(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
+  std::call_once(g_noalloc_once[dev], [dev] {
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+    if (g_noalloc_err[dev] != cudaSuccess) cudaGetLastError();
+  });
+  if (g_noalloc_err[dev] != cudaSuccess || !g_noalloc_ptr[dev]) return LA_ERR_CUDA;
+  *ptr = g_noalloc_ptr[dev];
+  return LA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -371,6 +401,30 @@ la_status lin_attn_forward_timed(const la_params* p, const void* q, const void* 
   if ((s = check_workspace(pl, workspace, workspace_bytes)) != LA_OK) return s;
   Launch L{p, &pl, q, k, v, gate, out, static_cast<unsigned char*>(workspace), nullptr, nullptr,
            0, 0, 1, static_cast<cudaStream_t>(stream), events};
+  return run(L);
+}
+
+la_status lin_attn_forward_noalloc(const la_params* p, const void* q, const void* k,
+                                   const void* v, const void* gate, void* out, void* stream) {
+  la_status s = check_params(p, false);
+  if (s != LA_OK) return s;
+  if ((long long)p->B * p->H * p->N == 0) return LA_OK;
+  if ((s = check_io(p, q, k, v, gate, out, true)) != LA_OK) return s;
+  Plan pl;
+  if ((s = make_plan(p, false, 0, &pl)) != LA_OK) return s;
+  if (pl.total > (size_t)LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != LA_OK) return s;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // the bounded-wait flag word must start at zero; everything else the
+  // kernels read is written earlier in the same call
+  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + pl.off_flag, 0, sizeof(int), cs) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  Launch L{p, &pl, q, k, v, gate, out, static_cast<unsigned char*>(scratch), nullptr, nullptr,
+           0, 0, 1, cs, nullptr};
   return run(L);
 }
 
