@@ -34,6 +34,7 @@ struct Plan {
   Sched sc;
   long long heads;
   int apply_tps;       // SIMT apply: tiles per segment
+  int sms;             // SM count of the device
   size_t off_flag, off_tab, off_part, off_apply, total;
 };
 
@@ -86,7 +87,11 @@ la_status check_params(const la_params* p, bool one_block) {
 }
 
 bool want_tc(const la_params* p) {
-  return tc_supported(p->dtype == LA_BF16, p->D, p->rope, p->rope_dt, p->rope_dh, p->rope_dw);
+  const int entries = p->rope ? p->grid_t * (p->rope_dt / 2) + p->grid_h * (p->rope_dh / 2) +
+                                    p->grid_w * (p->rope_dw / 2)
+                              : 0;
+  return tc_supported(p->dtype == LA_BF16, p->D, p->rope, p->rope_dt, p->rope_dh, p->rope_dw,
+                      entries);
 }
 
 // Plan for a call of p (one_block: the N tokens are a single block of a
@@ -99,6 +104,7 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   if (st != LA_OK) return st;
   memset(pl, 0, sizeof(*pl));
   pl->tc = want_tc(p);
+  pl->sms = sms;
   pl->heads = (long long)p->B * p->H;
 
   Rope& r = pl->rope;
@@ -274,7 +280,7 @@ la_status run(const Launch& L) {
     a.eps = L.p->eps;
     a.stream = L.stream;
     a.events = L.events;
-    return tc_run(a);
+    return tc_run(a, L.pl->sms);
   }
   if (L.p->dtype == LA_BF16) return dispatch_simt<__nv_bfloat16>(L);
   return dispatch_simt<float>(L);

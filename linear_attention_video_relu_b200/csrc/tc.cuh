@@ -1,10 +1,42 @@
-// tc.cuh -- tensor-core (tcgen05 + TMA) kernels for bf16 I/O.
+// tc.cuh -- tensor-core kernels (tcgen05 MMA, TMEM accumulators, TMA tiles)
+// for bf16 I/O with D in {64, 128}.
+//
+// state_build_tc: per CTA a contiguous range of token tiles. TMA brings the k
+//   and v tiles (128-byte swizzle) into a ring of stages; four warps apply
+//   phi = ReLU and the 3D RoPE to the k tile in place and sum phi(k) for z;
+//   one thread issues tcgen05.mma with A = RoPE(phi k)^T (MN-major) and
+//   B = v (MN-major) into an fp32 TMEM accumulator, one per segment (double
+//   buffered); the four warps copy the finished accumulator and z to the
+//   CTA's partial slot. Eq. 2's numerator state and denominator sum.
+// apply_tc: per CTA a contiguous range of 128-token tiles. TMA brings q (and
+//   the gate logits); four warps form phi(q) . z + eps and RoPE(phi q) in
+//   place; one thread issues A = RoPE(phi q) (K-major) x B = S (K-major, as
+//   bf16 hi + lo so S keeps ~16 bits) into TMEM; the same warps divide by the
+//   denominator, apply the gate, round to bf16 and TMA-store the tile (rows
+//   past the segment are clipped by the tensor map).
+//
+// (SANA-Video paper-graph page, section 3.4: the unnumbered ReLU linear
+// attention equation and Eq. 2.) No wait here is unbounded: every mbarrier
+// wait gives up after kWaitLimitNs, records the failure in the workspace flag
+// and makes the CTA drain its in-flight copies and MMAs and exit.
 #pragma once
+
+#include <cuda.h>
+#include <mutex>
 
 #include "common.cuh"
 #include "linattn.h"
+#include "ptx.cuh"
+#include "simt.cuh"
 
 namespace la {
+
+constexpr int kTcThreads = 192;         // warp 0 TMA, warp 1 MMA, warps 2-5 math
+constexpr int kTcMath = 128;            // threads of the math warps
+constexpr int kSmemBudget = 227 * 1024; // dynamic shared memory per CTA on sm_100
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+enum : int { kFlagStateTimeout = 1, kFlagApplyTimeout = 2 };
 
 struct TcArgs {
   int D;
@@ -26,12 +58,817 @@ struct TcArgs {
   void* const* events;
 };
 
-inline bool tc_supported(bool bf16, int D, int rope, int dt, int dh, int dw) {
-  (void)bf16; (void)D; (void)rope; (void)dt; (void)dh; (void)dw;
-  return false;
-}
-inline int tc_state_tile(int D) { return D == 128 ? 64 : 128; }
+__host__ __device__ constexpr int tc_state_tile_c(int D) { return D == 128 ? 64 : 128; }
+inline int tc_state_tile(int D) { return tc_state_tile_c(D); }
 inline int tc_state_ctas_per_sm(int) { return 1; }
-inline la_status tc_run(const TcArgs&) { return LA_ERR_UNSUPPORTED; }
+constexpr int kApplyTile = 128;
+
+// ---- shared-memory plans (host and device agree on these) -------------------
+
+struct StatePlan {
+  int stages;
+  uint32_t off_tab, off_z, off_bar, off_tmem, total;
+};
+
+struct ApplyPlan {
+  int stages;
+  uint32_t off_g, off_S, off_den, off_z, off_tab, off_bar, off_tmem, total;
+};
+
+__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline StatePlan state_plan(int D, int entries, int stages) {
+  StatePlan p;
+  const uint32_t stage_bytes = 2u * tc_state_tile_c(D) * D * 2;
+  p.stages = stages;
+  uint32_t off = stages * stage_bytes;
+  p.off_tab = off;
+  off = align_up(off + entries * 8u, 32);
+  p.off_z = off;
+  off += 4u * D * 4;
+  p.off_bar = align_up(off, 8);
+  off = p.off_bar + (3u * stages + 5u) * 8u;
+  p.off_tmem = off;
+  off += 16;
+  p.total = off + 1024;  // slack to align the base to 1024 bytes
+  return p;
+}
+
+__host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, int stages) {
+  ApplyPlan p;
+  const uint32_t tile = (uint32_t)kApplyTile * D * 2;
+  p.stages = stages;
+  uint32_t off = stages * tile;
+  p.off_g = off;
+  off += gate ? stages * tile : 0;
+  p.off_S = align_up(off, 1024);
+  off = p.off_S + 2u * D * D * 2;
+  p.off_den = off;
+  off += stages * kApplyTile * 4u;
+  p.off_z = off;
+  off += D * 4u;
+  p.off_tab = align_up(off, 32);
+  off = p.off_tab + entries * 8u;
+  p.off_bar = align_up(off, 8);
+  off = p.off_bar + (4u * stages + 5u) * 8u;
+  p.off_tmem = off;
+  off += 16;
+  p.total = off + 1024;
+  return p;
+}
+
+inline int pick_state_stages(int D, int entries) {
+  for (int s = 6; s >= 2; --s)
+    if (state_plan(D, entries, s).total <= (uint32_t)kSmemBudget) return s;
+  return 0;
+}
+
+inline int pick_apply_stages(int D, int entries, int gate) {
+  for (int s = 4; s >= 2; --s)
+    if (apply_plan(D, entries, gate, s).total <= (uint32_t)kSmemBudget) return s;
+  return 0;
+}
+
+// Which calls take the tensor-core kernels: bf16 I/O, D in {64, 128}, and RoPE
+// widths that are multiples of 8 (a 16-byte chunk never spans two axes), with
+// both kernels' shared memory within budget (gated or not).
+inline bool tc_supported(bool bf16, int D, int rope, int dt, int dh, int dw, int entries) {
+  if (!bf16 || (D != 64 && D != 128)) return false;
+  if (rope && ((dt % 8) || (dh % 8) || (dw % 8))) return false;
+  int e = rope ? entries : 0;
+  return pick_state_stages(D, e) > 0 && pick_apply_stages(D, e, 1) > 0;
+}
+
+// ---- device helpers ------------------------------------------------------------
+
+// Bounded mbarrier wait: false after kWaitLimitNs (then the flag records it
+// and *abort tells the other roles to stop), or as soon as *abort is set.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, int* flag, int code,
+                                             volatile int* abort_flag) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (uint32_t n = 1;; ++n) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((n & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+        atomicOr(flag, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Token position (local frame, row, column) of token n, and a cheap step to
+// the token `step` rows further.
+struct Pos {
+  int tl, h, w;
+};
+
+__device__ __forceinline__ Pos pos_of(const Rope& r, long long n) {
+  Pos p;
+  const long long hw = (long long)r.Hg * r.Wg;
+  p.tl = (int)(n / hw);
+  const int rem = (int)(n - (long long)p.tl * hw);
+  p.h = rem / r.Wg;
+  p.w = rem - p.h * r.Wg;
+  return p;
+}
+
+__device__ __forceinline__ void pos_advance(const Rope& r, Pos& p, int step) {
+  p.w += step;
+  while (p.w >= r.Wg) {
+    p.w -= r.Wg;
+    if (++p.h == r.Hg) {
+      p.h = 0;
+      ++p.tl;
+    }
+  }
+}
+
+// The rotation pairs of one 16-byte chunk (8 dims) all belong to one axis.
+struct ChunkRope {
+  int ax;       // axis of the chunk (0 t, 1 h, 2 w)
+  int base;     // table entry of (axis, position 0, first pair of the chunk)
+  int stride;   // table entries per position on that axis
+};
+
+__device__ __forceinline__ ChunkRope chunk_rope(const Rope& r, int chunk) {
+  ChunkRope c;
+  const int p0 = 4 * chunk;
+  c.ax = p0 < r.pair_base[1] ? 0 : (p0 < r.pair_base[2] ? 1 : 2);
+  c.stride = r.half[c.ax];
+  c.base = r.tab_off[c.ax] + (p0 - r.pair_base[c.ax]);
+  return c;
+}
+
+// ReLU (and RoPE, if `cs` is non-null) of one chunk of 8 bf16 values in
+// place; phi(x) (un-rotated) is returned in f[].
+__device__ __forceinline__ uint4 relu_rope_chunk(uint4 raw, const float2* cs, float (&f)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float a = ptx::bf16_lo(w[j]), b = ptx::bf16_hi(w[j]);
+    f[2 * j] = a > 0.f ? a : 0.f;
+    f[2 * j + 1] = b > 0.f ? b : 0.f;
+  }
+  uint32_t o[4];
+  if (cs) {
+    const float4 c01 = reinterpret_cast<const float4*>(cs)[0];
+    const float4 c23 = reinterpret_cast<const float4*>(cs)[1];
+    const float c[4] = {c01.x, c01.z, c23.x, c23.z};
+    const float s[4] = {c01.y, c01.w, c23.y, c23.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float x = f[2 * j], y = f[2 * j + 1];
+      o[j] = ptx::pack_bf16x2(x * c[j] - y * s[j], x * s[j] + y * c[j]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = ptx::pack_bf16x2(f[2 * j], f[2 * j + 1]);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ---- state build ------------------------------------------------------------------
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               Rope rope, Sched sc, int stages, float* __restrict__ partials,
+               float2* __restrict__ gtab, int* flag) {
+  constexpr int TT = tc_state_tile_c(D);      // tokens per tile
+  constexpr int HALVES = D / 64;              // 64-column (128-byte) halves
+  constexpr int HALF_BYTES = TT * 128;        // one half of one tensor's tile
+  constexpr int TILE_BYTES = HALVES * HALF_BYTES;
+  constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  constexpr int CPR = D / 8;                  // 16-byte chunks per row
+  constexpr int RPT = kTcMath / CPR;          // rows per pass of the math warps
+  constexpr int NI = TT / RPT;                // rows per thread per tile
+  constexpr int KSTEPS = TT / 16;             // MMAs per tile
+  constexpr int DD1 = D * (D + 1);
+  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(D, D, 1, 1);
+  constexpr uint32_t TMEM_COLS = 2 * D;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_u32(smem_raw);
+  const uint32_t base = align_up(raw_addr, 1024);
+  uint8_t* sm = smem_raw + (base - raw_addr);
+  const StatePlan P = state_plan(D, rope.on ? rope.entries : 0, stages);
+  float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
+  float* s_z = reinterpret_cast<float*>(sm + P.off_z);
+  const uint32_t bar0 = base + P.off_bar;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto kready_bar = [&](int s) { return bar0 + 8u * (stages + s); };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (2 * stages + s); };
+  auto accf_bar = [&](int b) { return bar0 + 8u * (3 * stages + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (3 * stages + 2 + b); };
+  const uint32_t done_bar = bar0 + 8u * (3 * stages + 4);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P.off_tmem);
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int cta = blockIdx.x;
+  const long long u0 = unit_begin(sc, cta), u1 = unit_begin(sc, cta + 1);
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(kready_bar(s), kTcMath);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(accf_bar(b), 1);
+      ptx::mbar_init(acce_bar(b), kTcMath);
+    }
+    ptx::mbar_init(done_bar, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(s_tmem), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      long long j = 0;
+      for (long long u = u0; u < u1; ++u, ++j) {
+        const int seg = (int)(u / sc.tps);
+        const int tile = (int)(u - (long long)seg * sc.tps);
+        const int s = (int)(j % stages);
+        const uint32_t ph = (uint32_t)((j / stages) & 1);
+        if (!wait_bounded(empty_bar(s), ph ^ 1u, flag, kFlagStateTimeout, &s_abort)) break;
+        const uint32_t kt = base + s * STAGE_BYTES, vt = kt + TILE_BYTES;
+        ptx::mbar_expect_tx(full_bar(s), STAGE_BYTES);
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h) {
+          ptx::tma_load_3d(kt + h * HALF_BYTES, &tm_k, 64 * h, tile * TT, seg, full_bar(s));
+          ptx::tma_load_3d(vt + h * HALF_BYTES, &tm_v, 64 * h, tile * TT, seg, full_bar(s));
+        }
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      const long long issued = j;
+      for (long long i = issued - stages < 0 ? 0 : issued - stages; i < issued; ++i)
+        wait_bounded(full_bar((int)(i % stages)), (uint32_t)((i / stages) & 1), flag,
+                     kFlagStateTimeout, &s_abort);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t tmem = *s_tmem;
+      long long j = 0;
+      int sidx = -1, prev_seg = -1, first = 1;
+      for (long long u = u0; u < u1; ++u, ++j) {
+        const int seg = (int)(u / sc.tps);
+        if (seg != prev_seg) {
+          ++sidx;
+          prev_seg = seg;
+          first = 1;
+          const int b = sidx & 1;
+          if (!wait_bounded(acce_bar(b), (uint32_t)(((sidx >> 1) & 1) ^ 1), flag,
+                            kFlagStateTimeout, &s_abort))
+            break;
+        }
+        const int s = (int)(j % stages);
+        if (!wait_bounded(kready_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagStateTimeout,
+                          &s_abort))
+          break;
+        ptx::tc_fence_after();
+        const uint32_t kt = base + s * STAGE_BYTES, vt = kt + TILE_BYTES;
+        const uint32_t acc = tmem + (uint32_t)((sidx & 1) * D);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          const uint64_t a = ptx::smem_desc_sw128(kt + kk * 2048, HALF_BYTES, 1024);
+          const uint64_t b = ptx::smem_desc_sw128(vt + kk * 2048, HALF_BYTES, 1024);
+          ptx::mma_bf16(acc, a, b, IDESC, (first && kk == 0) ? 0u : 1u);
+        }
+        ptx::mma_commit(empty_bar(s));
+        first = 0;
+        const bool last = (u + 1 == u1) || ((u + 1) / sc.tps != seg);
+        if (last) ptx::mma_commit(accf_bar(sidx & 1));
+      }
+      ptx::mma_commit(done_bar);
+      wait_bounded(done_bar, 0, flag, kFlagStateTimeout, &s_abort);
+    }
+  } else {
+    // ---------------- math warps: ReLU + RoPE, z, epilogue ----------------
+    const int tt = threadIdx.x - 64;
+    const int c = tt % CPR, half = c >> 3, cc = c & 7, row0 = tt / CPR;
+    ChunkRope cr = {0, 0, 0};
+    if (rope.on) {
+      cr = chunk_rope(rope, c);
+      for (int e = tt; e < rope.entries; e += kTcMath) s_tab[e] = rope_entry(rope, e);
+      int e0 = (int)((long long)cta * rope.entries / gridDim.x);
+      int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);
+      ptx::bar_sync(1, kTcMath);
+      for (int e = e0 + tt; e < e1; e += kTcMath) gtab[e] = s_tab[e];
+    }
+    const uint32_t tmem = *s_tmem;
+    float z[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z[e] = 0.f;
+    long long j = 0;
+    int sidx = 0;
+    for (long long u = u0; u < u1; ++u, ++j) {
+      const int seg = (int)(u / sc.tps);
+      const int tile = (int)(u - (long long)seg * sc.tps);
+      const int s = (int)(j % stages);
+      bool ok = wait_bounded(full_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagStateTimeout,
+                             &s_abort);
+      if (!ptx::bar_all(1, kTcMath, ok)) break;
+      const int rows = min(TT, sc.L - tile * TT);
+      const uint32_t kt = base + s * STAGE_BYTES + half * HALF_BYTES;
+      Pos p = {0, 0, 0};
+      if (rope.on) {
+        const int blk = seg - (seg / sc.nblk) * sc.nblk;
+        p = pos_of(rope, (long long)blk * sc.L + (long long)tile * TT + row0);
+      }
+#pragma unroll 2
+      for (int i = 0; i < NI; ++i) {
+        const int r = row0 + i * RPT;
+        const uint32_t addr = kt + r * 128 + ((cc ^ (r & 7)) << 4);
+        const uint4 raw = ptx::ld_shared_v4(addr);
+        float f[8];
+        const float2* cs = nullptr;
+        if (rope.on && r < rows) {
+          const int pos = cr.ax == 0 ? p.tl : (cr.ax == 1 ? p.h : p.w);
+          cs = s_tab + cr.base + pos * cr.stride;
+        }
+        const uint4 o = relu_rope_chunk(raw, cs, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] += f[e];
+        ptx::st_shared_v4(addr, o);
+        if (rope.on) pos_advance(rope, p, RPT);
+      }
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(kready_bar(s));
+
+      const bool last = (u + 1 == u1) || ((u + 1) / sc.tps != seg);
+      if (last) {
+        const int b = sidx & 1;
+        ok = wait_bounded(accf_bar(b), (uint32_t)((sidx >> 1) & 1), flag, kFlagStateTimeout,
+                          &s_abort);
+        if (!ptx::bar_all(1, kTcMath, ok)) break;
+        ptx::tc_fence_after();
+        float* slot = partials + slot_index(sc, seg, cta) * DD1;
+        const int q = warp & 3;
+        // M = 64 keeps rows in lanes 0-15 of each 32-lane quadrant; M = 128
+        // uses all 128 lanes, row = lane.
+        const int row = D == 64 ? 16 * q + lane : 32 * q + lane;
+        const bool has_row = D == 64 ? lane < 16 : true;
+#pragma unroll
+        for (int cj = 0; cj < D / 32; ++cj) {
+          uint32_t v[32];
+          ptx::tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * D + 32 * cj), v);
+          ptx::tmem_wait_ld();
+          if (has_row) {
+            float4* dst = reinterpret_cast<float4*>(slot + (size_t)row * D + 32 * cj);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                   __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+          }
+        }
+        // z: sum the threads that own the same chunk, then the four warps in order
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float t = z[e];
+          for (int o = CPR; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          z[e] = t;
+        }
+        if (lane < CPR) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s_z[(warp - 2) * D + 8 * lane + e] = z[e];
+        }
+        ptx::bar_sync(1, kTcMath);
+        if (tt < D) slot[D * D + tt] = s_z[tt] + s_z[D + tt] + s_z[2 * D + tt] + s_z[3 * D + tt];
+        ptx::bar_sync(1, kTcMath);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] = 0.f;
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(acce_bar(b));
+        ++sidx;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(*s_tmem, TMEM_COLS);
+  }
+}
+
+// ---- apply ---------------------------------------------------------------------------
+
+constexpr int kTcThreadsApply = 224;  // warp 0 TMA load, 1 MMA, 2-5 math, 6 TMA store
+
+template <int D, bool GATE>
+__global__ void __launch_bounds__(kTcThreadsApply, 1)
+apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
+         const __grid_constant__ CUtensorMap tm_o, Rope rope, int L, int nblk, long long U,
+         int stages, const float* __restrict__ apply, const float2* __restrict__ gtab, float eps,
+         int* flag) {
+  constexpr int TM = kApplyTile;
+  constexpr int HALVES = D / 64;
+  constexpr int HALF_BYTES = TM * 128;
+  constexpr int TILE_BYTES = HALVES * HALF_BYTES;
+  constexpr int SHALF = D * 128;             // one K-half of the S operand
+  constexpr int CPR = D / 8;
+  constexpr int RPT = kTcMath / CPR;
+  constexpr int NI = TM / RPT;
+  constexpr int KSTEPS = D / 16;
+  constexpr int DD1 = D * (D + 1);
+  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, D, 0, 0);
+  constexpr uint32_t TMEM_COLS = 2 * D;
+  constexpr uint32_t TX = (GATE ? 2 : 1) * TILE_BYTES;
+  const int tps = (L + TM - 1) / TM;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_u32(smem_raw);
+  const uint32_t base = align_up(raw_addr, 1024);
+  uint8_t* sm = smem_raw + (base - raw_addr);
+  const ApplyPlan P = apply_plan(D, rope.on ? rope.entries : 0, GATE ? 1 : 0, stages);
+  const uint32_t gbase = base + P.off_g;
+  const uint32_t Shi = base + P.off_S, Slo = Shi + D * D * 2;
+  float* s_den = reinterpret_cast<float*>(sm + P.off_den);
+  float* s_z = reinterpret_cast<float*>(sm + P.off_z);
+  float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
+  const uint32_t bar0 = base + P.off_bar;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto qready_bar = [&](int s) { return bar0 + 8u * (stages + s); };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (2 * stages + s); };
+  auto oready_bar = [&](int s) { return bar0 + 8u * (3 * stages + s); };
+  auto accf_bar = [&](int b) { return bar0 + 8u * (4 * stages + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (4 * stages + 2 + b); };
+  const uint32_t done_bar = bar0 + 8u * (4 * stages + 4);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P.off_tmem);
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const long long u0 = (long long)blockIdx.x * U / gridDim.x;
+  const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(qready_bar(s), kTcMath);
+      ptx::mbar_init(empty_bar(s), 1);
+      ptx::mbar_init(oready_bar(s), kTcMath);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(accf_bar(b), 1);
+      ptx::mbar_init(acce_bar(b), kTcMath);
+    }
+    ptx::mbar_init(done_bar, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(s_tmem), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---------------- TMA loads: q (and gate) tiles ----------------
+    if (lane == 0) {
+      long long j = 0;
+      for (long long u = u0; u < u1; ++u, ++j) {
+        const int seg = (int)(u / tps);
+        const int tile = (int)(u - (long long)seg * tps);
+        const int s = (int)(j % stages);
+        if (!wait_bounded(empty_bar(s), (uint32_t)(((j / stages) & 1) ^ 1), flag,
+                          kFlagApplyTimeout, &s_abort))
+          break;
+        ptx::mbar_expect_tx(full_bar(s), TX);
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h) {
+          ptx::tma_load_3d(base + s * TILE_BYTES + h * HALF_BYTES, &tm_q, 64 * h, tile * TM, seg,
+                           full_bar(s));
+          if (GATE)
+            ptx::tma_load_3d(gbase + s * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h, tile * TM,
+                             seg, full_bar(s));
+        }
+      }
+      const long long issued = j;
+      for (long long i = issued - stages < 0 ? 0 : issued - stages; i < issued; ++i)
+        wait_bounded(full_bar((int)(i % stages)), (uint32_t)((i / stages) & 1), flag,
+                     kFlagApplyTimeout, &s_abort);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t tmem = *s_tmem;
+      long long j = 0;
+      for (long long u = u0; u < u1; ++u, ++j) {
+        const int s = (int)(j % stages);
+        const int b = (int)(j & 1);
+        if (!wait_bounded(acce_bar(b), (uint32_t)(((j >> 1) & 1) ^ 1), flag, kFlagApplyTimeout,
+                          &s_abort))
+          break;
+        if (!wait_bounded(qready_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagApplyTimeout,
+                          &s_abort))
+          break;
+        ptx::tc_fence_after();
+        const uint32_t qt = base + s * TILE_BYTES;
+        const uint32_t acc = tmem + (uint32_t)(b * D);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          const uint32_t aoff = (kk / 4) * HALF_BYTES + (kk % 4) * 32;
+          const uint32_t boff = (kk / 4) * SHALF + (kk % 4) * 32;
+          const uint64_t a = ptx::smem_desc_sw128(qt + aoff, 16, 1024);
+          ptx::mma_bf16(acc, a, ptx::smem_desc_sw128(Shi + boff, 16, 1024), IDESC,
+                        kk == 0 ? 0u : 1u);
+          ptx::mma_bf16(acc, a, ptx::smem_desc_sw128(Slo + boff, 16, 1024), IDESC, 1u);
+        }
+        ptx::mma_commit(accf_bar(b));
+      }
+      ptx::mma_commit(done_bar);
+      wait_bounded(done_bar, 0, flag, kFlagApplyTimeout, &s_abort);
+    }
+  } else if (warp == 6) {
+    // ---------------- TMA stores: out tiles, then free the stage ----------------
+    if (lane == 0) {
+      long long j = 0;
+      for (long long u = u0; u < u1; ++u, ++j) {
+        const int seg = (int)(u / tps);
+        const int tile = (int)(u - (long long)seg * tps);
+        const int s = (int)(j % stages);
+        if (!wait_bounded(oready_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagApplyTimeout,
+                          &s_abort))
+          break;
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h)
+          ptx::tma_store_3d(&tm_o, base + s * TILE_BYTES + h * HALF_BYTES, 64 * h, tile * TM,
+                            seg);
+        ptx::bulk_commit();
+        ptx::bulk_wait_read<0>();
+        ptx::mbar_arrive(empty_bar(s));
+      }
+      ptx::bulk_wait<0>();
+    }
+  } else {
+    // ---------------- math warps: phi(q), den, RoPE; epilogue ----------------
+    const int tt = threadIdx.x - 64;
+    const int c = tt % CPR, half = c >> 3, cc = c & 7, row0 = tt / CPR;
+    ChunkRope cr = {0, 0, 0};
+    if (rope.on) {
+      cr = chunk_rope(rope, c);
+      for (int e = tt; e < rope.entries; e += kTcMath) s_tab[e] = gtab[e];
+    }
+    const uint32_t tmem = *s_tmem;
+    const int q4 = warp & 3;
+    const int erow = 32 * q4 + lane;  // epilogue row = TMEM lane
+    float zc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zc[e] = 0.f;
+    int cur_seg = -1;
+    long long pend = -1;
+
+    // out = acc / den (* sigmoid(g)), bf16, written over the q tile of the stage
+    auto epilogue = [&](long long jj) -> bool {
+      const int s = (int)(jj % stages);
+      const int b = (int)(jj & 1);
+      bool ok = wait_bounded(accf_bar(b), (uint32_t)((jj >> 1) & 1), flag, kFlagApplyTimeout,
+                             &s_abort);
+      if (!ptx::bar_all(1, kTcMath, ok)) return false;
+      ptx::tc_fence_after();
+      const float inv = 1.f / s_den[s * TM + erow];
+      const uint32_t qt = base + s * TILE_BYTES;
+      const uint32_t gt = gbase + s * TILE_BYTES;
+#pragma unroll
+      for (int cj = 0; cj < D / 32; ++cj) {
+        uint32_t v[32];
+        ptx::tmem_ld_32x32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(b * D + 32 * cj), v);
+        ptx::tmem_wait_ld();
+        const int h = (32 * cj) / 64;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int chunk = ((32 * cj) % 64) / 8 + k4;
+          const uint32_t off = h * HALF_BYTES + erow * 128 + ((chunk ^ (erow & 7)) << 4);
+          float o[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = __uint_as_float(v[8 * k4 + e]) * inv;
+          if (GATE) {
+            const uint4 gr = ptx::ld_shared_v4(gt + off);
+            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              o[2 * e] *= 1.f / (1.f + __expf(-ptx::bf16_lo(gw[e])));
+              o[2 * e + 1] *= 1.f / (1.f + __expf(-ptx::bf16_hi(gw[e])));
+            }
+          }
+          ptx::st_shared_v4(qt + off, make_uint4(ptx::pack_bf16x2(o[0], o[1]),
+                                                  ptx::pack_bf16x2(o[2], o[3]),
+                                                  ptx::pack_bf16x2(o[4], o[5]),
+                                                  ptx::pack_bf16x2(o[6], o[7])));
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(acce_bar(b));
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(oready_bar(s));
+      return true;
+    };
+
+    long long j = 0;
+    bool alive = true;
+    for (long long u = u0; u < u1; ++u, ++j) {
+      const int seg = (int)(u / tps);
+      const int tile = (int)(u - (long long)seg * tps);
+      const int s = (int)(j % stages);
+      if (seg != cur_seg) {
+        // every MMA that reads the current S must be done before it is replaced
+        if (pend >= 0) {
+          if (!epilogue(pend)) { alive = false; break; }
+          pend = -1;
+        }
+        const float* src = apply + (long long)seg * DD1;
+        for (int it = tt; it < D * CPR; it += kTcMath) {
+          const int n = it % D, ac = it / D;        // output column n, K chunk ac
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = src[(8 * ac + e) * D + n];
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            hi[e] = ptx::pack_bf16x2(x[2 * e], x[2 * e + 1]);
+            lo[e] = ptx::pack_bf16x2(x[2 * e] - ptx::bf16_lo(hi[e]),
+                                     x[2 * e + 1] - ptx::bf16_hi(hi[e]));
+          }
+          const uint32_t off = (ac >> 3) * SHALF + n * 128 + (((ac & 7) ^ (n & 7)) << 4);
+          ptx::st_shared_v4(Shi + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+          ptx::st_shared_v4(Slo + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+        }
+        if (tt < D) s_z[tt] = src[D * D + tt];
+        ptx::fence_proxy_async();
+        ptx::bar_sync(1, kTcMath);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) zc[e] = s_z[8 * c + e];
+        cur_seg = seg;
+      }
+      bool ok = wait_bounded(full_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagApplyTimeout,
+                             &s_abort);
+      if (!ptx::bar_all(1, kTcMath, ok)) { alive = false; break; }
+      const int rows = min(TM, L - tile * TM);
+      const uint32_t qt = base + s * TILE_BYTES + half * HALF_BYTES;
+      Pos p = {0, 0, 0};
+      if (rope.on) {
+        const int blk = seg - (seg / nblk) * nblk;
+        p = pos_of(rope, (long long)blk * L + (long long)tile * TM + row0);
+      }
+#pragma unroll 2
+      for (int i = 0; i < NI; ++i) {
+        const int r = row0 + i * RPT;
+        const uint32_t addr = qt + r * 128 + ((cc ^ (r & 7)) << 4);
+        const uint4 raw = ptx::ld_shared_v4(addr);
+        float f[8];
+        const float2* cs = nullptr;
+        if (rope.on && r < rows) {
+          const int pos = cr.ax == 0 ? p.tl : (cr.ax == 1 ? p.h : p.w);
+          cs = s_tab + cr.base + pos * cr.stride;
+        }
+        const uint4 o = relu_rope_chunk(raw, cs, f);
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d = fmaf(f[e], zc[e], d);
+#pragma unroll
+        for (int o2 = 1; o2 < CPR; o2 <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
+        if (c == 0) s_den[s * TM + r] = d + eps;
+        ptx::st_shared_v4(addr, o);
+        if (rope.on) pos_advance(rope, p, RPT);
+      }
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(qready_bar(s));
+      if (pend >= 0 && !epilogue(pend)) { alive = false; break; }
+      pend = j;
+    }
+    if (alive && pend >= 0) epilogue(pend);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(*s_tmem, TMEM_COLS);
+  }
+}
+
+// ---- host launcher ---------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// [nseg][L][D] bf16 view of a [B,H,N,D] tensor; box = 64 columns x rows x 1.
+inline bool make_map(CUtensorMap* m, const void* ptr, int D, int L, int nseg, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)nseg};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)L * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+inline la_status tc_mark(const TcArgs& a, int i) {
+  if (!a.events || !a.events[i]) return LA_OK;
+  if (cudaEventRecord(static_cast<cudaEvent_t>(a.events[i]), a.stream) != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  return LA_OK;
+}
+
+inline la_status tc_check_launch() {
+  if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+  return LA_OK;
+}
+
+template <typename K>
+inline la_status tc_smem_attr(K kernel, uint32_t bytes) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_UNSUPPORTED;
+  }
+  return LA_OK;
+}
+
+template <int D>
+la_status tc_run_d(const TcArgs& a, int sms) {
+  const int entries = a.rope.on ? a.rope.entries : 0;
+  const Sched& sc = a.sc;
+  CUtensorMap mk, mv, mq, mg, mo;
+  if (!make_map(&mk, a.k, D, sc.L, sc.nseg, tc_state_tile_c(D)) ||
+      !make_map(&mv, a.v, D, sc.L, sc.nseg, tc_state_tile_c(D)))
+    return LA_ERR_CUDA;
+  la_status st;
+  const int s1 = pick_state_stages(D, entries);
+  const StatePlan p1 = state_plan(D, entries, s1);
+  if ((st = tc_smem_attr(state_build_tc<D>, p1.total)) != LA_OK) return st;
+  if ((st = tc_mark(a, 0)) != LA_OK) return st;
+  state_build_tc<D><<<sc.G, kTcThreads, p1.total, a.stream>>>(mk, mv, a.rope, sc, s1, a.part,
+                                                              a.gtab, a.flag);
+  if ((st = tc_check_launch()) != LA_OK) return st;
+  if ((st = tc_mark(a, 1)) != LA_OK) return st;
+  dim3 g2((D * (D + 1) + 255) / 256, (unsigned)(a.heads < 65535 ? a.heads : 65535));
+  reduce_states<D><<<g2, 256, 0, a.stream>>>(a.part, sc, a.apply, a.stS, a.stz, a.use_state,
+                                              a.commit);
+  if ((st = tc_check_launch()) != LA_OK) return st;
+  if ((st = tc_mark(a, 2)) != LA_OK) return st;
+  if (!a.do_apply) return LA_OK;
+
+  const bool gate = a.g != nullptr;
+  if (!make_map(&mq, a.q, D, sc.L, sc.nseg, kApplyTile) ||
+      !make_map(&mo, a.out, D, sc.L, sc.nseg, kApplyTile) ||
+      !make_map(&mg, gate ? a.g : a.q, D, sc.L, sc.nseg, kApplyTile))
+    return LA_ERR_CUDA;
+  const int s3 = pick_apply_stages(D, entries, gate ? 1 : 0);
+  const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3);
+  const long long U3 = (long long)sc.nseg * ((sc.L + kApplyTile - 1) / kApplyTile);
+  const int G3 = (int)(U3 < sms ? U3 : sms);
+  if (gate) {
+    if ((st = tc_smem_attr(apply_tc<D, true>, p3.total)) != LA_OK) return st;
+    apply_tc<D, true><<<G3, kTcThreadsApply, p3.total, a.stream>>>(
+        mq, mg, mo, a.rope, sc.L, sc.nblk, U3, s3, a.apply, a.gtab, a.eps, a.flag);
+  } else {
+    if ((st = tc_smem_attr(apply_tc<D, false>, p3.total)) != LA_OK) return st;
+    apply_tc<D, false><<<G3, kTcThreadsApply, p3.total, a.stream>>>(
+        mq, mg, mo, a.rope, sc.L, sc.nblk, U3, s3, a.apply, a.gtab, a.eps, a.flag);
+  }
+  if ((st = tc_check_launch()) != LA_OK) return st;
+  return tc_mark(a, 3);
+}
+
+inline la_status tc_run(const TcArgs& a, int sms) {
+  if (a.D == 64) return tc_run_d<64>(a, sms);
+  if (a.D == 128) return tc_run_d<128>(a, sms);
+  return LA_ERR_UNSUPPORTED;
+}
 
 }  // namespace la

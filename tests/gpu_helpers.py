@@ -26,10 +26,16 @@ def upload(w: workloads.Workload, x: dict, dev="cuda"):
 
 
 def run_forward(w: workloads.Workload, t: dict, mode: str, **kw) -> torch.Tensor:
-    out = la.forward(t["q"], t["k"], t["v"], t.get("g"), mode=mode,
-                     block_tokens=w.block_tokens if mode == "block_causal" else 0,
-                     grid=w.grid, rope_split=w.rope_split, theta=w.rope_theta, eps=w.eps, **kw)
+    bt = w.block_tokens if mode == "block_causal" else 0
+    p = la.make_params(w.B, w.H, w.N, w.D, t["q"].dtype, mode, bt, w.grid, w.rope_split,
+                       w.rope_theta, w.eps)
+    ws = la.workspace_for(p, t["q"].device)
+    out = la.forward(t["q"], t["k"], t["v"], t.get("g"), mode=mode, block_tokens=bt,
+                     grid=w.grid, rope_split=w.rope_split, theta=w.rope_theta, eps=w.eps,
+                     workspace=ws, **kw)
     torch.cuda.synchronize()
+    # no kernel may have given up a bounded wait
+    assert ws.status() == la._native.LA_OK
     return out
 
 

@@ -130,8 +130,10 @@ def test_state_init_and_block_step_argument_checks():
 
 def test_tensor_core_path_selection_is_host_logic():
     # bf16 with D in {64, 128} and rope widths that are multiples of 8 take the
-    # tensor-core kernels once they exist; fp32 and D = 32 never do.
-    p = _params(dtype=C.LA_F32)
-    assert C.lin_attn_uses_tensor_cores(p) == 0
-    p = _params(D=32)
-    assert C.lin_attn_uses_tensor_cores(p) == 0
+    # tensor-core kernels; fp32, D = 32 and other widths never do.
+    assert C.lin_attn_uses_tensor_cores(_params(dtype=C.LA_F32)) == 0
+    assert C.lin_attn_uses_tensor_cores(_params(D=32)) == 0
+    assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=16, rope_dh=24, rope_dw=24)) == 1
+    assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=20, rope_dh=22, rope_dw=22)) == 0
+    assert C.lin_attn_uses_tensor_cores(_params(D=128, rope_dt=32, rope_dh=48, rope_dw=48)) == 1
+    assert C.lin_attn_uses_tensor_cores(_params(D=64, rope=0)) == 1

@@ -246,7 +246,13 @@ def test_workspace_too_small_is_rejected():
 
 
 def test_tensor_core_path_is_selected_for_the_bf16_workloads():
-    for name in ("480p_bidir", "720p_long", "gated_d128"):
+    for name in ("480p_bidir", "480p_block_causal", "720p_long", "gated_d128"):
         w = W[name]
         assert la.uses_tensor_cores(w.B, w.H, w.N, w.D, torch.bfloat16, grid=w.grid,
-                                    rope_split=w.rope_split) in (True, False)
+                                    rope_split=w.rope_split)
+    # fp32 I/O, D = 32 and RoPE widths that are not multiples of 8 use CUDA cores
+    assert not la.uses_tensor_cores(1, 2, 256, 32, torch.float32)
+    assert not la.uses_tensor_cores(1, 4, 60, 32, torch.bfloat16, grid=(3, 4, 5),
+                                    rope_split=(8, 12, 12))
+    assert not la.uses_tensor_cores(1, 2, 24, 64, torch.bfloat16, grid=(2, 3, 4),
+                                    rope_split=(20, 22, 22))
