@@ -31,8 +31,6 @@
 
 namespace la {
 
-constexpr int kTcThreads = 192;         // warp 0 TMA, warp 1 MMA, warps 2-5 math
-constexpr int kTcMath = 128;            // threads of the math warps
 constexpr int kSmemBudget = 227 * 1024; // dynamic shared memory per CTA on sm_100
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -85,7 +83,7 @@ __host__ __device__ inline StatePlan state_plan(int D, int entries, int stages) 
   p.off_tab = off;
   off = align_up(off + entries * 8u, 32);
   p.off_z = off;
-  off += 4u * D * 4;
+  off += 8u * D * 4;  // z of each math warp
   p.off_bar = align_up(off, 8);
   off = p.off_bar + (3u * stages + 5u) * 8u;
   p.off_tmem = off;
@@ -102,7 +100,7 @@ __host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, in
   p.off_g = off;
   off += gate ? stages * tile : 0;
   p.off_S = align_up(off, 1024);
-  off = p.off_S + 2u * D * D * 2;
+  off = p.off_S + 2u * D * D * 2;  // B operand: S_hi^T and S_lo^T rows
   p.off_den = off;
   off += stages * kApplyTile * 4u;
   p.off_z = off;
@@ -203,26 +201,103 @@ __device__ __forceinline__ ChunkRope chunk_rope(const Rope& r, int chunk) {
   return c;
 }
 
-// ReLU (and RoPE, if `cs` is non-null) of one chunk of 8 bf16 values in
-// place; phi(x) (un-rotated) is returned in f[].
-__device__ __forceinline__ uint4 relu_rope_chunk(uint4 raw, const float2* cs, float (&f)[8]) {
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+// ---- shared pieces of the two kernels --------------------------------------------
+
+constexpr int kMathWarps = 8;
+constexpr int kMath = 32 * kMathWarps;  // threads of the math warps (warps 2 .. 9)
+
+// Walks a CTA's contiguous tile range: segment, tile in segment, ring stage
+// and phase, all advanced incrementally (no division inside the loops).
+struct TileIter {
+  int seg, tile, tps;
+  int stage, stages;
+  uint32_t phase;
+  __device__ __forceinline__ void init(long long u0, int tps_, int stages_) {
+    tps = tps_;
+    seg = (int)(u0 / tps_);
+    tile = (int)(u0 - (long long)seg * tps_);
+    stages = stages_;
+    stage = 0;
+    phase = 0;
+  }
+  __device__ __forceinline__ bool last_of_segment(long long u, long long u1) const {
+    return u + 1 == u1 || tile + 1 == tps;
+  }
+  __device__ __forceinline__ void next() {
+    if (++tile == tps) {
+      tile = 0;
+      ++seg;
+    }
+    if (++stage == stages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// Rotation factors of one chunk (4 pairs) for a run of consecutive tokens.
+// The t and h factors are reloaded only when the token's frame or row
+// changes; the w factors change every token.
+struct RopeRun {
+  int ax, base, stride;
+  int tl, h, w;
+  int last_pos;
+  float4 c01, c23;
+};
+
+__device__ __forceinline__ void rope_run_start(RopeRun& rr, const Rope& r, int chunk, long long n) {
+  const ChunkRope c = chunk_rope(r, chunk);
+  rr.ax = c.ax;
+  rr.base = c.base;
+  rr.stride = c.stride;
+  const Pos p = pos_of(r, n);
+  rr.tl = p.tl;
+  rr.h = p.h;
+  rr.w = p.w;
+  rr.last_pos = -1;
+}
+
+__device__ __forceinline__ void rope_run_load(RopeRun& rr, const float2* tab) {
+  const int pos = rr.ax == 0 ? rr.tl : (rr.ax == 1 ? rr.h : rr.w);
+  if (pos != rr.last_pos) {
+    const float4* t4 = reinterpret_cast<const float4*>(tab + rr.base + pos * rr.stride);
+    rr.c01 = t4[0];
+    rr.c23 = t4[1];
+    rr.last_pos = pos;
+  }
+}
+
+__device__ __forceinline__ void rope_run_next(RopeRun& rr, const Rope& r) {
+  if (++rr.w == r.Wg) {
+    rr.w = 0;
+    if (++rr.h == r.Hg) {
+      rr.h = 0;
+      ++rr.tl;
+    }
+  }
+}
+
+// phi = ReLU on 8 bf16 values, optionally the rotation of the 4 pairs; the
+// un-rotated phi values come back in f[] (fp32).
+__device__ __forceinline__ uint4 phi_rope(uint4 raw, bool rotate, const float4& c01,
+                                          const float4& c23, float (&f)[8]) {
+  const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    float a = ptx::bf16_lo(w[j]), b = ptx::bf16_hi(w[j]);
-    f[2 * j] = a > 0.f ? a : 0.f;
-    f[2 * j + 1] = b > 0.f ? b : 0.f;
+    // ReLU on the packed pair: max(x, 0) in bf16 is exact
+    uint32_t m;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(w4[j]), "r"(0u));
+    f[2 * j] = ptx::bf16_lo(m);
+    f[2 * j + 1] = ptx::bf16_hi(m);
   }
   uint32_t o[4];
-  if (cs) {
-    const float4 c01 = reinterpret_cast<const float4*>(cs)[0];
-    const float4 c23 = reinterpret_cast<const float4*>(cs)[1];
-    const float c[4] = {c01.x, c01.z, c23.x, c23.z};
-    const float s[4] = {c01.y, c01.w, c23.y, c23.w};
+  if (rotate) {
+    const float cs[4] = {c01.x, c01.z, c23.x, c23.z};
+    const float sn[4] = {c01.y, c01.w, c23.y, c23.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float x = f[2 * j], y = f[2 * j + 1];
-      o[j] = ptx::pack_bf16x2(x * c[j] - y * s[j], x * s[j] + y * c[j]);
+      o[j] = ptx::pack_bf16x2(fmaf(x, cs[j], -y * sn[j]), fmaf(x, sn[j], y * cs[j]));
     }
   } else {
 #pragma unroll
@@ -233,8 +308,10 @@ __device__ __forceinline__ uint4 relu_rope_chunk(uint4 raw, const float2* cs, fl
 
 // ---- state build ------------------------------------------------------------------
 
+constexpr int kTcThreadsState = 64 + kMath;  // warp 0 TMA, warp 1 MMA, warps 2-9 math
+
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreadsState, 1)
 state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                Rope rope, Sched sc, int stages, float* __restrict__ partials,
                float2* __restrict__ gtab, int* flag) {
@@ -244,12 +321,12 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   constexpr int TILE_BYTES = HALVES * HALF_BYTES;
   constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   constexpr int CPR = D / 8;                  // 16-byte chunks per row
-  constexpr int RPT = kTcMath / CPR;          // rows per pass of the math warps
-  constexpr int NI = TT / RPT;                // rows per thread per tile
+  constexpr int RT = TT * CPR / kMath;        // consecutive rows per thread (4)
   constexpr int KSTEPS = TT / 16;             // MMAs per tile
   constexpr int DD1 = D * (D + 1);
   constexpr uint32_t IDESC = ptx::idesc_bf16_f32(D, D, 1, 1);
   constexpr uint32_t TMEM_COLS = 2 * D;
+  static_assert(RT * kMath == TT * CPR, "tile must split evenly over the math threads");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
@@ -276,12 +353,12 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     s_abort = 0;
     for (int s = 0; s < stages; ++s) {
       ptx::mbar_init(full_bar(s), 1);
-      ptx::mbar_init(kready_bar(s), kTcMath);
+      ptx::mbar_init(kready_bar(s), kMath);
       ptx::mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(accf_bar(b), 1);
-      ptx::mbar_init(acce_bar(b), kTcMath);
+      ptx::mbar_init(acce_bar(b), kMath);
     }
     ptx::mbar_init(done_bar, 1);
     ptx::fence_mbar_init();
@@ -295,23 +372,24 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      long long j = 0;
-      for (long long u = u0; u < u1; ++u, ++j) {
-        const int seg = (int)(u / sc.tps);
-        const int tile = (int)(u - (long long)seg * sc.tps);
-        const int s = (int)(j % stages);
-        const uint32_t ph = (uint32_t)((j / stages) & 1);
-        if (!wait_bounded(empty_bar(s), ph ^ 1u, flag, kFlagStateTimeout, &s_abort)) break;
-        const uint32_t kt = base + s * STAGE_BYTES, vt = kt + TILE_BYTES;
-        ptx::mbar_expect_tx(full_bar(s), STAGE_BYTES);
+      TileIter it;
+      it.init(u0, sc.tps, stages);
+      long long issued = 0;
+      for (long long u = u0; u < u1; ++u, it.next()) {
+        if (!wait_bounded(empty_bar(it.stage), it.phase ^ 1u, flag, kFlagStateTimeout, &s_abort))
+          break;
+        const uint32_t kt = base + it.stage * STAGE_BYTES, vt = kt + TILE_BYTES;
+        ptx::mbar_expect_tx(full_bar(it.stage), STAGE_BYTES);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h) {
-          ptx::tma_load_3d(kt + h * HALF_BYTES, &tm_k, 64 * h, tile * TT, seg, full_bar(s));
-          ptx::tma_load_3d(vt + h * HALF_BYTES, &tm_v, 64 * h, tile * TT, seg, full_bar(s));
+          ptx::tma_load_3d(kt + h * HALF_BYTES, &tm_k, 64 * h, it.tile * TT, it.seg,
+                           full_bar(it.stage));
+          ptx::tma_load_3d(vt + h * HALF_BYTES, &tm_v, 64 * h, it.tile * TT, it.seg,
+                           full_bar(it.stage));
         }
+        ++issued;
       }
       // drain: every issued copy has landed before the CTA may exit
-      const long long issued = j;
       for (long long i = issued - stages < 0 ? 0 : issued - stages; i < issued; ++i)
         wait_bounded(full_bar((int)(i % stages)), (uint32_t)((i / stages) & 1), flag,
                      kFlagStateTimeout, &s_abort);
@@ -320,25 +398,15 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t tmem = *s_tmem;
-      long long j = 0;
-      int sidx = -1, prev_seg = -1, first = 1;
-      for (long long u = u0; u < u1; ++u, ++j) {
-        const int seg = (int)(u / sc.tps);
-        if (seg != prev_seg) {
-          ++sidx;
-          prev_seg = seg;
-          first = 1;
-          const int b = sidx & 1;
-          if (!wait_bounded(acce_bar(b), (uint32_t)(((sidx >> 1) & 1) ^ 1), flag,
-                            kFlagStateTimeout, &s_abort))
-            break;
-        }
-        const int s = (int)(j % stages);
-        if (!wait_bounded(kready_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagStateTimeout,
-                          &s_abort))
+      TileIter it;
+      it.init(u0, sc.tps, stages);
+      int sidx = 0, first = 1;
+      bool ok = wait_bounded(acce_bar(0), 1u, flag, kFlagStateTimeout, &s_abort);
+      for (long long u = u0; u < u1 && ok; ++u) {
+        if (!wait_bounded(kready_bar(it.stage), it.phase, flag, kFlagStateTimeout, &s_abort))
           break;
         ptx::tc_fence_after();
-        const uint32_t kt = base + s * STAGE_BYTES, vt = kt + TILE_BYTES;
+        const uint32_t kt = base + it.stage * STAGE_BYTES, vt = kt + TILE_BYTES;
         const uint32_t acc = tmem + (uint32_t)((sidx & 1) * D);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -346,10 +414,18 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           const uint64_t b = ptx::smem_desc_sw128(vt + kk * 2048, HALF_BYTES, 1024);
           ptx::mma_bf16(acc, a, b, IDESC, (first && kk == 0) ? 0u : 1u);
         }
-        ptx::mma_commit(empty_bar(s));
+        ptx::mma_commit(empty_bar(it.stage));
         first = 0;
-        const bool last = (u + 1 == u1) || ((u + 1) / sc.tps != seg);
-        if (last) ptx::mma_commit(accf_bar(sidx & 1));
+        if (it.last_of_segment(u, u1)) {
+          ptx::mma_commit(accf_bar(sidx & 1));
+          ++sidx;
+          first = 1;
+          if (u + 1 < u1 &&
+              !wait_bounded(acce_bar(sidx & 1), (uint32_t)(((sidx >> 1) & 1) ^ 1), flag,
+                            kFlagStateTimeout, &s_abort))
+            break;
+        }
+        it.next();
       }
       ptx::mma_commit(done_bar);
       wait_bounded(done_bar, 0, flag, kFlagStateTimeout, &s_abort);
@@ -357,98 +433,93 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   } else {
     // ---------------- math warps: ReLU + RoPE, z, epilogue ----------------
     const int tt = threadIdx.x - 64;
-    const int c = tt % CPR, half = c >> 3, cc = c & 7, row0 = tt / CPR;
-    ChunkRope cr = {0, 0, 0};
+    const int mw = warp - 2;                     // math warp 0..7
+    const int c = tt % CPR, half = c >> 3, cc = c & 7, k = tt / CPR;
     if (rope.on) {
-      cr = chunk_rope(rope, c);
-      for (int e = tt; e < rope.entries; e += kTcMath) s_tab[e] = rope_entry(rope, e);
-      int e0 = (int)((long long)cta * rope.entries / gridDim.x);
-      int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);
-      ptx::bar_sync(1, kTcMath);
-      for (int e = e0 + tt; e < e1; e += kTcMath) gtab[e] = s_tab[e];
+      for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = rope_entry(rope, e);
+      ptx::bar_sync(1, kMath);
+      const int e0 = (int)((long long)cta * rope.entries / gridDim.x);
+      const int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);
+      for (int e = e0 + tt; e < e1; e += kMath) gtab[e] = s_tab[e];
     }
     const uint32_t tmem = *s_tmem;
     float z[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) z[e] = 0.f;
-    long long j = 0;
+    TileIter it;
+    it.init(u0, sc.tps, stages);
     int sidx = 0;
-    for (long long u = u0; u < u1; ++u, ++j) {
-      const int seg = (int)(u / sc.tps);
-      const int tile = (int)(u - (long long)seg * sc.tps);
-      const int s = (int)(j % stages);
-      bool ok = wait_bounded(full_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagStateTimeout,
-                             &s_abort);
-      if (!ptx::bar_all(1, kTcMath, ok)) break;
-      const int rows = min(TT, sc.L - tile * TT);
-      const uint32_t kt = base + s * STAGE_BYTES + half * HALF_BYTES;
-      Pos p = {0, 0, 0};
-      if (rope.on) {
-        const int blk = seg - (seg / sc.nblk) * sc.nblk;
-        p = pos_of(rope, (long long)blk * sc.L + (long long)tile * TT + row0);
-      }
-#pragma unroll 2
-      for (int i = 0; i < NI; ++i) {
-        const int r = row0 + i * RPT;
-        const uint32_t addr = kt + r * 128 + ((cc ^ (r & 7)) << 4);
-        const uint4 raw = ptx::ld_shared_v4(addr);
-        float f[8];
-        const float2* cs = nullptr;
-        if (rope.on && r < rows) {
-          const int pos = cr.ax == 0 ? p.tl : (cr.ax == 1 ? p.h : p.w);
-          cs = s_tab + cr.base + pos * cr.stride;
+    for (long long u = u0; u < u1; ++u, it.next()) {
+      const bool ok = wait_bounded(full_bar(it.stage), it.phase, flag, kFlagStateTimeout,
+                                   &s_abort);
+      if (ok) {
+        const int rows = min(TT, sc.L - it.tile * TT);
+        const uint32_t kt = base + it.stage * STAGE_BYTES + half * HALF_BYTES;
+        RopeRun rr;
+        if (rope.on) {
+          const int blk = it.seg - (it.seg / sc.nblk) * sc.nblk;
+          rope_run_start(rr, rope, c, (long long)blk * sc.L + (long long)it.tile * TT + RT * k);
         }
-        const uint4 o = relu_rope_chunk(raw, cs, f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) z[e] += f[e];
-        ptx::st_shared_v4(addr, o);
-        if (rope.on) pos_advance(rope, p, RPT);
+        for (int i = 0; i < RT; ++i) {
+          const int r = RT * k + i;
+          const uint32_t addr = kt + r * 128 + ((cc ^ (r & 7)) << 4);
+          const uint4 raw = ptx::ld_shared_v4(addr);
+          const bool rot = rope.on && r < rows;
+          if (rot) rope_run_load(rr, s_tab);
+          float f[8];
+          const uint4 o = phi_rope(raw, rot, rr.c01, rr.c23, f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) z[e] += f[e];
+          ptx::st_shared_v4(addr, o);
+          if (rope.on) rope_run_next(rr, rope);
+        }
+        ptx::fence_proxy_async();
+        ptx::mbar_arrive(kready_bar(it.stage));
       }
-      ptx::fence_proxy_async();
-      ptx::mbar_arrive(kready_bar(s));
-
-      const bool last = (u + 1 == u1) || ((u + 1) / sc.tps != seg);
-      if (last) {
+      if (it.last_of_segment(u, u1)) {
+        // the segment's partial: TMEM accumulator -> S rows, then z
         const int b = sidx & 1;
-        ok = wait_bounded(accf_bar(b), (uint32_t)((sidx >> 1) & 1), flag, kFlagStateTimeout,
-                          &s_abort);
-        if (!ptx::bar_all(1, kTcMath, ok)) break;
+        const bool ready = wait_bounded(accf_bar(b), (uint32_t)((sidx >> 1) & 1), flag,
+                                        kFlagStateTimeout, &s_abort);
         ptx::tc_fence_after();
-        float* slot = partials + slot_index(sc, seg, cta) * DD1;
-        const int q = warp & 3;
+        float* slot = partials + slot_index(sc, it.seg, cta) * DD1;
+        const int q = warp & 3, pw = mw >> 2;    // lane quadrant, column half
         // M = 64 keeps rows in lanes 0-15 of each 32-lane quadrant; M = 128
         // uses all 128 lanes, row = lane.
         const int row = D == 64 ? 16 * q + lane : 32 * q + lane;
         const bool has_row = D == 64 ? lane < 16 : true;
 #pragma unroll
-        for (int cj = 0; cj < D / 32; ++cj) {
+        for (int cj = 0; cj < D / 64; ++cj) {
+          const int col = pw * (D / 2) + 32 * cj;
           uint32_t v[32];
-          ptx::tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * D + 32 * cj), v);
+          ptx::tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * D + col), v);
           ptx::tmem_wait_ld();
-          if (has_row) {
-            float4* dst = reinterpret_cast<float4*>(slot + (size_t)row * D + 32 * cj);
+          if (ready && has_row) {
+            float4* dst = reinterpret_cast<float4*>(slot + (size_t)row * D + col);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
                                    __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
           }
         }
-        // z: sum the threads that own the same chunk, then the four warps in order
+        // z: the threads of one chunk within a warp, then the 8 warps in order
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float t = z[e];
+#pragma unroll
           for (int o = CPR; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          z[e] = t;
+          z[e] = 0.f;
+          if (lane < CPR) s_z[mw * D + 8 * lane + e] = t;
         }
-        if (lane < CPR) {
+        ptx::bar_sync(1, kMath);
+        if (tt < D && ready) {
+          float t = 0.f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) s_z[(warp - 2) * D + 8 * lane + e] = z[e];
+          for (int w = 0; w < kMathWarps; ++w) t += s_z[w * D + tt];
+          slot[D * D + tt] = t;
         }
-        ptx::bar_sync(1, kTcMath);
-        if (tt < D) slot[D * D + tt] = s_z[tt] + s_z[D + tt] + s_z[2 * D + tt] + s_z[3 * D + tt];
-        ptx::bar_sync(1, kTcMath);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) z[e] = 0.f;
+        ptx::bar_sync(1, kMath);
         ptx::tc_fence_before();
         ptx::mbar_arrive(acce_bar(b));
         ++sidx;
@@ -465,7 +536,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
 // ---- apply ---------------------------------------------------------------------------
 
-constexpr int kTcThreadsApply = 224;  // warp 0 TMA load, 1 MMA, 2-5 math, 6 TMA store
+constexpr int kTcThreadsApply = 96 + kMath;  // warp 0 load, 1 MMA, 2-9 math, 10 store
 
 template <int D, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
@@ -477,15 +548,17 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   constexpr int HALVES = D / 64;
   constexpr int HALF_BYTES = TM * 128;
   constexpr int TILE_BYTES = HALVES * HALF_BYTES;
-  constexpr int SHALF = D * 128;             // one K-half of the S operand
+  constexpr int NB = 2 * D;                  // B operand rows: S_hi^T then S_lo^T
+  constexpr int SHALF = NB * 128;            // one K-half of the B operand
   constexpr int CPR = D / 8;
-  constexpr int RPT = kTcMath / CPR;
-  constexpr int NI = TM / RPT;
+  constexpr int RT = TM * CPR / kMath;       // consecutive rows per thread (4 or 8)
   constexpr int KSTEPS = D / 16;
   constexpr int DD1 = D * (D + 1);
-  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, D, 0, 0);
-  constexpr uint32_t TMEM_COLS = 2 * D;
+  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, NB, 0, 0);
+  constexpr uint32_t TMEM_COLS = 2 * NB;
   constexpr uint32_t TX = (GATE ? 2 : 1) * TILE_BYTES;
+  constexpr int EC = D / 2;                  // epilogue columns per thread
+  static_assert(RT * kMath == TM * CPR, "tile must split evenly over the math threads");
   const int tps = (L + TM - 1) / TM;
 
   extern __shared__ uint8_t smem_raw[];
@@ -494,7 +567,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   uint8_t* sm = smem_raw + (base - raw_addr);
   const ApplyPlan P = apply_plan(D, rope.on ? rope.entries : 0, GATE ? 1 : 0, stages);
   const uint32_t gbase = base + P.off_g;
-  const uint32_t Shi = base + P.off_S, Slo = Shi + D * D * 2;
+  const uint32_t Sb = base + P.off_S;
   float* s_den = reinterpret_cast<float*>(sm + P.off_den);
   float* s_z = reinterpret_cast<float*>(sm + P.off_z);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
@@ -517,13 +590,13 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     s_abort = 0;
     for (int s = 0; s < stages; ++s) {
       ptx::mbar_init(full_bar(s), 1);
-      ptx::mbar_init(qready_bar(s), kTcMath);
+      ptx::mbar_init(qready_bar(s), kMath);
       ptx::mbar_init(empty_bar(s), 1);
-      ptx::mbar_init(oready_bar(s), kTcMath);
+      ptx::mbar_init(oready_bar(s), kMath);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(accf_bar(b), 1);
-      ptx::mbar_init(acce_bar(b), kTcMath);
+      ptx::mbar_init(acce_bar(b), kMath);
     }
     ptx::mbar_init(done_bar, 1);
     ptx::fence_mbar_init();
@@ -537,123 +610,124 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   if (warp == 0) {
     // ---------------- TMA loads: q (and gate) tiles ----------------
     if (lane == 0) {
-      long long j = 0;
-      for (long long u = u0; u < u1; ++u, ++j) {
-        const int seg = (int)(u / tps);
-        const int tile = (int)(u - (long long)seg * tps);
-        const int s = (int)(j % stages);
-        if (!wait_bounded(empty_bar(s), (uint32_t)(((j / stages) & 1) ^ 1), flag,
-                          kFlagApplyTimeout, &s_abort))
+      TileIter it;
+      it.init(u0, tps, stages);
+      long long issued = 0;
+      for (long long u = u0; u < u1; ++u, it.next()) {
+        if (!wait_bounded(empty_bar(it.stage), it.phase ^ 1u, flag, kFlagApplyTimeout, &s_abort))
           break;
-        ptx::mbar_expect_tx(full_bar(s), TX);
+        ptx::mbar_expect_tx(full_bar(it.stage), TX);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h) {
-          ptx::tma_load_3d(base + s * TILE_BYTES + h * HALF_BYTES, &tm_q, 64 * h, tile * TM, seg,
-                           full_bar(s));
+          ptx::tma_load_3d(base + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_q, 64 * h,
+                           it.tile * TM, it.seg, full_bar(it.stage));
           if (GATE)
-            ptx::tma_load_3d(gbase + s * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h, tile * TM,
-                             seg, full_bar(s));
+            ptx::tma_load_3d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h,
+                             it.tile * TM, it.seg, full_bar(it.stage));
         }
+        ++issued;
       }
-      const long long issued = j;
       for (long long i = issued - stages < 0 ? 0 : issued - stages; i < issued; ++i)
         wait_bounded(full_bar((int)(i % stages)), (uint32_t)((i / stages) & 1), flag,
                      kFlagApplyTimeout, &s_abort);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- MMA issuer: acc[b] = RoPE(phi q) [S_hi | S_lo] ----------------
     if (lane == 0) {
       const uint32_t tmem = *s_tmem;
-      long long j = 0;
-      for (long long u = u0; u < u1; ++u, ++j) {
-        const int s = (int)(j % stages);
-        const int b = (int)(j & 1);
-        if (!wait_bounded(acce_bar(b), (uint32_t)(((j >> 1) & 1) ^ 1), flag, kFlagApplyTimeout,
-                          &s_abort))
-          break;
-        if (!wait_bounded(qready_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagApplyTimeout,
-                          &s_abort))
+      TileIter it;
+      it.init(u0, tps, stages);
+      int b = 0;
+      uint32_t bph = 0;
+      for (long long u = u0; u < u1; ++u, it.next()) {
+        if (!wait_bounded(acce_bar(b), bph ^ 1u, flag, kFlagApplyTimeout, &s_abort)) break;
+        if (!wait_bounded(qready_bar(it.stage), it.phase, flag, kFlagApplyTimeout, &s_abort))
           break;
         ptx::tc_fence_after();
-        const uint32_t qt = base + s * TILE_BYTES;
-        const uint32_t acc = tmem + (uint32_t)(b * D);
+        const uint32_t qt = base + it.stage * TILE_BYTES;
+        const uint32_t acc = tmem + (uint32_t)(b * NB);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
           const uint32_t aoff = (kk / 4) * HALF_BYTES + (kk % 4) * 32;
           const uint32_t boff = (kk / 4) * SHALF + (kk % 4) * 32;
-          const uint64_t a = ptx::smem_desc_sw128(qt + aoff, 16, 1024);
-          ptx::mma_bf16(acc, a, ptx::smem_desc_sw128(Shi + boff, 16, 1024), IDESC,
-                        kk == 0 ? 0u : 1u);
-          ptx::mma_bf16(acc, a, ptx::smem_desc_sw128(Slo + boff, 16, 1024), IDESC, 1u);
+          ptx::mma_bf16(acc, ptx::smem_desc_sw128(qt + aoff, 16, 1024),
+                        ptx::smem_desc_sw128(Sb + boff, 16, 1024), IDESC, kk == 0 ? 0u : 1u);
         }
         ptx::mma_commit(accf_bar(b));
+        if (++b == 2) {
+          b = 0;
+          bph ^= 1u;
+        }
       }
       ptx::mma_commit(done_bar);
       wait_bounded(done_bar, 0, flag, kFlagApplyTimeout, &s_abort);
     }
-  } else if (warp == 6) {
+  } else if (warp == 2 + kMathWarps) {
     // ---------------- TMA stores: out tiles, then free the stage ----------------
     if (lane == 0) {
-      long long j = 0;
-      for (long long u = u0; u < u1; ++u, ++j) {
-        const int seg = (int)(u / tps);
-        const int tile = (int)(u - (long long)seg * tps);
-        const int s = (int)(j % stages);
-        if (!wait_bounded(oready_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagApplyTimeout,
-                          &s_abort))
+      TileIter it;
+      it.init(u0, tps, stages);
+      for (long long u = u0; u < u1; ++u, it.next()) {
+        if (!wait_bounded(oready_bar(it.stage), it.phase, flag, kFlagApplyTimeout, &s_abort))
           break;
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
-          ptx::tma_store_3d(&tm_o, base + s * TILE_BYTES + h * HALF_BYTES, 64 * h, tile * TM,
-                            seg);
+          ptx::tma_store_3d(&tm_o, base + it.stage * TILE_BYTES + h * HALF_BYTES, 64 * h,
+                            it.tile * TM, it.seg);
         ptx::bulk_commit();
         ptx::bulk_wait_read<0>();
-        ptx::mbar_arrive(empty_bar(s));
+        ptx::mbar_arrive(empty_bar(it.stage));
       }
       ptx::bulk_wait<0>();
     }
   } else {
     // ---------------- math warps: phi(q), den, RoPE; epilogue ----------------
     const int tt = threadIdx.x - 64;
-    const int c = tt % CPR, half = c >> 3, cc = c & 7, row0 = tt / CPR;
-    ChunkRope cr = {0, 0, 0};
-    if (rope.on) {
-      cr = chunk_rope(rope, c);
-      for (int e = tt; e < rope.entries; e += kTcMath) s_tab[e] = gtab[e];
-    }
+    const int mw = warp - 2;
+    const int q4 = warp & 3, pw = mw >> 2;   // TMEM lane quadrant, column half
+    // a warp transforms 16 rows of its own lane quadrant, so the den values
+    // the epilogue reads come from the two warps that share the quadrant
+    const int c = lane % CPR, half = c >> 3, cc = c & 7;
+    const int row_first = 32 * q4 + 16 * pw + RT * (lane / CPR);
+    if (rope.on)
+      for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = gtab[e];
     const uint32_t tmem = *s_tmem;
-    const int q4 = warp & 3;
-    const int erow = 32 * q4 + lane;  // epilogue row = TMEM lane
+    const int erow = 32 * q4 + lane;   // epilogue row = TMEM lane
     float zc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) zc[e] = 0.f;
     int cur_seg = -1;
-    long long pend = -1;
+    int pend_stage = -1, pend_b = 0;
+    uint32_t pend_bph = 0;
+    int b = 0;
+    uint32_t bph = 0;
 
-    // out = acc / den (* sigmoid(g)), bf16, written over the q tile of the stage
-    auto epilogue = [&](long long jj) -> bool {
-      const int s = (int)(jj % stages);
-      const int b = (int)(jj & 1);
-      bool ok = wait_bounded(accf_bar(b), (uint32_t)((jj >> 1) & 1), flag, kFlagApplyTimeout,
-                             &s_abort);
-      if (!ptx::bar_all(1, kTcMath, ok)) return false;
+    // out = (acc_hi + acc_lo) / den (* sigmoid(g)) as bf16, over the q tile
+    auto epilogue = [&](int s, int eb, uint32_t ebph) {
+      const bool ready = wait_bounded(accf_bar(eb), ebph, flag, kFlagApplyTimeout, &s_abort);
+      ptx::bar_sync(2 + q4, 64);   // den of this quadrant's rows is in shared memory
       ptx::tc_fence_after();
       const float inv = 1.f / s_den[s * TM + erow];
       const uint32_t qt = base + s * TILE_BYTES;
       const uint32_t gt = gbase + s * TILE_BYTES;
+      const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(eb * NB);
 #pragma unroll
-      for (int cj = 0; cj < D / 32; ++cj) {
-        uint32_t v[32];
-        ptx::tmem_ld_32x32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(b * D + 32 * cj), v);
+      for (int cj = 0; cj < EC / 32; ++cj) {
+        const int col = pw * EC + 32 * cj;
+        uint32_t vh[32], vl[32];
+        ptx::tmem_ld_32x32(lane_base + col, vh);
+        ptx::tmem_ld_32x32(lane_base + D + col, vl);
         ptx::tmem_wait_ld();
-        const int h = (32 * cj) / 64;
+        if (!ready) continue;
+        const int h = col / 64;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
-          const int chunk = ((32 * cj) % 64) / 8 + k4;
+          const int chunk = (col % 64) / 8 + k4;
           const uint32_t off = h * HALF_BYTES + erow * 128 + ((chunk ^ (erow & 7)) << 4);
           float o[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[e] = __uint_as_float(v[8 * k4 + e]) * inv;
+          for (int e = 0; e < 8; ++e)
+            o[e] = (__uint_as_float(vh[8 * k4 + e]) + __uint_as_float(vl[8 * k4 + e])) * inv;
           if (GATE) {
             const uint4 gr = ptx::ld_shared_v4(gt + off);
             const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
@@ -670,27 +744,23 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         }
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(acce_bar(b));
+      ptx::mbar_arrive(acce_bar(eb));
       ptx::fence_proxy_async();
       ptx::mbar_arrive(oready_bar(s));
-      return true;
     };
 
-    long long j = 0;
-    bool alive = true;
-    for (long long u = u0; u < u1; ++u, ++j) {
-      const int seg = (int)(u / tps);
-      const int tile = (int)(u - (long long)seg * tps);
-      const int s = (int)(j % stages);
-      if (seg != cur_seg) {
+    TileIter it;
+    it.init(u0, tps, stages);
+    for (long long u = u0; u < u1; ++u, it.next()) {
+      if (it.seg != cur_seg) {
         // every MMA that reads the current S must be done before it is replaced
-        if (pend >= 0) {
-          if (!epilogue(pend)) { alive = false; break; }
-          pend = -1;
+        if (pend_stage >= 0) {
+          epilogue(pend_stage, pend_b, pend_bph);
+          pend_stage = -1;
         }
-        const float* src = apply + (long long)seg * DD1;
-        for (int it = tt; it < D * CPR; it += kTcMath) {
-          const int n = it % D, ac = it / D;        // output column n, K chunk ac
+        const float* src = apply + (long long)it.seg * DD1;
+        for (int item = tt; item < D * CPR; item += kMath) {
+          const int n = item % D, ac = item / D;    // output column n, K chunk ac
           float x[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = src[(8 * ac + e) * D + n];
@@ -701,54 +771,59 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
             lo[e] = ptx::pack_bf16x2(x[2 * e] - ptx::bf16_lo(hi[e]),
                                      x[2 * e + 1] - ptx::bf16_hi(hi[e]));
           }
-          const uint32_t off = (ac >> 3) * SHALF + n * 128 + (((ac & 7) ^ (n & 7)) << 4);
-          ptx::st_shared_v4(Shi + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-          ptx::st_shared_v4(Slo + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+          const uint32_t kof = (ac >> 3) * SHALF, sw = ((ac & 7) ^ (n & 7)) << 4;
+          ptx::st_shared_v4(Sb + kof + n * 128 + sw, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+          ptx::st_shared_v4(Sb + kof + (D + n) * 128 + sw,
+                            make_uint4(lo[0], lo[1], lo[2], lo[3]));
         }
         if (tt < D) s_z[tt] = src[D * D + tt];
         ptx::fence_proxy_async();
-        ptx::bar_sync(1, kTcMath);
+        ptx::bar_sync(1, kMath);
 #pragma unroll
         for (int e = 0; e < 8; ++e) zc[e] = s_z[8 * c + e];
-        cur_seg = seg;
+        cur_seg = it.seg;
       }
-      bool ok = wait_bounded(full_bar(s), (uint32_t)((j / stages) & 1), flag, kFlagApplyTimeout,
-                             &s_abort);
-      if (!ptx::bar_all(1, kTcMath, ok)) { alive = false; break; }
-      const int rows = min(TM, L - tile * TM);
-      const uint32_t qt = base + s * TILE_BYTES + half * HALF_BYTES;
-      Pos p = {0, 0, 0};
-      if (rope.on) {
-        const int blk = seg - (seg / nblk) * nblk;
-        p = pos_of(rope, (long long)blk * L + (long long)tile * TM + row0);
-      }
-#pragma unroll 2
-      for (int i = 0; i < NI; ++i) {
-        const int r = row0 + i * RPT;
-        const uint32_t addr = qt + r * 128 + ((cc ^ (r & 7)) << 4);
-        const uint4 raw = ptx::ld_shared_v4(addr);
-        float f[8];
-        const float2* cs = nullptr;
-        if (rope.on && r < rows) {
-          const int pos = cr.ax == 0 ? p.tl : (cr.ax == 1 ? p.h : p.w);
-          cs = s_tab + cr.base + pos * cr.stride;
+      const bool ok = wait_bounded(full_bar(it.stage), it.phase, flag, kFlagApplyTimeout,
+                                   &s_abort);
+      if (ok) {
+        const int rows = min(TM, L - it.tile * TM);
+        const uint32_t qt = base + it.stage * TILE_BYTES + half * HALF_BYTES;
+        RopeRun rr;
+        if (rope.on) {
+          const int blk = it.seg - (it.seg / nblk) * nblk;
+          rope_run_start(rr, rope, c, (long long)blk * L + (long long)it.tile * TM + row_first);
         }
-        const uint4 o = relu_rope_chunk(raw, cs, f);
-        float d = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) d = fmaf(f[e], zc[e], d);
+        for (int i = 0; i < RT; ++i) {
+          const int r = row_first + i;
+          const uint32_t addr = qt + r * 128 + ((cc ^ (r & 7)) << 4);
+          const uint4 raw = ptx::ld_shared_v4(addr);
+          const bool rot = rope.on && r < rows;
+          if (rot) rope_run_load(rr, s_tab);
+          float f[8];
+          const uint4 o = phi_rope(raw, rot, rr.c01, rr.c23, f);
+          float d = 0.f;
 #pragma unroll
-        for (int o2 = 1; o2 < CPR; o2 <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
-        if (c == 0) s_den[s * TM + r] = d + eps;
-        ptx::st_shared_v4(addr, o);
-        if (rope.on) pos_advance(rope, p, RPT);
+          for (int e = 0; e < 8; ++e) d = fmaf(f[e], zc[e], d);
+#pragma unroll
+          for (int o2 = 1; o2 < CPR; o2 <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
+          if (c == 0) s_den[it.stage * TM + r] = d + eps;
+          ptx::st_shared_v4(addr, o);
+          if (rope.on) rope_run_next(rr, rope);
+        }
+        ptx::fence_proxy_async();
+        ptx::mbar_arrive(qready_bar(it.stage));
       }
-      ptx::fence_proxy_async();
-      ptx::mbar_arrive(qready_bar(s));
-      if (pend >= 0 && !epilogue(pend)) { alive = false; break; }
-      pend = j;
+      if (pend_stage >= 0) epilogue(pend_stage, pend_b, pend_bph);
+      pend_stage = it.stage;
+      pend_b = b;
+      pend_bph = bph;
+      if (++b == 2) {
+        b = 0;
+        bph ^= 1u;
+      }
     }
-    if (alive && pend >= 0) epilogue(pend);
+    if (pend_stage >= 0) epilogue(pend_stage, pend_b, pend_bph);
   }
   __syncthreads();
   if (warp == 1) {
@@ -832,7 +907,7 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   const StatePlan p1 = state_plan(D, entries, s1);
   if ((st = tc_smem_attr(state_build_tc<D>, p1.total)) != LA_OK) return st;
   if ((st = tc_mark(a, 0)) != LA_OK) return st;
-  state_build_tc<D><<<sc.G, kTcThreads, p1.total, a.stream>>>(mk, mv, a.rope, sc, s1, a.part,
+  state_build_tc<D><<<sc.G, kTcThreadsState, p1.total, a.stream>>>(mk, mv, a.rope, sc, s1, a.part,
                                                               a.gtab, a.flag);
   if ((st = tc_check_launch()) != LA_OK) return st;
   if ((st = tc_mark(a, 1)) != LA_OK) return st;
