@@ -15,6 +15,29 @@ namespace la {
 // Upper bound on the cos/sin table of one call (float2 entries, 48 KB).
 constexpr int kMaxRopeEntries = 6144;
 
+// Division by a runtime constant d >= 1 for dividends 0 <= n < 2^31:
+// n / d == (n * m) >> p with p = 31 + ceil(log2 d), m = ceil(2^p / d) (the
+// rounding-up method of Granlund and Montgomery, exact in this range).
+struct FastDiv {
+  unsigned long long m;
+  int p;
+  int d;
+};
+
+inline FastDiv make_fastdiv(int d) {
+  FastDiv f;
+  int l = 0;
+  while ((1LL << l) < d) ++l;
+  f.p = 31 + l;
+  f.m = (unsigned long long)((((unsigned __int128)1 << f.p) + (unsigned)d - 1) / (unsigned)d);
+  f.d = d;
+  return f;
+}
+
+__host__ __device__ __forceinline__ int fdiv(const FastDiv& f, int n) {
+  return (int)(((unsigned long long)(unsigned)n * f.m) >> f.p);
+}
+
 // Geometry of the 3D rotary embedding for one call. The D dims are split into
 // t | h | w segments; segment a holds half[a] rotation pairs. The table holds
 // (cos, sin) for every (axis, position, pair): t positions are the call's
@@ -28,6 +51,8 @@ struct Rope {
   int tab_off[3];    // first table entry of each axis
   int entries;       // table size in float2
   double theta;
+  FastDiv div_hw;    // by Hg * Wg
+  FastDiv div_w;     // by Wg
 };
 
 // Work schedule of the state build. The tokens of every head are cut into

@@ -125,6 +125,8 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
     r.tab_off[2] = r.tab_off[1] + r.Hg * r.half[1];
     r.entries = r.tab_off[2] + r.Wg * r.half[2];
     r.theta = p->rope_theta;
+    r.div_hw = make_fastdiv(r.Hg * r.Wg);
+    r.div_w = make_fastdiv(r.Wg);
   }
 
   Sched& sc = pl->sc;

@@ -164,12 +164,11 @@ struct Pos {
   int tl, h, w;
 };
 
-__device__ __forceinline__ Pos pos_of(const Rope& r, long long n) {
+__device__ __forceinline__ Pos pos_of(const Rope& r, int n) {
   Pos p;
-  const long long hw = (long long)r.Hg * r.Wg;
-  p.tl = (int)(n / hw);
-  const int rem = (int)(n - (long long)p.tl * hw);
-  p.h = rem / r.Wg;
+  p.tl = fdiv(r.div_hw, n);
+  const int rem = n - p.tl * r.div_hw.d;
+  p.h = fdiv(r.div_w, rem);
   p.w = rem - p.h * r.Wg;
   return p;
 }
@@ -235,73 +234,68 @@ struct TileIter {
   }
 };
 
-// Rotation factors of one chunk (4 pairs) for a run of consecutive tokens.
-// The t and h factors are reloaded only when the token's frame or row
-// changes; the w factors change every token.
+// Rotation factors of one 16-byte chunk (4 pairs, all on one axis) along a
+// run of consecutive tokens: the table row is picked by the token's position
+// on that axis, stepped without branches. Positions past the grid (rows of a
+// ragged tile, which hold zeros) are clamped into the table.
 struct RopeRun {
-  int ax, base, stride;
+  int ax, base, stride, maxpos;
   int tl, h, w;
-  int last_pos;
-  float4 c01, c23;
 };
 
-__device__ __forceinline__ void rope_run_start(RopeRun& rr, const Rope& r, int chunk, long long n) {
+__device__ __forceinline__ void rope_run_init(RopeRun& rr, const Rope& r, int chunk) {
   const ChunkRope c = chunk_rope(r, chunk);
   rr.ax = c.ax;
   rr.base = c.base;
   rr.stride = c.stride;
+  rr.maxpos = c.ax == 0 ? r.T - 1 : (c.ax == 1 ? r.Hg - 1 : r.Wg - 1);
+}
+
+__device__ __forceinline__ void rope_run_seek(RopeRun& rr, const Rope& r, int n) {
   const Pos p = pos_of(r, n);
   rr.tl = p.tl;
   rr.h = p.h;
   rr.w = p.w;
-  rr.last_pos = -1;
 }
 
-__device__ __forceinline__ void rope_run_load(RopeRun& rr, const float2* tab) {
-  const int pos = rr.ax == 0 ? rr.tl : (rr.ax == 1 ? rr.h : rr.w);
-  if (pos != rr.last_pos) {
-    const float4* t4 = reinterpret_cast<const float4*>(tab + rr.base + pos * rr.stride);
-    rr.c01 = t4[0];
-    rr.c23 = t4[1];
-    rr.last_pos = pos;
-  }
+__device__ __forceinline__ const float4* rope_run_ptr(const RopeRun& rr, const float2* tab) {
+  int pos = rr.ax == 0 ? rr.tl : (rr.ax == 1 ? rr.h : rr.w);
+  pos = min(pos, rr.maxpos);
+  return reinterpret_cast<const float4*>(tab + rr.base + pos * rr.stride);
 }
 
-__device__ __forceinline__ void rope_run_next(RopeRun& rr, const Rope& r) {
-  if (++rr.w == r.Wg) {
-    rr.w = 0;
-    if (++rr.h == r.Hg) {
-      rr.h = 0;
-      ++rr.tl;
-    }
-  }
+__device__ __forceinline__ void rope_run_step(RopeRun& rr, const Rope& r) {
+  const int w = rr.w + 1;
+  const int wrap_w = w == r.Wg;
+  rr.w = wrap_w ? 0 : w;
+  const int h = rr.h + wrap_w;
+  const int wrap_h = h == r.Hg;
+  rr.h = wrap_h ? 0 : h;
+  rr.tl += wrap_h;
 }
 
-// phi = ReLU on 8 bf16 values, optionally the rotation of the 4 pairs; the
-// un-rotated phi values come back in f[] (fp32).
-__device__ __forceinline__ uint4 phi_rope(uint4 raw, bool rotate, const float4& c01,
-                                          const float4& c23, float (&f)[8]) {
+// phi = ReLU on 8 bf16 values (packed max with 0, exact in bf16), then, with
+// ROPE, the rotation of the 4 pairs by the (cos, sin) at cs. The un-rotated
+// phi values come back in f[] (fp32).
+template <bool ROPE>
+__device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, float (&f)[8]) {
   const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t m[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    // ReLU on the packed pair: max(x, 0) in bf16 is exact
-    uint32_t m;
-    asm("max.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(w4[j]), "r"(0u));
-    f[2 * j] = ptx::bf16_lo(m);
-    f[2 * j + 1] = ptx::bf16_hi(m);
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m[j]) : "r"(w4[j]), "r"(0u));
+    f[2 * j] = ptx::bf16_lo(m[j]);
+    f[2 * j + 1] = ptx::bf16_hi(m[j]);
   }
+  if (!ROPE) return make_uint4(m[0], m[1], m[2], m[3]);
+  const float4 c01 = cs[0], c23 = cs[1];
+  const float cv[4] = {c01.x, c01.z, c23.x, c23.z};
+  const float sv[4] = {c01.y, c01.w, c23.y, c23.w};
   uint32_t o[4];
-  if (rotate) {
-    const float cs[4] = {c01.x, c01.z, c23.x, c23.z};
-    const float sn[4] = {c01.y, c01.w, c23.y, c23.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float x = f[2 * j], y = f[2 * j + 1];
-      o[j] = ptx::pack_bf16x2(fmaf(x, cs[j], -y * sn[j]), fmaf(x, sn[j], y * cs[j]));
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) o[j] = ptx::pack_bf16x2(f[2 * j], f[2 * j + 1]);
+  for (int j = 0; j < 4; ++j) {
+    const float x = f[2 * j], y = f[2 * j + 1];
+    o[j] = ptx::pack_bf16x2(fmaf(x, cv[j], -y * sv[j]), fmaf(x, sv[j], y * cv[j]));
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -310,7 +304,7 @@ __device__ __forceinline__ uint4 phi_rope(uint4 raw, bool rotate, const float4& 
 
 constexpr int kTcThreadsState = 64 + kMath;  // warp 0 TMA, warp 1 MMA, warps 2-9 math
 
-template <int D>
+template <int D, bool ROPE>
 __global__ void __launch_bounds__(kTcThreadsState, 1)
 state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                Rope rope, Sched sc, int stages, float* __restrict__ partials,
@@ -435,7 +429,9 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     const int tt = threadIdx.x - 64;
     const int mw = warp - 2;                     // math warp 0..7
     const int c = tt % CPR, half = c >> 3, cc = c & 7, k = tt / CPR;
-    if (rope.on) {
+    RopeRun rr;
+    if (ROPE) rope_run_init(rr, rope, c);
+    if (ROPE) {
       for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = rope_entry(rope, e);
       ptx::bar_sync(1, kMath);
       const int e0 = (int)((long long)cta * rope.entries / gridDim.x);
@@ -453,26 +449,22 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const bool ok = wait_bounded(full_bar(it.stage), it.phase, flag, kFlagStateTimeout,
                                    &s_abort);
       if (ok) {
-        const int rows = min(TT, sc.L - it.tile * TT);
         const uint32_t kt = base + it.stage * STAGE_BYTES + half * HALF_BYTES;
-        RopeRun rr;
-        if (rope.on) {
+        if (ROPE) {
           const int blk = it.seg - (it.seg / sc.nblk) * sc.nblk;
-          rope_run_start(rr, rope, c, (long long)blk * sc.L + (long long)it.tile * TT + RT * k);
+          rope_run_seek(rr, rope, blk * sc.L + it.tile * TT + RT * k);
         }
 #pragma unroll
         for (int i = 0; i < RT; ++i) {
           const int r = RT * k + i;
           const uint32_t addr = kt + r * 128 + ((cc ^ (r & 7)) << 4);
           const uint4 raw = ptx::ld_shared_v4(addr);
-          const bool rot = rope.on && r < rows;
-          if (rot) rope_run_load(rr, s_tab);
           float f[8];
-          const uint4 o = phi_rope(raw, rot, rr.c01, rr.c23, f);
+          const uint4 o = phi_rope<ROPE>(raw, ROPE ? rope_run_ptr(rr, s_tab) : nullptr, f);
 #pragma unroll
           for (int e = 0; e < 8; ++e) z[e] += f[e];
           ptx::st_shared_v4(addr, o);
-          if (rope.on) rope_run_next(rr, rope);
+          if (ROPE) rope_run_step(rr, rope);
         }
         ptx::fence_proxy_async();
         ptx::mbar_arrive(kready_bar(it.stage));
@@ -538,7 +530,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
 constexpr int kTcThreadsApply = 96 + kMath;  // warp 0 load, 1 MMA, 2-9 math, 10 store
 
-template <int D, bool GATE>
+template <int D, bool ROPE, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
          const __grid_constant__ CUtensorMap tm_o, Rope rope, int L, int nblk, long long U,
@@ -689,8 +681,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     // the epilogue reads come from the two warps that share the quadrant
     const int c = lane % CPR, half = c >> 3, cc = c & 7;
     const int row_first = 32 * q4 + 16 * pw + RT * (lane / CPR);
-    if (rope.on)
+    RopeRun rr;
+    if (ROPE) {
+      rope_run_init(rr, rope, c);
       for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = gtab[e];
+    }
     const uint32_t tmem = *s_tmem;
     const int erow = 32 * q4 + lane;   // epilogue row = TMEM lane
     float zc[8];
@@ -786,22 +781,18 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       const bool ok = wait_bounded(full_bar(it.stage), it.phase, flag, kFlagApplyTimeout,
                                    &s_abort);
       if (ok) {
-        const int rows = min(TM, L - it.tile * TM);
         const uint32_t qt = base + it.stage * TILE_BYTES + half * HALF_BYTES;
-        RopeRun rr;
-        if (rope.on) {
+        if (ROPE) {
           const int blk = it.seg - (it.seg / nblk) * nblk;
-          rope_run_start(rr, rope, c, (long long)blk * L + (long long)it.tile * TM + row_first);
+          rope_run_seek(rr, rope, blk * L + it.tile * TM + row_first);
         }
 #pragma unroll
         for (int i = 0; i < RT; ++i) {
           const int r = row_first + i;
           const uint32_t addr = qt + r * 128 + ((cc ^ (r & 7)) << 4);
           const uint4 raw = ptx::ld_shared_v4(addr);
-          const bool rot = rope.on && r < rows;
-          if (rot) rope_run_load(rr, s_tab);
           float f[8];
-          const uint4 o = phi_rope(raw, rot, rr.c01, rr.c23, f);
+          const uint4 o = phi_rope<ROPE>(raw, ROPE ? rope_run_ptr(rr, s_tab) : nullptr, f);
           float d = 0.f;
 #pragma unroll
           for (int e = 0; e < 8; ++e) d = fmaf(f[e], zc[e], d);
@@ -809,7 +800,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           for (int o2 = 1; o2 < CPR; o2 <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
           if (c == 0) s_den[it.stage * TM + r] = d + eps;
           ptx::st_shared_v4(addr, o);
-          if (rope.on) rope_run_next(rr, rope);
+          if (ROPE) rope_run_step(rr, rope);
         }
         ptx::fence_proxy_async();
         ptx::mbar_arrive(qready_bar(it.stage));
@@ -905,10 +896,11 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   la_status st;
   const int s1 = pick_state_stages(D, entries);
   const StatePlan p1 = state_plan(D, entries, s1);
-  if ((st = tc_smem_attr(state_build_tc<D>, p1.total)) != LA_OK) return st;
+  auto k1 = a.rope.on ? state_build_tc<D, true> : state_build_tc<D, false>;
+  if ((st = tc_smem_attr(k1, p1.total)) != LA_OK) return st;
   if ((st = tc_mark(a, 0)) != LA_OK) return st;
-  state_build_tc<D><<<sc.G, kTcThreadsState, p1.total, a.stream>>>(mk, mv, a.rope, sc, s1, a.part,
-                                                              a.gtab, a.flag);
+  k1<<<sc.G, kTcThreadsState, p1.total, a.stream>>>(mk, mv, a.rope, sc, s1, a.part, a.gtab,
+                                                    a.flag);
   if ((st = tc_check_launch()) != LA_OK) return st;
   if ((st = tc_mark(a, 1)) != LA_OK) return st;
   dim3 g2((D * (D + 1) + 255) / 256, (unsigned)(a.heads < 65535 ? a.heads : 65535));
@@ -927,15 +919,11 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3);
   const long long U3 = (long long)sc.nseg * ((sc.L + kApplyTile - 1) / kApplyTile);
   const int G3 = (int)(U3 < sms ? U3 : sms);
-  if (gate) {
-    if ((st = tc_smem_attr(apply_tc<D, true>, p3.total)) != LA_OK) return st;
-    apply_tc<D, true><<<G3, kTcThreadsApply, p3.total, a.stream>>>(
-        mq, mg, mo, a.rope, sc.L, sc.nblk, U3, s3, a.apply, a.gtab, a.eps, a.flag);
-  } else {
-    if ((st = tc_smem_attr(apply_tc<D, false>, p3.total)) != LA_OK) return st;
-    apply_tc<D, false><<<G3, kTcThreadsApply, p3.total, a.stream>>>(
-        mq, mg, mo, a.rope, sc.L, sc.nblk, U3, s3, a.apply, a.gtab, a.eps, a.flag);
-  }
+  auto k3 = a.rope.on ? (gate ? apply_tc<D, true, true> : apply_tc<D, true, false>)
+                      : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
+  if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
+  k3<<<G3, kTcThreadsApply, p3.total, a.stream>>>(mq, mg, mo, a.rope, sc.L, sc.nblk, U3, s3,
+                                                  a.apply, a.gtab, a.eps, a.flag);
   if ((st = tc_check_launch()) != LA_OK) return st;
   return tc_mark(a, 3);
 }
