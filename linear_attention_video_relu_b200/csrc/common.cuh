@@ -47,6 +47,8 @@ struct Rope {
   int T, Hg, Wg;
   int t_offset;
   int half[3];       // pairs per axis (d_axis / 2)
+  int stride[3];     // table entries per position (half, padded so that a
+                     // position step is an odd number of 16-byte units)
   int pair_base[3];  // first pair index of each axis
   int tab_off[3];    // first table entry of each axis
   int entries;       // table size in float2
@@ -89,14 +91,35 @@ __host__ __device__ inline long long slot_index(const Sched& s, int seg, int cta
 
 // ---- RoPE table ----------------------------------------------------------
 
+// Table stride for an axis with `half` pairs: half rounded up so that one
+// position step spans an odd number of 16-byte units (conflict-free loads of
+// consecutive positions). Zero-width axes keep stride 0.
+__host__ __device__ inline int rope_stride(int half) {
+  if (half == 0) return 0;
+  int units = (half + 1) / 2;
+  if ((units & 1) == 0) ++units;
+  return 2 * units;
+}
+
+// Inverse frequencies theta^(-2m/d) of the pairs of every axis, written to
+// inv[pair index] (at most 64 pairs); computed once per CTA.
+__device__ inline double rope_inv_freq(const Rope& r, int p) {
+  int ax = p < r.pair_base[1] ? 0 : (p < r.pair_base[2] ? 1 : 2);
+  int m = p - r.pair_base[ax];
+  return pow(r.theta, -(double)m / (double)r.half[ax]);  // -2m/d
+}
+
 // (cos, sin) of table entry e. The angle pos * theta^(-2m/d) is formed and
 // reduced to [-pi, pi] in double, then sincosf runs on the reduced value.
-__device__ inline float2 rope_entry(const Rope& r, int e) {
+// inv holds the inverse frequency of every pair (rope_inv_freq). Padding
+// entries get (1, 0).
+__device__ inline float2 rope_entry(const Rope& r, const double* inv, int e) {
   int ax = e < r.tab_off[1] ? 0 : (e < r.tab_off[2] ? 1 : 2);
   int local = e - r.tab_off[ax];
-  int pos = local / r.half[ax];
-  int m = local - pos * r.half[ax];
-  double inv_freq = pow(r.theta, -(double)m / (double)r.half[ax]);  // -2m/d
+  int pos = local / r.stride[ax];
+  int m = local - pos * r.stride[ax];
+  if (m >= r.half[ax]) return make_float2(1.f, 0.f);
+  double inv_freq = inv[r.pair_base[ax] + m];
   double ang = (double)(pos + (ax == 0 ? r.t_offset : 0)) * inv_freq;
   double red = ang - 6.283185307179586476925 * rint(ang * 0.159154943091895335769);
   float s, c;
@@ -110,7 +133,7 @@ __device__ inline int rope_index(const Rope& r, int p, int tl, int h, int w) {
   int ax = p < r.pair_base[1] ? 0 : (p < r.pair_base[2] ? 1 : 2);
   int m = p - r.pair_base[ax];
   int pos = ax == 0 ? tl : (ax == 1 ? h : w);
-  return r.tab_off[ax] + pos * r.half[ax] + m;
+  return r.tab_off[ax] + pos * r.stride[ax] + m;
 }
 
 // ---- element access --------------------------------------------------------

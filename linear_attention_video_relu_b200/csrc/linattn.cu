@@ -76,9 +76,9 @@ la_status check_params(const la_params* p, bool one_block) {
     if (p->grid_t < 1 || p->grid_h < 1 || p->grid_w < 1) return LA_ERR_INVALID_ARG;
     if ((long long)p->grid_t * p->grid_h * p->grid_w != (long long)p->N) return LA_ERR_INVALID_ARG;
     if (!(p->rope_theta > 0.0) || isinf(p->rope_theta)) return LA_ERR_INVALID_ARG;
-    long long entries = (long long)p->grid_t * (p->rope_dt / 2) +
-                        (long long)p->grid_h * (p->rope_dh / 2) +
-                        (long long)p->grid_w * (p->rope_dw / 2);
+    long long entries = (long long)p->grid_t * rope_stride(p->rope_dt / 2) +
+                        (long long)p->grid_h * rope_stride(p->rope_dh / 2) +
+                        (long long)p->grid_w * rope_stride(p->rope_dw / 2);
     if (entries > kMaxRopeEntries) return LA_ERR_UNSUPPORTED;
   }
   long long heads = (long long)p->B * p->H;
@@ -87,8 +87,9 @@ la_status check_params(const la_params* p, bool one_block) {
 }
 
 bool want_tc(const la_params* p) {
-  const int entries = p->rope ? p->grid_t * (p->rope_dt / 2) + p->grid_h * (p->rope_dh / 2) +
-                                    p->grid_w * (p->rope_dw / 2)
+  const int entries = p->rope ? p->grid_t * rope_stride(p->rope_dt / 2) +
+                                    p->grid_h * rope_stride(p->rope_dh / 2) +
+                                    p->grid_w * rope_stride(p->rope_dw / 2)
                               : 0;
   return tc_supported(p->dtype == LA_BF16, p->D, p->rope, p->rope_dt, p->rope_dh, p->rope_dw,
                       entries);
@@ -120,10 +121,11 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
     r.pair_base[0] = 0;
     r.pair_base[1] = r.half[0];
     r.pair_base[2] = r.half[0] + r.half[1];
+    for (int a = 0; a < 3; ++a) r.stride[a] = rope_stride(r.half[a]);
     r.tab_off[0] = 0;
-    r.tab_off[1] = r.T * r.half[0];
-    r.tab_off[2] = r.tab_off[1] + r.Hg * r.half[1];
-    r.entries = r.tab_off[2] + r.Wg * r.half[2];
+    r.tab_off[1] = r.T * r.stride[0];
+    r.tab_off[2] = r.tab_off[1] + r.Hg * r.stride[1];
+    r.entries = r.tab_off[2] + r.Wg * r.stride[2];
     r.theta = p->rope_theta;
     r.div_hw = make_fastdiv(r.Hg * r.Wg);
     r.div_w = make_fastdiv(r.Wg);

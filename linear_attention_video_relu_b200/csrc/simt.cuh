@@ -46,7 +46,10 @@ state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N
   const int cta = blockIdx.x;
 
   if (rope.on) {
-    for (int e = tid; e < rope.entries; e += kSimtThreads) s_tab[e] = rope_entry(rope, e);
+    __shared__ double s_inv[64];
+    if (tid < D / 2) s_inv[tid] = rope_inv_freq(rope, tid);
+    __syncthreads();
+    for (int e = tid; e < rope.entries; e += kSimtThreads) s_tab[e] = rope_entry(rope, s_inv, e);
     __syncthreads();
     int e0 = (int)((long long)cta * rope.entries / gridDim.x);
     int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);

@@ -83,7 +83,7 @@ __host__ __device__ inline StatePlan state_plan(int D, int entries, int stages) 
   p.off_tab = off;
   off = align_up(off + entries * 8u, 32);
   p.off_z = off;
-  off += 8u * D * 4;  // z of each math warp
+  off += 16u * 8 * 4;  // z of each math warp (8 values)
   p.off_bar = align_up(off, 8);
   off = p.off_bar + (3u * stages + 5u) * 8u;
   p.off_tmem = off;
@@ -102,7 +102,7 @@ __host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, in
   p.off_S = align_up(off, 1024);
   off = p.off_S + 2u * D * D * 2;  // B operand: S_hi^T and S_lo^T rows
   p.off_den = off;
-  off += stages * kApplyTile * 4u;
+  off += stages * (D / 8) * kApplyTile * 4u;
   p.off_z = off;
   off += D * 4u;
   p.off_tab = align_up(off, 32);
@@ -202,8 +202,8 @@ __device__ __forceinline__ ChunkRope chunk_rope(const Rope& r, int chunk) {
 
 // ---- shared pieces of the two kernels --------------------------------------------
 
-constexpr int kMathWarps = 8;
-constexpr int kMath = 32 * kMathWarps;  // threads of the math warps (warps 2 .. 9)
+constexpr int kMathWarps = 16;
+constexpr int kMath = 32 * kMathWarps;  // threads of the math warps (warps 2 .. 17)
 
 // Walks a CTA's contiguous tile range: segment, tile in segment, ring stage
 // and phase, all advanced incrementally (no division inside the loops).
@@ -234,44 +234,34 @@ struct TileIter {
   }
 };
 
-// Rotation factors of one 16-byte chunk (4 pairs, all on one axis) along a
-// run of consecutive tokens: the table row is picked by the token's position
-// on that axis, stepped without branches. Positions past the grid (rows of a
-// ragged tile, which hold zeros) are clamped into the table.
-struct RopeRun {
+// A math warp owns one 16-byte chunk column (8 dims = 4 rotation pairs, all on
+// one axis) and its lanes walk consecutive token rows. These are the chunk's
+// constants: where its pairs sit in the cos/sin table and how far a token
+// may go along its axis (zero-filled rows past the grid are clamped).
+struct ChunkCol {
   int ax, base, stride, maxpos;
-  int tl, h, w;
 };
 
-__device__ __forceinline__ void rope_run_init(RopeRun& rr, const Rope& r, int chunk) {
-  const ChunkRope c = chunk_rope(r, chunk);
-  rr.ax = c.ax;
-  rr.base = c.base;
-  rr.stride = c.stride;
-  rr.maxpos = c.ax == 0 ? r.T - 1 : (c.ax == 1 ? r.Hg - 1 : r.Wg - 1);
+__device__ __forceinline__ ChunkCol chunk_col(const Rope& r, int chunk) {
+  ChunkCol c;
+  const int p0 = 4 * chunk;
+  c.ax = p0 < r.pair_base[1] ? 0 : (p0 < r.pair_base[2] ? 1 : 2);
+  c.stride = r.stride[c.ax];
+  c.base = r.tab_off[c.ax] + (p0 - r.pair_base[c.ax]);
+  c.maxpos = c.ax == 0 ? r.T - 1 : (c.ax == 1 ? r.Hg - 1 : r.Wg - 1);
+  return c;
 }
 
-__device__ __forceinline__ void rope_run_seek(RopeRun& rr, const Rope& r, int n) {
-  const Pos p = pos_of(r, n);
-  rr.tl = p.tl;
-  rr.h = p.h;
-  rr.w = p.w;
-}
-
-__device__ __forceinline__ const float4* rope_run_ptr(const RopeRun& rr, const float2* tab) {
-  int pos = rr.ax == 0 ? rr.tl : (rr.ax == 1 ? rr.h : rr.w);
-  pos = min(pos, rr.maxpos);
-  return reinterpret_cast<const float4*>(tab + rr.base + pos * rr.stride);
-}
-
-__device__ __forceinline__ void rope_run_step(RopeRun& rr, const Rope& r) {
-  const int w = rr.w + 1;
-  const int wrap_w = w == r.Wg;
-  rr.w = wrap_w ? 0 : w;
-  const int h = rr.h + wrap_w;
-  const int wrap_h = h == r.Hg;
-  rr.h = wrap_h ? 0 : h;
-  rr.tl += wrap_h;
+// (cos, sin) of the chunk's 4 pairs for token n of the head.
+__device__ __forceinline__ const float4* chunk_cs(const ChunkCol& cc, const Rope& r,
+                                                  const float2* tab, int n) {
+  const int tl = fdiv(r.div_hw, n);
+  const int rem = n - tl * r.div_hw.d;
+  const int h = fdiv(r.div_w, rem);
+  const int w = rem - h * r.Wg;
+  int pos = cc.ax == 0 ? tl : (cc.ax == 1 ? h : w);
+  pos = min(pos, cc.maxpos);
+  return reinterpret_cast<const float4*>(tab + cc.base + pos * cc.stride);
 }
 
 // phi = ReLU on 8 bf16 values (packed max with 0, exact in bf16), then, with
@@ -300,9 +290,39 @@ __device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, float (&f
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Builds the CTA's cos/sin table in shared memory (all math threads), then
+// synchronises them.
+__device__ __forceinline__ void build_rope_table(const Rope& r, float2* tab, double* inv, int tt,
+                                                 int D) {
+  if (tt < D / 2) inv[tt] = rope_inv_freq(r, tt);
+  ptx::bar_sync(1, kMath);
+  for (int e = tt; e < r.entries; e += kMath) tab[e] = rope_entry(r, inv, e);
+  ptx::bar_sync(1, kMath);
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* v);
+
+template <>
+__device__ __forceinline__ void tmem_ld_cols<32>(uint32_t taddr, uint32_t* v) {
+  ptx::tmem_ld_32x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 // ---- state build ------------------------------------------------------------------
 
-constexpr int kTcThreadsState = 64 + kMath;  // warp 0 TMA, warp 1 MMA, warps 2-9 math
+constexpr int kTcThreadsState = 64 + kMath;  // warp 0 TMA, warp 1 MMA, warps 2-17 math
 
 template <int D, bool ROPE>
 __global__ void __launch_bounds__(kTcThreadsState, 1)
@@ -315,18 +335,20 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   constexpr int TILE_BYTES = HALVES * HALF_BYTES;
   constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   constexpr int CPR = D / 8;                  // 16-byte chunks per row
-  constexpr int RT = TT * CPR / kMath;        // consecutive rows per thread (4)
+  constexpr int WPC = kMathWarps / CPR;       // warps per chunk column
+  constexpr int IPW = TT / 32 / WPC;          // 32-row groups per warp and tile
   constexpr int KSTEPS = TT / 16;             // MMAs per tile
   constexpr int DD1 = D * (D + 1);
   constexpr uint32_t IDESC = ptx::idesc_bf16_f32(D, D, 1, 1);
   constexpr uint32_t TMEM_COLS = 2 * D;
-  static_assert(RT * kMath == TT * CPR, "tile must split evenly over the math threads");
+  constexpr int ECOLS = D / 4;                // epilogue columns per warp
+  static_assert(WPC >= 1 && IPW * WPC * 32 == TT, "tile must split over the math warps");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
   const uint32_t base = align_up(raw_addr, 1024);
   uint8_t* sm = smem_raw + (base - raw_addr);
-  const StatePlan P = state_plan(D, rope.on ? rope.entries : 0, stages);
+  const StatePlan P = state_plan(D, ROPE ? rope.entries : 0, stages);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
   float* s_z = reinterpret_cast<float*>(sm + P.off_z);
   const uint32_t bar0 = base + P.off_bar;
@@ -338,6 +360,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   const uint32_t done_bar = bar0 + 8u * (3 * stages + 4);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P.off_tmem);
   __shared__ int s_abort;
+  __shared__ double s_inv[64];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int cta = blockIdx.x;
@@ -427,17 +450,17 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   } else {
     // ---------------- math warps: ReLU + RoPE, z, epilogue ----------------
     const int tt = threadIdx.x - 64;
-    const int mw = warp - 2;                     // math warp 0..7
-    const int c = tt % CPR, half = c >> 3, cc = c & 7, k = tt / CPR;
-    RopeRun rr;
-    if (ROPE) rope_run_init(rr, rope, c);
+    const int mw = warp - 2;                     // math warp 0..15
+    const int c = mw % CPR, rg0 = mw / CPR;      // chunk column, first row group
+    const int half = c >> 3, cc = c & 7;
     if (ROPE) {
-      for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = rope_entry(rope, e);
-      ptx::bar_sync(1, kMath);
+      build_rope_table(rope, s_tab, s_inv, tt, D);
       const int e0 = (int)((long long)cta * rope.entries / gridDim.x);
       const int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);
       for (int e = e0 + tt; e < e1; e += kMath) gtab[e] = s_tab[e];
     }
+    ChunkCol col{};
+    if (ROPE) col = chunk_col(rope, c);
     const uint32_t tmem = *s_tmem;
     float z[8];
 #pragma unroll
@@ -450,21 +473,19 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                                    &s_abort);
       if (ok) {
         const uint32_t kt = base + it.stage * STAGE_BYTES + half * HALF_BYTES;
-        if (ROPE) {
-          const int blk = it.seg - (it.seg / sc.nblk) * sc.nblk;
-          rope_run_seek(rr, rope, blk * sc.L + it.tile * TT + RT * k);
-        }
+        const int blk = ROPE ? it.seg - (it.seg / sc.nblk) * sc.nblk : 0;
+        const int n0 = blk * sc.L + it.tile * TT;
 #pragma unroll
-        for (int i = 0; i < RT; ++i) {
-          const int r = RT * k + i;
+        for (int i = 0; i < IPW; ++i) {
+          const int r = 32 * (rg0 + WPC * i) + lane;
           const uint32_t addr = kt + r * 128 + ((cc ^ (r & 7)) << 4);
           const uint4 raw = ptx::ld_shared_v4(addr);
           float f[8];
-          const uint4 o = phi_rope<ROPE>(raw, ROPE ? rope_run_ptr(rr, s_tab) : nullptr, f);
+          const uint4 o =
+              phi_rope<ROPE>(raw, ROPE ? chunk_cs(col, rope, s_tab, n0 + r) : nullptr, f);
 #pragma unroll
           for (int e = 0; e < 8; ++e) z[e] += f[e];
           ptx::st_shared_v4(addr, o);
-          if (ROPE) rope_run_step(rr, rope);
         }
         ptx::fence_proxy_async();
         ptx::mbar_arrive(kready_bar(it.stage));
@@ -476,39 +497,37 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                                         kFlagStateTimeout, &s_abort);
         ptx::tc_fence_after();
         float* slot = partials + slot_index(sc, it.seg, cta) * DD1;
-        const int q = warp & 3, pw = mw >> 2;    // lane quadrant, column half
+        const int q = warp & 3, quarter = mw >> 2;   // lane quadrant, column quarter
         // M = 64 keeps rows in lanes 0-15 of each 32-lane quadrant; M = 128
         // uses all 128 lanes, row = lane.
         const int row = D == 64 ? 16 * q + lane : 32 * q + lane;
         const bool has_row = D == 64 ? lane < 16 : true;
+        const int col0 = quarter * ECOLS;
+        uint32_t v[ECOLS];
+        tmem_ld_cols<ECOLS>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * D + col0), v);
+        ptx::tmem_wait_ld();
+        if (ready && has_row) {
+          float4* dst = reinterpret_cast<float4*>(slot + (size_t)row * D + col0);
 #pragma unroll
-        for (int cj = 0; cj < D / 64; ++cj) {
-          const int col = pw * (D / 2) + 32 * cj;
-          uint32_t v[32];
-          ptx::tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * D + col), v);
-          ptx::tmem_wait_ld();
-          if (ready && has_row) {
-            float4* dst = reinterpret_cast<float4*>(slot + (size_t)row * D + col);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                   __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-          }
+          for (int e = 0; e < ECOLS / 4; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         }
-        // z: the threads of one chunk within a warp, then the 8 warps in order
+        // z: the 32 lanes of a warp, then the warps of a chunk column in order
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float t = z[e];
 #pragma unroll
-          for (int o = CPR; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
           z[e] = 0.f;
-          if (lane < CPR) s_z[mw * D + 8 * lane + e] = t;
+          if (lane == 0) s_z[mw * 8 + e] = t;
         }
         ptx::bar_sync(1, kMath);
         if (tt < D && ready) {
+          const int ch = tt >> 3, e = tt & 7;
           float t = 0.f;
 #pragma unroll
-          for (int w = 0; w < kMathWarps; ++w) t += s_z[w * D + tt];
+          for (int g = 0; g < WPC; ++g) t += s_z[(g * CPR + ch) * 8 + e];
           slot[D * D + tt] = t;
         }
         ptx::bar_sync(1, kMath);
@@ -528,7 +547,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
 // ---- apply ---------------------------------------------------------------------------
 
-constexpr int kTcThreadsApply = 96 + kMath;  // warp 0 load, 1 MMA, 2-9 math, 10 store
+constexpr int kTcThreadsApply = 96 + kMath;  // warp 0 load, 1 MMA, 2-17 math, 18 store
 
 template <int D, bool ROPE, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
@@ -543,24 +562,25 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   constexpr int NB = 2 * D;                  // B operand rows: S_hi^T then S_lo^T
   constexpr int SHALF = NB * 128;            // one K-half of the B operand
   constexpr int CPR = D / 8;
-  constexpr int RT = TM * CPR / kMath;       // consecutive rows per thread (4 or 8)
+  constexpr int WPC = kMathWarps / CPR;      // warps per chunk column
+  constexpr int IPW = TM / 32 / WPC;         // 32-row groups per warp and tile
   constexpr int KSTEPS = D / 16;
   constexpr int DD1 = D * (D + 1);
   constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, NB, 0, 0);
   constexpr uint32_t TMEM_COLS = 2 * NB;
   constexpr uint32_t TX = (GATE ? 2 : 1) * TILE_BYTES;
-  constexpr int EC = D / 2;                  // epilogue columns per thread
-  static_assert(RT * kMath == TM * CPR, "tile must split evenly over the math threads");
+  constexpr int EC = D / 4;                  // epilogue columns per thread
+  static_assert(WPC >= 1 && IPW * WPC * 32 == TM, "tile must split over the math warps");
   const int tps = (L + TM - 1) / TM;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
   const uint32_t base = align_up(raw_addr, 1024);
   uint8_t* sm = smem_raw + (base - raw_addr);
-  const ApplyPlan P = apply_plan(D, rope.on ? rope.entries : 0, GATE ? 1 : 0, stages);
+  const ApplyPlan P = apply_plan(D, ROPE ? rope.entries : 0, GATE ? 1 : 0, stages);
   const uint32_t gbase = base + P.off_g;
   const uint32_t Sb = base + P.off_S;
-  float* s_den = reinterpret_cast<float*>(sm + P.off_den);
+  float* s_den = reinterpret_cast<float*>(sm + P.off_den);   // [stage][chunk][row]
   float* s_z = reinterpret_cast<float*>(sm + P.off_z);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
   const uint32_t bar0 = base + P.off_bar;
@@ -676,48 +696,50 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     // ---------------- math warps: phi(q), den, RoPE; epilogue ----------------
     const int tt = threadIdx.x - 64;
     const int mw = warp - 2;
-    const int q4 = warp & 3, pw = mw >> 2;   // TMEM lane quadrant, column half
-    // a warp transforms 16 rows of its own lane quadrant, so the den values
-    // the epilogue reads come from the two warps that share the quadrant
-    const int c = lane % CPR, half = c >> 3, cc = c & 7;
-    const int row_first = 32 * q4 + 16 * pw + RT * (lane / CPR);
-    RopeRun rr;
-    if (ROPE) {
-      rope_run_init(rr, rope, c);
+    const int c = mw % CPR, rg0 = mw / CPR;      // chunk column, first row group
+    const int half = c >> 3, cc = c & 7;
+    const int q4 = warp & 3, quarter = mw >> 2;  // TMEM lane quadrant, column quarter
+    const int erow = 32 * q4 + lane;             // epilogue row = TMEM lane
+    if (ROPE)
       for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = gtab[e];
-    }
+    ChunkCol col{};
+    if (ROPE) col = chunk_col(rope, c);
     const uint32_t tmem = *s_tmem;
-    const int erow = 32 * q4 + lane;   // epilogue row = TMEM lane
     float zc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) zc[e] = 0.f;
     int cur_seg = -1;
     int pend_stage = -1, pend_b = 0;
-    uint32_t pend_bph = 0;
+    uint32_t pend_bph = 0, pend_ph = 0;
     int b = 0;
     uint32_t bph = 0;
 
     // out = (acc_hi + acc_lo) / den (* sigmoid(g)) as bf16, over the q tile
-    auto epilogue = [&](int s, int eb, uint32_t ebph) {
-      const bool ready = wait_bounded(accf_bar(eb), ebph, flag, kFlagApplyTimeout, &s_abort);
-      ptx::bar_sync(2 + q4, 64);   // den of this quadrant's rows is in shared memory
+    auto epilogue = [&](int s, uint32_t sph, int eb, uint32_t ebph) {
+      // all den partials of the tile are in shared memory once every math
+      // thread has arrived on the tile's qready barrier
+      const bool seen = wait_bounded(qready_bar(s), sph, flag, kFlagApplyTimeout, &s_abort);
+      const bool ready =
+          wait_bounded(accf_bar(eb), ebph, flag, kFlagApplyTimeout, &s_abort) && seen;
       ptx::tc_fence_after();
-      const float inv = 1.f / s_den[s * TM + erow];
+      float den = eps;
+      const float* dp = s_den + s * CPR * TM + erow;
+#pragma unroll
+      for (int ch = 0; ch < CPR; ++ch) den += dp[ch * TM];
+      const float inv = 1.f / den;
       const uint32_t qt = base + s * TILE_BYTES;
       const uint32_t gt = gbase + s * TILE_BYTES;
       const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(eb * NB);
+      const int col0 = quarter * EC;
+      uint32_t vh[EC], vl[EC];
+      tmem_ld_cols<EC>(lane_base + col0, vh);
+      tmem_ld_cols<EC>(lane_base + D + col0, vl);
+      ptx::tmem_wait_ld();
+      if (ready) {
+        const int h = col0 / 64;
 #pragma unroll
-      for (int cj = 0; cj < EC / 32; ++cj) {
-        const int col = pw * EC + 32 * cj;
-        uint32_t vh[32], vl[32];
-        ptx::tmem_ld_32x32(lane_base + col, vh);
-        ptx::tmem_ld_32x32(lane_base + D + col, vl);
-        ptx::tmem_wait_ld();
-        if (!ready) continue;
-        const int h = col / 64;
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int chunk = (col % 64) / 8 + k4;
+        for (int k4 = 0; k4 < EC / 8; ++k4) {
+          const int chunk = (col0 % 64) / 8 + k4;
           const uint32_t off = h * HALF_BYTES + erow * 128 + ((chunk ^ (erow & 7)) << 4);
           float o[8];
 #pragma unroll
@@ -750,7 +772,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       if (it.seg != cur_seg) {
         // every MMA that reads the current S must be done before it is replaced
         if (pend_stage >= 0) {
-          epilogue(pend_stage, pend_b, pend_bph);
+          epilogue(pend_stage, pend_ph, pend_b, pend_bph);
           pend_stage = -1;
         }
         const float* src = apply + (long long)it.seg * DD1;
@@ -782,31 +804,29 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                                    &s_abort);
       if (ok) {
         const uint32_t qt = base + it.stage * TILE_BYTES + half * HALF_BYTES;
-        if (ROPE) {
-          const int blk = it.seg - (it.seg / nblk) * nblk;
-          rope_run_seek(rr, rope, blk * L + it.tile * TM + row_first);
-        }
+        const int blk = ROPE ? it.seg - (it.seg / nblk) * nblk : 0;
+        const int n0 = blk * L + it.tile * TM;
+        float* dst_den = s_den + (it.stage * CPR + c) * TM;
 #pragma unroll
-        for (int i = 0; i < RT; ++i) {
-          const int r = row_first + i;
+        for (int i = 0; i < IPW; ++i) {
+          const int r = 32 * (rg0 + WPC * i) + lane;
           const uint32_t addr = qt + r * 128 + ((cc ^ (r & 7)) << 4);
           const uint4 raw = ptx::ld_shared_v4(addr);
           float f[8];
-          const uint4 o = phi_rope<ROPE>(raw, ROPE ? rope_run_ptr(rr, s_tab) : nullptr, f);
+          const uint4 o =
+              phi_rope<ROPE>(raw, ROPE ? chunk_cs(col, rope, s_tab, n0 + r) : nullptr, f);
           float d = 0.f;
 #pragma unroll
           for (int e = 0; e < 8; ++e) d = fmaf(f[e], zc[e], d);
-#pragma unroll
-          for (int o2 = 1; o2 < CPR; o2 <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
-          if (c == 0) s_den[it.stage * TM + r] = d + eps;
+          dst_den[r] = d;
           ptx::st_shared_v4(addr, o);
-          if (ROPE) rope_run_step(rr, rope);
         }
         ptx::fence_proxy_async();
         ptx::mbar_arrive(qready_bar(it.stage));
       }
-      if (pend_stage >= 0) epilogue(pend_stage, pend_b, pend_bph);
+      if (pend_stage >= 0) epilogue(pend_stage, pend_ph, pend_b, pend_bph);
       pend_stage = it.stage;
+      pend_ph = it.phase;
       pend_b = b;
       pend_bph = bph;
       if (++b == 2) {
@@ -814,7 +834,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         bph ^= 1u;
       }
     }
-    if (pend_stage >= 0) epilogue(pend_stage, pend_b, pend_bph);
+    if (pend_stage >= 0) epilogue(pend_stage, pend_ph, pend_b, pend_bph);
   }
   __syncthreads();
   if (warp == 1) {
