@@ -55,6 +55,7 @@ struct Rope {
   double theta;
   FastDiv div_hw;    // by Hg * Wg
   FastDiv div_w;     // by Wg
+  double inv_freq[64];  // theta^(-2m/d) of every pair, in pair order
 };
 
 // Work schedule of the state build. The tokens of every head are cut into
@@ -101,27 +102,23 @@ __host__ __device__ inline int rope_stride(int half) {
   return 2 * units;
 }
 
-// Inverse frequencies theta^(-2m/d) of the pairs of every axis, written to
-// inv[pair index] (at most 64 pairs); computed once per CTA.
-__device__ inline double rope_inv_freq(const Rope& r, int p) {
-  int ax = p < r.pair_base[1] ? 0 : (p < r.pair_base[2] ? 1 : 2);
-  int m = p - r.pair_base[ax];
-  return pow(r.theta, -(double)m / (double)r.half[ax]);  // -2m/d
-}
-
 // (cos, sin) of table entry e. The angle pos * theta^(-2m/d) is formed and
 // reduced to [-pi, pi] in double, then sincosf runs on the reduced value.
-// inv holds the inverse frequency of every pair (rope_inv_freq). Padding
+// inv holds theta^(-2m/d) of every pair (a copy of Rope::inv_freq). Padding
 // entries get (1, 0).
 __device__ inline float2 rope_entry(const Rope& r, const double* inv, int e) {
-  int ax = e < r.tab_off[1] ? 0 : (e < r.tab_off[2] ? 1 : 2);
-  int local = e - r.tab_off[ax];
-  int pos = local / r.stride[ax];
-  int m = local - pos * r.stride[ax];
-  if (m >= r.half[ax]) return make_float2(1.f, 0.f);
-  double inv_freq = inv[r.pair_base[ax] + m];
-  double ang = (double)(pos + (ax == 0 ? r.t_offset : 0)) * inv_freq;
-  double red = ang - 6.283185307179586476925 * rint(ang * 0.159154943091895335769);
+  int base = 0, stride = r.stride[0], half = r.half[0], pb = 0, toff = r.t_offset;
+  if (e >= r.tab_off[2]) {
+    base = r.tab_off[2]; stride = r.stride[2]; half = r.half[2]; pb = r.pair_base[2]; toff = 0;
+  } else if (e >= r.tab_off[1]) {
+    base = r.tab_off[1]; stride = r.stride[1]; half = r.half[1]; pb = r.pair_base[1]; toff = 0;
+  }
+  const int local = e - base;
+  const int pos = local / stride;
+  const int m = local - pos * stride;
+  if (m >= half) return make_float2(1.f, 0.f);
+  const double ang = (double)(pos + toff) * inv[pb + m];
+  const double red = fma(-6.283185307179586476925, rint(ang * 0.159154943091895335769), ang);
   float s, c;
   sincosf((float)red, &s, &c);
   return make_float2(c, s);

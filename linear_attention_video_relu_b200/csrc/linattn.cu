@@ -129,6 +129,10 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
     r.theta = p->rope_theta;
     r.div_hw = make_fastdiv(r.Hg * r.Wg);
     r.div_w = make_fastdiv(r.Wg);
+    // constants of the rotary parameterisation: theta^(-2m/d) per pair
+    for (int a = 0; a < 3; ++a)
+      for (int m = 0; m < r.half[a]; ++m)
+        r.inv_freq[r.pair_base[a] + m] = pow(r.theta, -(double)m / (double)r.half[a]);
   }
 
   Sched& sc = pl->sc;

@@ -47,7 +47,7 @@ state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N
 
   if (rope.on) {
     __shared__ double s_inv[64];
-    if (tid < D / 2) s_inv[tid] = rope_inv_freq(rope, tid);
+    if (tid < D / 2) s_inv[tid] = rope.inv_freq[tid];
     __syncthreads();
     for (int e = tid; e < rope.entries; e += kSimtThreads) s_tab[e] = rope_entry(rope, s_inv, e);
     __syncthreads();

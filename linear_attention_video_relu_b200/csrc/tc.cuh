@@ -65,12 +65,12 @@ constexpr int kApplyTile = 128;
 
 struct StatePlan {
   int stages;
-  uint32_t off_tab, off_z, off_bar, off_tmem, total;
+  uint32_t off_tab, off_pos, off_z, off_bar, off_tmem, total;
 };
 
 struct ApplyPlan {
   int stages;
-  uint32_t off_g, off_S, off_den, off_z, off_tab, off_bar, off_tmem, total;
+  uint32_t off_g, off_S, off_den, off_z, off_tab, off_pos, off_bar, off_tmem, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -82,6 +82,8 @@ __host__ __device__ inline StatePlan state_plan(int D, int entries, int stages) 
   uint32_t off = stages * stage_bytes;
   p.off_tab = off;
   off = align_up(off + entries * 8u, 32);
+  p.off_pos = off;  // per stage: table row offset of each token row, per axis
+  off += entries ? stages * 3u * tc_state_tile_c(D) * 4 : 0;
   p.off_z = off;
   off += 16u * 8 * 4;  // z of each math warp (8 values)
   p.off_bar = align_up(off, 8);
@@ -107,6 +109,8 @@ __host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, in
   off += D * 4u;
   p.off_tab = align_up(off, 32);
   off = p.off_tab + entries * 8u;
+  p.off_pos = align_up(off, 16);
+  off = p.off_pos + (entries ? stages * 3u * kApplyTile * 4 : 0);
   p.off_bar = align_up(off, 8);
   off = p.off_bar + (4u * stages + 5u) * 8u;
   p.off_tmem = off;
@@ -122,7 +126,7 @@ inline int pick_state_stages(int D, int entries) {
 }
 
 inline int pick_apply_stages(int D, int entries, int gate) {
-  for (int s = 4; s >= 2; --s)
+  for (int s = 8; s >= 2; --s)
     if (apply_plan(D, entries, gate, s).total <= (uint32_t)kSmemBudget) return s;
   return 0;
 }
@@ -235,47 +239,52 @@ struct TileIter {
 };
 
 // A math warp owns one 16-byte chunk column (8 dims = 4 rotation pairs, all on
-// one axis) and its lanes walk consecutive token rows. These are the chunk's
-// constants: where its pairs sit in the cos/sin table and how far a token
-// may go along its axis (zero-filled rows past the grid are clamped).
+// one axis) and its lanes walk consecutive token rows. The TMA warp writes,
+// for every row of a tile, the table offset of the row's position on each
+// axis (clamped into the table for zero-filled rows past the grid); a chunk
+// adds its first pair's index within the axis.
 struct ChunkCol {
-  int ax, base, stride, maxpos;
+  int ax, pair_off;
 };
 
 __device__ __forceinline__ ChunkCol chunk_col(const Rope& r, int chunk) {
   ChunkCol c;
   const int p0 = 4 * chunk;
   c.ax = p0 < r.pair_base[1] ? 0 : (p0 < r.pair_base[2] ? 1 : 2);
-  c.stride = r.stride[c.ax];
-  c.base = r.tab_off[c.ax] + (p0 - r.pair_base[c.ax]);
-  c.maxpos = c.ax == 0 ? r.T - 1 : (c.ax == 1 ? r.Hg - 1 : r.Wg - 1);
+  c.pair_off = p0 - (c.ax == 0 ? 0 : (c.ax == 1 ? r.pair_base[1] : r.pair_base[2]));
   return c;
 }
 
-// (cos, sin) of the chunk's 4 pairs for token n of the head.
-__device__ __forceinline__ const float4* chunk_cs(const ChunkCol& cc, const Rope& r,
-                                                  const float2* tab, int n) {
-  const int tl = fdiv(r.div_hw, n);
-  const int rem = n - tl * r.div_hw.d;
-  const int h = fdiv(r.div_w, rem);
-  const int w = rem - h * r.Wg;
-  int pos = cc.ax == 0 ? tl : (cc.ax == 1 ? h : w);
-  pos = min(pos, cc.maxpos);
-  return reinterpret_cast<const float4*>(tab + cc.base + pos * cc.stride);
+// Table row offsets (per axis) of rows [0, rows) of a tile whose first token
+// is n0, written by the 32 lanes of the TMA warp.
+__device__ __forceinline__ void write_row_offsets(const Rope& r, int* pos, int rows, int n0,
+                                                  int lane) {
+  for (int row = lane; row < rows; row += 32) {
+    const int n = n0 + row;
+    const int tl = fdiv(r.div_hw, n);
+    const int rem = n - tl * r.div_hw.d;
+    const int h = fdiv(r.div_w, rem);
+    const int w = rem - h * r.Wg;
+    pos[row] = r.tab_off[0] + min(tl, r.T - 1) * r.stride[0];
+    pos[rows + row] = r.tab_off[1] + h * r.stride[1];
+    pos[2 * rows + row] = r.tab_off[2] + w * r.stride[2];
+  }
 }
 
 // phi = ReLU on 8 bf16 values (packed max with 0, exact in bf16), then, with
 // ROPE, the rotation of the 4 pairs by the (cos, sin) at cs. The un-rotated
-// phi values come back in f[] (fp32).
+// phi values come back as 4 packed fp32 pairs.
 template <bool ROPE>
-__device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, float (&f)[8]) {
+__device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, uint64_t (&f)[4]) {
   const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
   uint32_t m[4];
+  float x[4], y[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     asm("max.bf16x2 %0, %1, %2;" : "=r"(m[j]) : "r"(w4[j]), "r"(0u));
-    f[2 * j] = ptx::bf16_lo(m[j]);
-    f[2 * j + 1] = ptx::bf16_hi(m[j]);
+    x[j] = ptx::bf16_lo(m[j]);
+    y[j] = ptx::bf16_hi(m[j]);
+    f[j] = ptx::f2(x[j], y[j]);
   }
   if (!ROPE) return make_uint4(m[0], m[1], m[2], m[3]);
   const float4 c01 = cs[0], c23 = cs[1];
@@ -283,10 +292,8 @@ __device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, float (&f
   const float sv[4] = {c01.y, c01.w, c23.y, c23.w};
   uint32_t o[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float x = f[2 * j], y = f[2 * j + 1];
-    o[j] = ptx::pack_bf16x2(fmaf(x, cv[j], -y * sv[j]), fmaf(x, sv[j], y * cv[j]));
-  }
+  for (int j = 0; j < 4; ++j)
+    o[j] = ptx::pack_bf16x2(fmaf(x[j], cv[j], -y[j] * sv[j]), fmaf(x[j], sv[j], y[j] * cv[j]));
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
@@ -294,7 +301,7 @@ __device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, float (&f
 // synchronises them.
 __device__ __forceinline__ void build_rope_table(const Rope& r, float2* tab, double* inv, int tt,
                                                  int D) {
-  if (tt < D / 2) inv[tt] = rope_inv_freq(r, tt);
+  if (tt < D / 2) inv[tt] = r.inv_freq[tt];
   ptx::bar_sync(1, kMath);
   for (int e = tt; e < r.entries; e += kMath) tab[e] = rope_entry(r, inv, e);
   ptx::bar_sync(1, kMath);
@@ -350,6 +357,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   uint8_t* sm = smem_raw + (base - raw_addr);
   const StatePlan P = state_plan(D, ROPE ? rope.entries : 0, stages);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
+  int* s_pos = reinterpret_cast<int*>(sm + P.off_pos);
   float* s_z = reinterpret_cast<float*>(sm + P.off_z);
   const uint32_t bar0 = base + P.off_bar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -387,14 +395,21 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   __syncthreads();
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      TileIter it;
-      it.init(u0, sc.tps, stages);
-      long long issued = 0;
-      for (long long u = u0; u < u1; ++u, it.next()) {
-        if (!wait_bounded(empty_bar(it.stage), it.phase ^ 1u, flag, kFlagStateTimeout, &s_abort))
-          break;
+    // ---------------- TMA producer (+ row offsets of the RoPE table) ----------------
+    TileIter it;
+    it.init(u0, sc.tps, stages);
+    long long issued = 0;
+    for (long long u = u0; u < u1; ++u, it.next()) {
+      int ok = 1;
+      if (lane == 0)
+        ok = wait_bounded(empty_bar(it.stage), it.phase ^ 1u, flag, kFlagStateTimeout, &s_abort);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (ROPE) {
+        const int blk = it.seg - (it.seg / sc.nblk) * sc.nblk;
+        write_row_offsets(rope, s_pos + it.stage * 3 * TT, TT, blk * sc.L + it.tile * TT, lane);
+        __syncwarp();
+      }
+      if (lane == 0) {
         const uint32_t kt = base + it.stage * STAGE_BYTES, vt = kt + TILE_BYTES;
         ptx::mbar_expect_tx(full_bar(it.stage), STAGE_BYTES);
 #pragma unroll
@@ -404,13 +419,14 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           ptx::tma_load_3d(vt + h * HALF_BYTES, &tm_v, 64 * h, it.tile * TT, it.seg,
                            full_bar(it.stage));
         }
-        ++issued;
       }
-      // drain: every issued copy has landed before the CTA may exit
+      ++issued;
+    }
+    // drain: every issued copy has landed before the CTA may exit
+    if (lane == 0)
       for (long long i = issued - stages < 0 ? 0 : issued - stages; i < issued; ++i)
         wait_bounded(full_bar((int)(i % stages)), (uint32_t)((i / stages) & 1), flag,
                      kFlagStateTimeout, &s_abort);
-    }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -462,9 +478,9 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     ChunkCol col{};
     if (ROPE) col = chunk_col(rope, c);
     const uint32_t tmem = *s_tmem;
-    float z[8];
+    uint64_t z2[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) z[e] = 0.f;
+    for (int e = 0; e < 4; ++e) z2[e] = ptx::f2(0.f, 0.f);
     TileIter it;
     it.init(u0, sc.tps, stages);
     int sidx = 0;
@@ -473,18 +489,18 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                                    &s_abort);
       if (ok) {
         const uint32_t kt = base + it.stage * STAGE_BYTES + half * HALF_BYTES;
-        const int blk = ROPE ? it.seg - (it.seg / sc.nblk) * sc.nblk : 0;
-        const int n0 = blk * sc.L + it.tile * TT;
+        const int* rowoff = s_pos + (it.stage * 3 + col.ax) * TT;
 #pragma unroll
         for (int i = 0; i < IPW; ++i) {
           const int r = 32 * (rg0 + WPC * i) + lane;
           const uint32_t addr = kt + r * 128 + ((cc ^ (r & 7)) << 4);
           const uint4 raw = ptx::ld_shared_v4(addr);
-          float f[8];
-          const uint4 o =
-              phi_rope<ROPE>(raw, ROPE ? chunk_cs(col, rope, s_tab, n0 + r) : nullptr, f);
+          uint64_t f[4];
+          const float4* cs =
+              ROPE ? reinterpret_cast<const float4*>(s_tab + rowoff[r] + col.pair_off) : nullptr;
+          const uint4 o = phi_rope<ROPE>(raw, cs, f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) z[e] += f[e];
+          for (int e = 0; e < 4; ++e) z2[e] = ptx::add2(z2[e], f[e]);
           ptx::st_shared_v4(addr, o);
         }
         ptx::fence_proxy_async();
@@ -514,12 +530,17 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                                  __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         }
         // z: the 32 lanes of a warp, then the warps of a chunk column in order
+        float z[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          ptx::f2_split(z2[e], z[2 * e], z[2 * e + 1]);
+          z2[e] = ptx::f2(0.f, 0.f);
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float t = z[e];
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          z[e] = 0.f;
           if (lane == 0) s_z[mw * 8 + e] = t;
         }
         ptx::bar_sync(1, kMath);
@@ -552,9 +573,10 @@ constexpr int kTcThreadsApply = 96 + kMath;  // warp 0 load, 1 MMA, 2-17 math, 1
 template <int D, bool ROPE, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
-         const __grid_constant__ CUtensorMap tm_o, Rope rope, int L, int nblk, long long U,
-         int stages, const float* __restrict__ apply, const float2* __restrict__ gtab, float eps,
-         int* flag) {
+         const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ Rope rope, int L,
+         int nblk, long long U, int stages, const float* __restrict__ apply,
+         const float* __restrict__ partials, const __grid_constant__ Sched ssc, int direct,
+         const float2* __restrict__ gtab, float eps, int* flag) {
   constexpr int TM = kApplyTile;
   constexpr int HALVES = D / 64;
   constexpr int HALF_BYTES = TM * 128;
@@ -583,6 +605,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   float* s_den = reinterpret_cast<float*>(sm + P.off_den);   // [stage][chunk][row]
   float* s_z = reinterpret_cast<float*>(sm + P.off_z);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
+  int* s_pos = reinterpret_cast<int*>(sm + P.off_pos);
   const uint32_t bar0 = base + P.off_bar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto qready_bar = [&](int s) { return bar0 + 8u * (stages + s); };
@@ -620,14 +643,21 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   __syncthreads();
 
   if (warp == 0) {
-    // ---------------- TMA loads: q (and gate) tiles ----------------
-    if (lane == 0) {
-      TileIter it;
-      it.init(u0, tps, stages);
-      long long issued = 0;
-      for (long long u = u0; u < u1; ++u, it.next()) {
-        if (!wait_bounded(empty_bar(it.stage), it.phase ^ 1u, flag, kFlagApplyTimeout, &s_abort))
-          break;
+    // ---------------- TMA loads: q (and gate) tiles, RoPE row offsets ----------------
+    TileIter it;
+    it.init(u0, tps, stages);
+    long long issued = 0;
+    for (long long u = u0; u < u1; ++u, it.next()) {
+      int ok = 1;
+      if (lane == 0)
+        ok = wait_bounded(empty_bar(it.stage), it.phase ^ 1u, flag, kFlagApplyTimeout, &s_abort);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (ROPE) {
+        const int blk = it.seg - (it.seg / nblk) * nblk;
+        write_row_offsets(rope, s_pos + it.stage * 3 * TM, TM, blk * L + it.tile * TM, lane);
+        __syncwarp();
+      }
+      if (lane == 0) {
         ptx::mbar_expect_tx(full_bar(it.stage), TX);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h) {
@@ -637,12 +667,13 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
             ptx::tma_load_3d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h,
                              it.tile * TM, it.seg, full_bar(it.stage));
         }
-        ++issued;
       }
+      ++issued;
+    }
+    if (lane == 0)
       for (long long i = issued - stages < 0 ? 0 : issued - stages; i < issued; ++i)
         wait_bounded(full_bar((int)(i % stages)), (uint32_t)((i / stages) & 1), flag,
                      kFlagApplyTimeout, &s_abort);
-    }
   } else if (warp == 1) {
     // ---------------- MMA issuer: acc[b] = RoPE(phi q) [S_hi | S_lo] ----------------
     if (lane == 0) {
@@ -705,9 +736,9 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     ChunkCol col{};
     if (ROPE) col = chunk_col(rope, c);
     const uint32_t tmem = *s_tmem;
-    float zc[8];
+    uint64_t zc2[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) zc[e] = 0.f;
+    for (int e = 0; e < 4; ++e) zc2[e] = ptx::f2(0.f, 0.f);
     int cur_seg = -1;
     int pend_stage = -1, pend_b = 0;
     uint32_t pend_bph = 0, pend_ph = 0;
@@ -727,6 +758,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
 #pragma unroll
       for (int ch = 0; ch < CPR; ++ch) den += dp[ch * TM];
       const float inv = 1.f / den;
+      const uint64_t inv2 = ptx::f2(inv, inv);
       const uint32_t qt = base + s * TILE_BYTES;
       const uint32_t gt = gbase + s * TILE_BYTES;
       const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(eb * NB);
@@ -743,8 +775,13 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           const uint32_t off = h * HALF_BYTES + erow * 128 + ((chunk ^ (erow & 7)) << 4);
           float o[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            o[e] = (__uint_as_float(vh[8 * k4 + e]) + __uint_as_float(vl[8 * k4 + e])) * inv;
+          for (int e = 0; e < 4; ++e) {
+            const uint64_t hv = ptx::f2(__uint_as_float(vh[8 * k4 + 2 * e]),
+                                        __uint_as_float(vh[8 * k4 + 2 * e + 1]));
+            const uint64_t lv = ptx::f2(__uint_as_float(vl[8 * k4 + 2 * e]),
+                                        __uint_as_float(vl[8 * k4 + 2 * e + 1]));
+            ptx::f2_split(ptx::mul2(ptx::add2(hv, lv), inv2), o[2 * e], o[2 * e + 1]);
+          }
           if (GATE) {
             const uint4 gr = ptx::ld_shared_v4(gt + off);
             const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
@@ -775,12 +812,24 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           epilogue(pend_stage, pend_ph, pend_b, pend_bph);
           pend_stage = -1;
         }
+        // S and z of the segment: the reduced state, or (bidirectional, no
+        // carried state) the sum of the state kernel's partials in CTA order
         const float* src = apply + (long long)it.seg * DD1;
+        int nparts = 1;
+        if (direct) {
+          const long long ub = (long long)it.seg * ssc.tps;
+          nparts = cta_of_unit(ssc, ub + ssc.tps - 1) - cta_of_unit(ssc, ub) + 1;
+          src = partials + (long long)it.seg * ssc.maxc * DD1;
+        }
         for (int item = tt; item < D * CPR; item += kMath) {
           const int n = item % D, ac = item / D;    // output column n, K chunk ac
           float x[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = src[(8 * ac + e) * D + n];
+          for (int i = 1; i < nparts; ++i) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] += src[(long long)i * DD1 + (8 * ac + e) * D + n];
+          }
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -793,32 +842,38 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           ptx::st_shared_v4(Sb + kof + (D + n) * 128 + sw,
                             make_uint4(lo[0], lo[1], lo[2], lo[3]));
         }
-        if (tt < D) s_z[tt] = src[D * D + tt];
+        if (tt < D) {
+          float zz = src[D * D + tt];
+          for (int i = 1; i < nparts; ++i) zz += src[(long long)i * DD1 + D * D + tt];
+          s_z[tt] = zz;
+        }
         ptx::fence_proxy_async();
         ptx::bar_sync(1, kMath);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) zc[e] = s_z[8 * c + e];
+        for (int e = 0; e < 4; ++e) zc2[e] = ptx::f2(s_z[8 * c + 2 * e], s_z[8 * c + 2 * e + 1]);
         cur_seg = it.seg;
       }
       const bool ok = wait_bounded(full_bar(it.stage), it.phase, flag, kFlagApplyTimeout,
                                    &s_abort);
       if (ok) {
         const uint32_t qt = base + it.stage * TILE_BYTES + half * HALF_BYTES;
-        const int blk = ROPE ? it.seg - (it.seg / nblk) * nblk : 0;
-        const int n0 = blk * L + it.tile * TM;
+        const int* rowoff = s_pos + (it.stage * 3 + col.ax) * TM;
         float* dst_den = s_den + (it.stage * CPR + c) * TM;
 #pragma unroll
         for (int i = 0; i < IPW; ++i) {
           const int r = 32 * (rg0 + WPC * i) + lane;
           const uint32_t addr = qt + r * 128 + ((cc ^ (r & 7)) << 4);
           const uint4 raw = ptx::ld_shared_v4(addr);
-          float f[8];
-          const uint4 o =
-              phi_rope<ROPE>(raw, ROPE ? chunk_cs(col, rope, s_tab, n0 + r) : nullptr, f);
-          float d = 0.f;
+          uint64_t f[4];
+          const float4* cs =
+              ROPE ? reinterpret_cast<const float4*>(s_tab + rowoff[r] + col.pair_off) : nullptr;
+          const uint4 o = phi_rope<ROPE>(raw, cs, f);
+          uint64_t d2 = ptx::mul2(f[0], zc2[0]);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) d = fmaf(f[e], zc[e], d);
-          dst_den[r] = d;
+          for (int e = 1; e < 4; ++e) d2 = ptx::fma2(f[e], zc2[e], d2);
+          float dlo, dhi;
+          ptx::f2_split(d2, dlo, dhi);
+          dst_den[r] = dlo + dhi;
           ptx::st_shared_v4(addr, o);
         }
         ptx::fence_proxy_async();
@@ -923,10 +978,15 @@ la_status tc_run_d(const TcArgs& a, int sms) {
                                                     a.flag);
   if ((st = tc_check_launch()) != LA_OK) return st;
   if ((st = tc_mark(a, 1)) != LA_OK) return st;
-  dim3 g2((D * (D + 1) + 255) / 256, (unsigned)(a.heads < 65535 ? a.heads : 65535));
-  reduce_states<D><<<g2, 256, 0, a.stream>>>(a.part, sc, a.apply, a.stS, a.stz, a.use_state,
-                                              a.commit);
-  if ((st = tc_check_launch()) != LA_OK) return st;
+  // one segment per head and no carried state: the apply kernel sums the
+  // partials itself (same order as reduce_states) and the reduction is skipped
+  const int direct = (!a.use_state && sc.nblk == 1 && a.do_apply) ? 1 : 0;
+  if (!direct) {
+    dim3 g2((D * (D + 1) + 255) / 256, (unsigned)(a.heads < 65535 ? a.heads : 65535));
+    reduce_states<D><<<g2, 256, 0, a.stream>>>(a.part, sc, a.apply, a.stS, a.stz, a.use_state,
+                                                a.commit);
+    if ((st = tc_check_launch()) != LA_OK) return st;
+  }
   if ((st = tc_mark(a, 2)) != LA_OK) return st;
   if (!a.do_apply) return LA_OK;
 
@@ -943,7 +1003,8 @@ la_status tc_run_d(const TcArgs& a, int sms) {
                       : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
   if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
   k3<<<G3, kTcThreadsApply, p3.total, a.stream>>>(mq, mg, mo, a.rope, sc.L, sc.nblk, U3, s3,
-                                                  a.apply, a.gtab, a.eps, a.flag);
+                                                  a.apply, a.part, sc, direct, a.gtab, a.eps,
+                                                  a.flag);
   if ((st = tc_check_launch()) != LA_OK) return st;
   return tc_mark(a, 3);
 }
