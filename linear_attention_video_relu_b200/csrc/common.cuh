@@ -55,7 +55,11 @@ struct Rope {
   double theta;
   FastDiv div_hw;    // by Hg * Wg
   FastDiv div_w;     // by Wg
-  double inv_freq[64];  // theta^(-2m/d) of every pair, in pair order
+  float rcp_stride[3];  // 1 / stride[a] (exact position recovery for entry < 2^20)
+  // theta^(-2m/d) / pi of every pair (pair order) as an unevaluated float sum
+  // hi + lo, so that position * frequency / pi is formed to ~2^-48 relative
+  float inv_pi_hi[64];
+  float inv_pi_lo[64];
 };
 
 // Work schedule of the state build. The tokens of every head are cut into
@@ -102,25 +106,36 @@ __host__ __device__ inline int rope_stride(int half) {
   return 2 * units;
 }
 
-// (cos, sin) of table entry e. The angle pos * theta^(-2m/d) is formed and
-// reduced to [-pi, pi] in double, then sincosf runs on the reduced value.
-// inv holds theta^(-2m/d) of every pair (a copy of Rope::inv_freq). Padding
-// entries get (1, 0).
-__device__ inline float2 rope_entry(const Rope& r, const double* inv, int e) {
+// (cos, sin) of table entry e: the angle pos * theta^(-2m/d) of its axis
+// position and pair. With x = angle / pi carried as x_hi + x_lo (the product
+// error of x_hi recovered exactly by an FMA), x_hi - 2 rint(x_hi / 2) is exact,
+// so the reduced argument r in [-1, 1] is accurate to a few ulp and
+// sincospif(r) gives cos(angle), sin(angle) to float precision. Padding
+// entries get (1, 0). ih / il are copies of r.inv_pi_hi / r.inv_pi_lo in shared
+// memory (lanes read different pairs; a parameter-space read of a per-lane
+// index would be serialised).
+__device__ inline float2 rope_entry(const Rope& r, const float* ih_tab, const float* il_tab,
+                                    int e) {
   int base = 0, stride = r.stride[0], half = r.half[0], pb = 0, toff = r.t_offset;
+  float rcp = r.rcp_stride[0];
   if (e >= r.tab_off[2]) {
-    base = r.tab_off[2]; stride = r.stride[2]; half = r.half[2]; pb = r.pair_base[2]; toff = 0;
+    base = r.tab_off[2]; stride = r.stride[2]; half = r.half[2]; pb = r.pair_base[2];
+    toff = 0; rcp = r.rcp_stride[2];
   } else if (e >= r.tab_off[1]) {
-    base = r.tab_off[1]; stride = r.stride[1]; half = r.half[1]; pb = r.pair_base[1]; toff = 0;
+    base = r.tab_off[1]; stride = r.stride[1]; half = r.half[1]; pb = r.pair_base[1];
+    toff = 0; rcp = r.rcp_stride[1];
   }
   const int local = e - base;
-  const int pos = local / stride;
+  const int pos = (int)(((float)local + 0.5f) * rcp);
   const int m = local - pos * stride;
   if (m >= half) return make_float2(1.f, 0.f);
-  const double ang = (double)(pos + toff) * inv[pb + m];
-  const double red = fma(-6.283185307179586476925, rint(ang * 0.159154943091895335769), ang);
+  const float P = (float)(pos + toff);                // exact: positions < 2^24
+  const float ih = ih_tab[pb + m], il = il_tab[pb + m];
+  const float x_hi = P * ih;
+  const float x_lo = fmaf(P, ih, -x_hi) + P * il;
+  const float red = (x_hi - 2.f * rintf(0.5f * x_hi)) + x_lo;
   float s, c;
-  sincosf((float)red, &s, &c);
+  sincospif(red, &s, &c);
   return make_float2(c, s);
 }
 

@@ -46,10 +46,14 @@ state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N
   const int cta = blockIdx.x;
 
   if (rope.on) {
-    __shared__ double s_inv[64];
-    if (tid < D / 2) s_inv[tid] = rope.inv_freq[tid];
+    __shared__ float s_ih[64], s_il[64];
+    if (tid < D / 2) {
+      s_ih[tid] = rope.inv_pi_hi[tid];
+      s_il[tid] = rope.inv_pi_lo[tid];
+    }
     __syncthreads();
-    for (int e = tid; e < rope.entries; e += kSimtThreads) s_tab[e] = rope_entry(rope, s_inv, e);
+    for (int e = tid; e < rope.entries; e += kSimtThreads)
+      s_tab[e] = rope_entry(rope, s_ih, s_il, e);
     __syncthreads();
     int e0 = (int)((long long)cta * rope.entries / gridDim.x);
     int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);

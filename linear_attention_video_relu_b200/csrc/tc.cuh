@@ -69,9 +69,15 @@ struct StatePlan {
 };
 
 struct ApplyPlan {
-  int stages;
-  uint32_t off_g, off_S, off_den, off_z, off_tab, off_pos, off_bar, off_tmem, total;
+  int stages, sbuf;
+  uint32_t off_g, off_S, off_den, off_tab, off_pos, off_bar, off_tmem, total;
 };
+
+// Bytes of one segment's B-operand image: S as bf16 hi and lo rows (K-major,
+// 128-byte swizzle, 2D rows of D values) followed by z as D floats. This is
+// exactly the size of a D x (D + 1) fp32 state.
+__host__ __device__ constexpr uint32_t image_bytes(int D) { return 4u * D * (D + 1); }
+__host__ __device__ constexpr uint32_t image_slot(int D) { return (image_bytes(D) + 1023u) / 1024u * 1024u; }
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
@@ -85,34 +91,34 @@ __host__ __device__ inline StatePlan state_plan(int D, int entries, int stages) 
   p.off_pos = off;  // per stage: table row offset of each token row, per axis
   off += entries ? stages * 3u * tc_state_tile_c(D) * 4 : 0;
   p.off_z = off;
-  off += 16u * 8 * 4;  // z of each math warp (8 values)
+  off += 2u * 16 * 8 * 4;  // z of each math warp (8 values), per accumulator buffer
   p.off_bar = align_up(off, 8);
-  off = p.off_bar + (3u * stages + 5u) * 8u;
+  off = p.off_bar + (3u * stages + 9u) * 8u;
   p.off_tmem = off;
   off += 16;
   p.total = off + 1024;  // slack to align the base to 1024 bytes
   return p;
 }
 
-__host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, int stages) {
+__host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, int stages,
+                                                int sbuf) {
   ApplyPlan p;
   const uint32_t tile = (uint32_t)kApplyTile * D * 2;
   p.stages = stages;
+  p.sbuf = sbuf;
   uint32_t off = stages * tile;
   p.off_g = off;
   off += gate ? stages * tile : 0;
   p.off_S = align_up(off, 1024);
-  off = p.off_S + 2u * D * D * 2;  // B operand: S_hi^T and S_lo^T rows
+  off = p.off_S + sbuf * image_slot(D);  // B-operand images, one per S slot
   p.off_den = off;
   off += stages * (D / 8) * kApplyTile * 4u;
-  p.off_z = off;
-  off += D * 4u;
   p.off_tab = align_up(off, 32);
   off = p.off_tab + entries * 8u;
   p.off_pos = align_up(off, 16);
   off = p.off_pos + (entries ? stages * 3u * kApplyTile * 4 : 0);
   p.off_bar = align_up(off, 8);
-  off = p.off_bar + (4u * stages + 5u) * 8u;
+  off = p.off_bar + (4u * stages + 9u) * 8u;
   p.off_tmem = off;
   off += 16;
   p.total = off + 1024;
@@ -125,10 +131,28 @@ inline int pick_state_stages(int D, int entries) {
   return 0;
 }
 
-inline int pick_apply_stages(int D, int entries, int gate) {
+// Two S slots (the next segment's image prefetched while the current one is
+// in use) when at least 4 stages still fit, else one slot and the most stages.
+inline void pick_apply_plan(int D, int entries, int gate, int* stages, int* sbuf) {
+  *stages = 0;
+  *sbuf = 1;
+  for (int s = 8; s >= 4; --s)
+    if (apply_plan(D, entries, gate, s, 2).total <= (uint32_t)kSmemBudget) {
+      *stages = s;
+      *sbuf = 2;
+      return;
+    }
   for (int s = 8; s >= 2; --s)
-    if (apply_plan(D, entries, gate, s).total <= (uint32_t)kSmemBudget) return s;
-  return 0;
+    if (apply_plan(D, entries, gate, s, 1).total <= (uint32_t)kSmemBudget) {
+      *stages = s;
+      return;
+    }
+}
+
+inline int pick_apply_stages(int D, int entries, int gate) {
+  int st, sb;
+  pick_apply_plan(D, entries, gate, &st, &sb);
+  return st;
 }
 
 // Which calls take the tensor-core kernels: bf16 I/O, D in {64, 128}, and RoPE
@@ -299,11 +323,14 @@ __device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, uint64_t 
 
 // Builds the CTA's cos/sin table in shared memory (all math threads), then
 // synchronises them.
-__device__ __forceinline__ void build_rope_table(const Rope& r, float2* tab, double* inv, int tt,
-                                                 int D) {
-  if (tt < D / 2) inv[tt] = r.inv_freq[tt];
+__device__ __forceinline__ void build_rope_table(const Rope& r, float2* tab, int tt) {
+  __shared__ float s_ih[64], s_il[64];
+  if (tt < 64) {
+    s_ih[tt] = r.inv_pi_hi[tt];
+    s_il[tt] = r.inv_pi_lo[tt];
+  }
   ptx::bar_sync(1, kMath);
-  for (int e = tt; e < r.entries; e += kMath) tab[e] = rope_entry(r, inv, e);
+  for (int e = tt; e < r.entries; e += kMath) tab[e] = rope_entry(r, s_ih, s_il, e);
   ptx::bar_sync(1, kMath);
 }
 
@@ -329,13 +356,15 @@ __device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uint32_t* v) {
 
 // ---- state build ------------------------------------------------------------------
 
-constexpr int kTcThreadsState = 64 + kMath;  // warp 0 TMA, warp 1 MMA, warps 2-17 math
+// warp 0 TMA, warp 1 MMA, warps 2-17 math, warps 18-21 epilogue (one per TMEM
+// lane quadrant)
+constexpr int kTcThreadsState = 64 + kMath + 128;
 
 template <int D, bool ROPE>
 __global__ void __launch_bounds__(kTcThreadsState, 1)
 state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               Rope rope, Sched sc, int stages, float* __restrict__ partials,
-               float2* __restrict__ gtab, int* flag) {
+               const __grid_constant__ Rope rope, const __grid_constant__ Sched sc, int stages,
+               float* __restrict__ partials, float2* __restrict__ gtab, int* flag) {
   constexpr int TT = tc_state_tile_c(D);      // tokens per tile
   constexpr int HALVES = D / 64;              // 64-column (128-byte) halves
   constexpr int HALF_BYTES = TT * 128;        // one half of one tensor's tile
@@ -348,7 +377,6 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   constexpr int DD1 = D * (D + 1);
   constexpr uint32_t IDESC = ptx::idesc_bf16_f32(D, D, 1, 1);
   constexpr uint32_t TMEM_COLS = 2 * D;
-  constexpr int ECOLS = D / 4;                // epilogue columns per warp
   static_assert(WPC >= 1 && IPW * WPC * 32 == TT, "tile must split over the math warps");
 
   extern __shared__ uint8_t smem_raw[];
@@ -365,10 +393,11 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   auto empty_bar = [&](int s) { return bar0 + 8u * (2 * stages + s); };
   auto accf_bar = [&](int b) { return bar0 + 8u * (3 * stages + b); };
   auto acce_bar = [&](int b) { return bar0 + 8u * (3 * stages + 2 + b); };
-  const uint32_t done_bar = bar0 + 8u * (3 * stages + 4);
+  auto zrdy_bar = [&](int b) { return bar0 + 8u * (3 * stages + 4 + b); };
+  auto zfree_bar = [&](int b) { return bar0 + 8u * (3 * stages + 6 + b); };
+  const uint32_t done_bar = bar0 + 8u * (3 * stages + 8);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P.off_tmem);
   __shared__ int s_abort;
-  __shared__ double s_inv[64];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int cta = blockIdx.x;
@@ -383,7 +412,9 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(accf_bar(b), 1);
-      ptx::mbar_init(acce_bar(b), kMath);
+      ptx::mbar_init(acce_bar(b), 128);
+      ptx::mbar_init(zrdy_bar(b), kMathWarps);
+      ptx::mbar_init(zfree_bar(b), 128);
     }
     ptx::mbar_init(done_bar, 1);
     ptx::fence_mbar_init();
@@ -393,6 +424,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     ptx::tmem_relinquish();
   }
   __syncthreads();
+  if (threadIdx.x == 0) ptx::launch_dependents();
 
   if (warp == 0) {
     // ---------------- TMA producer (+ row offsets of the RoPE table) ----------------
@@ -463,21 +495,20 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       ptx::mma_commit(done_bar);
       wait_bounded(done_bar, 0, flag, kFlagStateTimeout, &s_abort);
     }
-  } else {
-    // ---------------- math warps: ReLU + RoPE, z, epilogue ----------------
+  } else if (warp < 2 + kMathWarps) {
+    // ---------------- math warps: ReLU + RoPE, z ----------------
     const int tt = threadIdx.x - 64;
     const int mw = warp - 2;                     // math warp 0..15
     const int c = mw % CPR, rg0 = mw / CPR;      // chunk column, first row group
     const int half = c >> 3, cc = c & 7;
     if (ROPE) {
-      build_rope_table(rope, s_tab, s_inv, tt, D);
+      build_rope_table(rope, s_tab, tt);
       const int e0 = (int)((long long)cta * rope.entries / gridDim.x);
       const int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);
       for (int e = e0 + tt; e < e1; e += kMath) gtab[e] = s_tab[e];
     }
     ChunkCol col{};
     if (ROPE) col = chunk_col(rope, c);
-    const uint32_t tmem = *s_tmem;
     uint64_t z2[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) z2[e] = ptx::f2(0.f, 0.f);
@@ -507,55 +538,73 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         ptx::mbar_arrive(kready_bar(it.stage));
       }
       if (it.last_of_segment(u, u1)) {
-        // the segment's partial: TMEM accumulator -> S rows, then z
+        // hand z over to the epilogue warps: this warp's 32 lanes summed, in
+        // the buffer of the segment's accumulator
         const int b = sidx & 1;
-        const bool ready = wait_bounded(accf_bar(b), (uint32_t)((sidx >> 1) & 1), flag,
-                                        kFlagStateTimeout, &s_abort);
-        ptx::tc_fence_after();
-        float* slot = partials + slot_index(sc, it.seg, cta) * DD1;
-        const int q = warp & 3, quarter = mw >> 2;   // lane quadrant, column quarter
-        // M = 64 keeps rows in lanes 0-15 of each 32-lane quadrant; M = 128
-        // uses all 128 lanes, row = lane.
-        const int row = D == 64 ? 16 * q + lane : 32 * q + lane;
-        const bool has_row = D == 64 ? lane < 16 : true;
-        const int col0 = quarter * ECOLS;
-        uint32_t v[ECOLS];
-        tmem_ld_cols<ECOLS>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * D + col0), v);
-        ptx::tmem_wait_ld();
-        if (ready && has_row) {
-          float4* dst = reinterpret_cast<float4*>(slot + (size_t)row * D + col0);
-#pragma unroll
-          for (int e = 0; e < ECOLS / 4; ++e)
-            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-        }
-        // z: the 32 lanes of a warp, then the warps of a chunk column in order
-        float z[8];
+        wait_bounded(zfree_bar(b), (uint32_t)(((sidx >> 1) & 1) ^ 1), flag, kFlagStateTimeout,
+                     &s_abort);
+        float zz[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          ptx::f2_split(z2[e], z[2 * e], z[2 * e + 1]);
+          ptx::f2_split(z2[e], zz[2 * e], zz[2 * e + 1]);
           z2[e] = ptx::f2(0.f, 0.f);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          float t = z[e];
+          float t = zz[e];
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          if (lane == 0) s_z[mw * 8 + e] = t;
+          if (lane == 0) s_z[(b * kMathWarps + mw) * 8 + e] = t;
         }
-        ptx::bar_sync(1, kMath);
-        if (tt < D && ready) {
-          const int ch = tt >> 3, e = tt & 7;
-          float t = 0.f;
-#pragma unroll
-          for (int g = 0; g < WPC; ++g) t += s_z[(g * CPR + ch) * 8 + e];
-          slot[D * D + tt] = t;
-        }
-        ptx::bar_sync(1, kMath);
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(acce_bar(b));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(zrdy_bar(b));
         ++sidx;
       }
+    }
+  } else {
+    // ---------------- epilogue warps: accumulator and z -> the CTA's partial slot ------
+    const int q = warp & 3;             // TMEM lane quadrant of this warp
+    const int te = threadIdx.x - (64 + kMath);
+    const uint32_t tmem = *s_tmem;
+    // M = 64 keeps rows in lanes 0-15 of each 32-lane quadrant; M = 128 uses
+    // all 128 lanes, row = lane.
+    const int row = D == 64 ? 16 * q + lane : 32 * q + lane;
+    const bool has_row = D == 64 ? lane < 16 : true;
+    TileIter it;
+    it.init(u0, sc.tps, 1);
+    int sidx = 0;
+    for (long long u = u0; u < u1; ++u, it.next()) {
+      if (!it.last_of_segment(u, u1)) continue;
+      const int b = sidx & 1;
+      const uint32_t ph = (uint32_t)((sidx >> 1) & 1);
+      const bool ready = wait_bounded(accf_bar(b), ph, flag, kFlagStateTimeout, &s_abort) &&
+                         wait_bounded(zrdy_bar(b), ph, flag, kFlagStateTimeout, &s_abort);
+      ptx::tc_fence_after();
+      float* slot = partials + slot_index(sc, it.seg, cta) * DD1;
+#pragma unroll 1
+      for (int cj = 0; cj < D / 16; ++cj) {
+        uint32_t v[16];
+        tmem_ld_cols<16>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * D + 16 * cj), v);
+        ptx::tmem_wait_ld();
+        if (ready && has_row) {
+          float4* dst = reinterpret_cast<float4*>(slot + (size_t)row * D + 16 * cj);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+      }
+      if (te < D && ready) {
+        const int ch = te >> 3, e = te & 7;
+        float t = 0.f;
+#pragma unroll
+        for (int g = 0; g < WPC; ++g) t += s_z[(b * kMathWarps + g * CPR + ch) * 8 + e];
+        slot[D * D + te] = t;
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(acce_bar(b));
+      ptx::mbar_arrive(zfree_bar(b));
+      ++sidx;
     }
   }
   __syncthreads();
@@ -563,6 +612,186 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     __syncwarp();
     ptx::tc_fence_after();
     ptx::tmem_dealloc(*s_tmem, TMEM_COLS);
+  }
+}
+
+// ---- reduction into B-operand images -------------------------------------------------
+
+// Writes the apply state of segment seg as the image the apply kernel copies
+// into shared memory: S as bf16 hi/lo K-major swizzled rows, z as floats.
+template <int D>
+__device__ __forceinline__ void write_image_chunk(uint8_t* images, int seg, bool zitem, int n,
+                                                  int ac, const float (&v)[8]) {
+  constexpr int SHALF = 2 * D * 128;  // one K-half of the image rows
+  uint8_t* img = images + (long long)seg * image_bytes(D);
+  if (zitem) {
+    float4* zdst = reinterpret_cast<float4*>(img + 4u * D * D + 32u * ac);
+    zdst[0] = make_float4(v[0], v[1], v[2], v[3]);
+    zdst[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      hi[e] = ptx::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+      lo[e] = ptx::pack_bf16x2(v[2 * e] - ptx::bf16_lo(hi[e]), v[2 * e + 1] - ptx::bf16_hi(hi[e]));
+    }
+    const uint32_t o = (ac >> 3) * SHALF + n * 128 + (((ac & 7) ^ (n & 7)) << 4);
+    *reinterpret_cast<uint4*>(img + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(img + o + D * 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
+// Sum of the partials of segment seg at the 8 element offsets off[], in CTA
+// order (the order reduce_states uses).
+template <int D>
+__device__ __forceinline__ void segment_sum(const float* __restrict__ partials, const Sched& sc,
+                                            int seg, const int (&off)[8], float (&blk)[8]) {
+  constexpr int DD1 = D * (D + 1);
+  const long long ub = (long long)seg * sc.tps;
+  const int np = cta_of_unit(sc, ub + sc.tps - 1) - cta_of_unit(sc, ub) + 1;
+  const float* base = partials + (long long)seg * sc.maxc * DD1;
+  // all loads of up to 8 partials are issued before the first add
+  float p[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) p[i][e] = i < np ? base[(long long)i * DD1 + off[e]] : 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) blk[e] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (i < np) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) blk[e] += p[i][e];
+    }
+  for (int i = 8; i < np; ++i) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) blk[e] += base[(long long)i * DD1 + off[e]];
+  }
+}
+
+// Sums of up to 8 consecutive segments (first..first+count-1) at the 8 element
+// offsets, with every load issued before any add; blk[j] for segment first+j.
+// Used by the block-causal scan, whose block sums have at most 2 partials in
+// the common case (more fall back to segment_sum).
+template <int D>
+__device__ __forceinline__ void segment_sums8(const float* __restrict__ partials,
+                                              const Sched& sc, int first, int count,
+                                              const int (&off)[8], float (&blk)[8][8]) {
+  constexpr int DD1 = D * (D + 1);
+  int np[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const long long ub = (long long)(first + j) * sc.tps;
+    np[j] = j < count ? cta_of_unit(sc, ub + sc.tps - 1) - cta_of_unit(sc, ub) + 1 : 0;
+  }
+  float p0[8][8], p1[8][8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float* base = partials + (long long)(first + j) * sc.maxc * DD1;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      p0[j][e] = np[j] > 0 ? base[off[e]] : 0.f;
+      p1[j][e] = np[j] > 1 ? base[DD1 + off[e]] : 0.f;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      blk[j][e] = 0.f;
+      if (np[j] > 0) blk[j][e] += p0[j][e];
+      if (np[j] > 1) blk[j][e] += p1[j][e];
+    }
+    if (np[j] > 2) {
+      const float* base = partials + (long long)(first + j) * sc.maxc * DD1;
+      for (int i = 2; i < np[j]; ++i) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) blk[j][e] += base[(long long)i * DD1 + off[e]];
+      }
+    }
+  }
+}
+
+// One segment per head (bidirectional, or one block with a carried state):
+// apply = run + blk with run the carried state (or zero), the fp32 operations
+// of reduce_states; committed back when asked. One thread per (head, chunk of
+// 8 values): chunk (column n, K chunk ac) of S, or K chunk ac of z.
+template <int D>
+__global__ void __launch_bounds__(64)
+finalize_single(const float* __restrict__ partials, const __grid_constant__ Sched sc,
+                uint8_t* __restrict__ images, float* __restrict__ stS, float* __restrict__ stz,
+                int use_state, int commit) {
+  constexpr int CPR = D / 8, DD = D * D;
+  constexpr int ITEMS = D * CPR + CPR;
+  ptx::grid_dependency_wait();
+  ptx::launch_dependents();
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)sc.nseg * ITEMS) return;
+  const int hh = (int)(gid / ITEMS), item = (int)(gid - (long long)hh * ITEMS);
+  const bool zitem = item >= D * CPR;
+  const int n = zitem ? 0 : item % D;
+  const int ac = zitem ? item - D * CPR : item / D;
+  int off[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) off[e] = zitem ? DD + 8 * ac + e : (8 * ac + e) * D + n;
+  float blk[8], run[8];
+  segment_sum<D>(partials, sc, hh, off, blk);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float r0 = !use_state ? 0.f
+                                : (zitem ? stz[(long long)hh * D + 8 * ac + e]
+                                         : stS[(long long)hh * DD + off[e]]);
+    run[e] = r0 + blk[e];
+  }
+  write_image_chunk<D>(images, hh, zitem, n, ac, run);
+  if (use_state && commit) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (zitem) stz[(long long)hh * D + 8 * ac + e] = run[e];
+      else stS[(long long)hh * DD + off[e]] = run[e];
+    }
+  }
+}
+
+// Several blocks per head (block-causal): the apply state of block b is
+// run + blk(b) with run the sum over blocks 0..b-1, in block order (the same
+// fp32 operations as reduce_states). One thread per (head, 8-value chunk),
+// consecutive threads on consecutive columns so loads coalesce; blocks go in
+// groups of 8 whose partial loads are all issued before the in-order adds.
+template <int D>
+__global__ void __launch_bounds__(64)
+finalize_scan(const float* __restrict__ partials, const __grid_constant__ Sched sc,
+              uint8_t* __restrict__ images) {
+  constexpr int CPR = D / 8, DD = D * D;
+  constexpr int ITEMS = D * CPR + CPR;
+  ptx::grid_dependency_wait();
+  ptx::launch_dependents();
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int heads = sc.nseg / sc.nblk;
+  if (gid >= (long long)heads * ITEMS) return;
+  const int hh = (int)(gid / ITEMS), item = (int)(gid - (long long)hh * ITEMS);
+  const bool zitem = item >= D * CPR;
+  const int n = zitem ? 0 : item % D;
+  const int ac = zitem ? item - D * CPR : item / D;
+  int off[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) off[e] = zitem ? DD + 8 * ac + e : (8 * ac + e) * D + n;
+  float run[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) run[e] = 0.f;
+  for (int b0 = 0; b0 < sc.nblk; b0 += 8) {
+    const int count = min(8, sc.nblk - b0);
+    float blk[8][8];
+    segment_sums8<D>(partials, sc, hh * sc.nblk + b0, count, off, blk);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j < count) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) run[e] = run[e] + blk[j][e];
+        write_image_chunk<D>(images, hh * sc.nblk + b0 + j, zitem, n, ac, run);
+      }
+    }
   }
 }
 
@@ -574,8 +803,7 @@ template <int D, bool ROPE, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
          const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ Rope rope, int L,
-         int nblk, long long U, int stages, const float* __restrict__ apply,
-         const float* __restrict__ partials, const __grid_constant__ Sched ssc, int direct,
+         int nblk, long long U, int stages, int sbuf, const uint8_t* __restrict__ images,
          const float2* __restrict__ gtab, float eps, int* flag) {
   constexpr int TM = kApplyTile;
   constexpr int HALVES = D / 64;
@@ -599,11 +827,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
   const uint32_t base = align_up(raw_addr, 1024);
   uint8_t* sm = smem_raw + (base - raw_addr);
-  const ApplyPlan P = apply_plan(D, ROPE ? rope.entries : 0, GATE ? 1 : 0, stages);
+  const ApplyPlan P = apply_plan(D, ROPE ? rope.entries : 0, GATE ? 1 : 0, stages, sbuf);
   const uint32_t gbase = base + P.off_g;
   const uint32_t Sb = base + P.off_S;
   float* s_den = reinterpret_cast<float*>(sm + P.off_den);   // [stage][chunk][row]
-  float* s_z = reinterpret_cast<float*>(sm + P.off_z);
+  constexpr uint32_t IMG = image_bytes(D);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
   int* s_pos = reinterpret_cast<int*>(sm + P.off_pos);
   const uint32_t bar0 = base + P.off_bar;
@@ -613,7 +841,10 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   auto oready_bar = [&](int s) { return bar0 + 8u * (3 * stages + s); };
   auto accf_bar = [&](int b) { return bar0 + 8u * (4 * stages + b); };
   auto acce_bar = [&](int b) { return bar0 + 8u * (4 * stages + 2 + b); };
-  const uint32_t done_bar = bar0 + 8u * (4 * stages + 4);
+  auto sfull_bar = [&](int k) { return bar0 + 8u * (4 * stages + 4 + k); };
+  auto sempty_bar = [&](int k) { return bar0 + 8u * (4 * stages + 6 + k); };
+  const uint32_t done_bar = bar0 + 8u * (4 * stages + 8);
+  auto s_slot = [&](int k) { return base + P.off_S + (uint32_t)k * image_slot(D); };
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P.off_tmem);
   __shared__ int s_abort;
 
@@ -632,6 +863,8 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(accf_bar(b), 1);
       ptx::mbar_init(acce_bar(b), kMath);
+      ptx::mbar_init(sfull_bar(b), 1);
+      ptx::mbar_init(sempty_bar(b), 1 + kMathWarps);
     }
     ptx::mbar_init(done_bar, 1);
     ptx::fence_mbar_init();
@@ -641,14 +874,33 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     ptx::tmem_relinquish();
   }
   __syncthreads();
+  // launched early (programmatic dependent launch): the images and the RoPE
+  // table are read only after the kernels that write them have completed
+  ptx::grid_dependency_wait();
 
   if (warp == 0) {
-    // ---------------- TMA loads: q (and gate) tiles, RoPE row offsets ----------------
+    // ---------------- TMA loads: S images per segment, q (and gate) tiles ----------------
     TileIter it;
     it.init(u0, tps, stages);
     long long issued = 0;
+    int cur_seg = -1, ss = -1;
     for (long long u = u0; u < u1; ++u, it.next()) {
       int ok = 1;
+      if (it.seg != cur_seg) {
+        // the segment's S image into the next slot, once its last user is done
+        cur_seg = it.seg;
+        ++ss;
+        if (lane == 0) {
+          const int k = ss % sbuf;
+          ok = wait_bounded(sempty_bar(k), (uint32_t)(((ss / sbuf) & 1) ^ 1), flag,
+                            kFlagApplyTimeout, &s_abort);
+          if (ok) {
+            ptx::mbar_expect_tx(sfull_bar(k), IMG);
+            ptx::bulk_load(s_slot(k), images + (long long)it.seg * IMG, IMG, sfull_bar(k));
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      }
       if (lane == 0)
         ok = wait_bounded(empty_bar(it.stage), it.phase ^ 1u, flag, kFlagApplyTimeout, &s_abort);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -670,10 +922,14 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       }
       ++issued;
     }
-    if (lane == 0)
+    if (lane == 0) {
       for (long long i = issued - stages < 0 ? 0 : issued - stages; i < issued; ++i)
         wait_bounded(full_bar((int)(i % stages)), (uint32_t)((i / stages) & 1), flag,
                      kFlagApplyTimeout, &s_abort);
+      for (int i = ss - sbuf + 1 < 0 ? 0 : ss - sbuf + 1; i <= ss; ++i)
+        wait_bounded(sfull_bar(i % sbuf), (uint32_t)((i / sbuf) & 1), flag, kFlagApplyTimeout,
+                     &s_abort);
+    }
   } else if (warp == 1) {
     // ---------------- MMA issuer: acc[b] = RoPE(phi q) [S_hi | S_lo] ----------------
     if (lane == 0) {
@@ -682,7 +938,18 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       it.init(u0, tps, stages);
       int b = 0;
       uint32_t bph = 0;
+      int cur_seg = -1, ss = -1;
+      uint32_t Sb = 0;
       for (long long u = u0; u < u1; ++u, it.next()) {
+        if (it.seg != cur_seg) {
+          cur_seg = it.seg;
+          ++ss;
+          const int k = ss % sbuf;
+          if (!wait_bounded(sfull_bar(k), (uint32_t)((ss / sbuf) & 1), flag, kFlagApplyTimeout,
+                            &s_abort))
+            break;
+          Sb = s_slot(k);
+        }
         if (!wait_bounded(acce_bar(b), bph ^ 1u, flag, kFlagApplyTimeout, &s_abort)) break;
         if (!wait_bounded(qready_bar(it.stage), it.phase, flag, kFlagApplyTimeout, &s_abort))
           break;
@@ -697,6 +964,8 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                         ptx::smem_desc_sw128(Sb + boff, 16, 1024), IDESC, kk == 0 ? 0u : 1u);
         }
         ptx::mma_commit(accf_bar(b));
+        // the slot is free for the next image once this segment's MMAs are done
+        if (it.last_of_segment(u, u1)) ptx::mma_commit(sempty_bar(ss % sbuf));
         if (++b == 2) {
           b = 0;
           bph ^= 1u;
@@ -739,7 +1008,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     uint64_t zc2[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) zc2[e] = ptx::f2(0.f, 0.f);
-    int cur_seg = -1;
+    int cur_seg = -1, ss = -1;
     int pend_stage = -1, pend_b = 0;
     uint32_t pend_bph = 0, pend_ph = 0;
     int b = 0;
@@ -807,51 +1076,23 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     it.init(u0, tps, stages);
     for (long long u = u0; u < u1; ++u, it.next()) {
       if (it.seg != cur_seg) {
-        // every MMA that reads the current S must be done before it is replaced
-        if (pend_stage >= 0) {
-          epilogue(pend_stage, pend_ph, pend_b, pend_bph);
-          pend_stage = -1;
-        }
-        // S and z of the segment: the reduced state, or (bidirectional, no
-        // carried state) the sum of the state kernel's partials in CTA order
-        const float* src = apply + (long long)it.seg * DD1;
-        int nparts = 1;
-        if (direct) {
-          const long long ub = (long long)it.seg * ssc.tps;
-          nparts = cta_of_unit(ssc, ub + ssc.tps - 1) - cta_of_unit(ssc, ub) + 1;
-          src = partials + (long long)it.seg * ssc.maxc * DD1;
-        }
-        for (int item = tt; item < D * CPR; item += kMath) {
-          const int n = item % D, ac = item / D;    // output column n, K chunk ac
-          float x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = src[(8 * ac + e) * D + n];
-          for (int i = 1; i < nparts; ++i) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] += src[(long long)i * DD1 + (8 * ac + e) * D + n];
-          }
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hi[e] = ptx::pack_bf16x2(x[2 * e], x[2 * e + 1]);
-            lo[e] = ptx::pack_bf16x2(x[2 * e] - ptx::bf16_lo(hi[e]),
-                                     x[2 * e + 1] - ptx::bf16_hi(hi[e]));
-          }
-          const uint32_t kof = (ac >> 3) * SHALF, sw = ((ac & 7) ^ (n & 7)) << 4;
-          ptx::st_shared_v4(Sb + kof + n * 128 + sw, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-          ptx::st_shared_v4(Sb + kof + (D + n) * 128 + sw,
-                            make_uint4(lo[0], lo[1], lo[2], lo[3]));
-        }
-        if (tt < D) {
-          float zz = src[D * D + tt];
-          for (int i = 1; i < nparts; ++i) zz += src[(long long)i * DD1 + D * D + tt];
-          s_z[tt] = zz;
-        }
-        ptx::fence_proxy_async();
-        ptx::bar_sync(1, kMath);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) zc2[e] = ptx::f2(s_z[8 * c + 2 * e], s_z[8 * c + 2 * e + 1]);
+        // the segment's image is in slot k: take z of this warp's chunk
         cur_seg = it.seg;
+        ++ss;
+        const int k = ss % sbuf;
+        const bool got = wait_bounded(sfull_bar(k), (uint32_t)((ss / sbuf) & 1), flag,
+                                      kFlagApplyTimeout, &s_abort);
+        if (got) {
+          const float4* zsrc = reinterpret_cast<const float4*>(
+              sm + P.off_S + (uint32_t)k * image_slot(D) + 4u * D * D + 32u * c);
+          const float4 za = zsrc[0], zb = zsrc[1];
+          zc2[0] = ptx::f2(za.x, za.y);
+          zc2[1] = ptx::f2(za.z, za.w);
+          zc2[2] = ptx::f2(zb.x, zb.y);
+          zc2[3] = ptx::f2(zb.z, zb.w);
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(sempty_bar(k));
       }
       const bool ok = wait_bounded(full_bar(it.stage), it.phase, flag, kFlagApplyTimeout,
                                    &s_abort);
@@ -950,6 +1191,29 @@ inline la_status tc_check_launch() {
   return LA_OK;
 }
 
+// Launch with programmatic stream serialisation: the kernel may begin while
+// the previous kernel on the stream is finishing and must call
+// griddepcontrol.wait before it touches that kernel's results.
+template <typename... KArgs, typename... Args>
+inline la_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  return LA_OK;
+}
+
 template <typename K>
 inline la_status tc_smem_attr(K kernel, uint32_t bytes) {
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
@@ -978,14 +1242,20 @@ la_status tc_run_d(const TcArgs& a, int sms) {
                                                     a.flag);
   if ((st = tc_check_launch()) != LA_OK) return st;
   if ((st = tc_mark(a, 1)) != LA_OK) return st;
-  // one segment per head and no carried state: the apply kernel sums the
-  // partials itself (same order as reduce_states) and the reduction is skipped
-  const int direct = (!a.use_state && sc.nblk == 1 && a.do_apply) ? 1 : 0;
-  if (!direct) {
-    dim3 g2((D * (D + 1) + 255) / 256, (unsigned)(a.heads < 65535 ? a.heads : 65535));
-    reduce_states<D><<<g2, 256, 0, a.stream>>>(a.part, sc, a.apply, a.stS, a.stz, a.use_state,
-                                                a.commit);
-    if ((st = tc_check_launch()) != LA_OK) return st;
+  {
+    // the reduction and the apply kernel are launched programmatically
+    // dependent: they start early and wait in griddepcontrol.wait
+    const long long items = a.heads * (long long)(D * (D / 8) + D / 8);
+    uint8_t* images = reinterpret_cast<uint8_t*>(a.apply);
+    if (sc.nblk == 1) {
+      st = launch_pdl(finalize_single<D>, dim3((unsigned)((items + 63) / 64)), dim3(64), 0,
+                      a.stream, (const float*)a.part, sc, images, a.stS, a.stz, a.use_state,
+                      a.commit);
+    } else {
+      st = launch_pdl(finalize_scan<D>, dim3((unsigned)((items + 63) / 64)), dim3(64), 0,
+                      a.stream, (const float*)a.part, sc, images);
+    }
+    if (st != LA_OK) return st;
   }
   if ((st = tc_mark(a, 2)) != LA_OK) return st;
   if (!a.do_apply) return LA_OK;
@@ -995,17 +1265,18 @@ la_status tc_run_d(const TcArgs& a, int sms) {
       !make_map(&mo, a.out, D, sc.L, sc.nseg, kApplyTile) ||
       !make_map(&mg, gate ? a.g : a.q, D, sc.L, sc.nseg, kApplyTile))
     return LA_ERR_CUDA;
-  const int s3 = pick_apply_stages(D, entries, gate ? 1 : 0);
-  const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3);
+  int s3 = 0, sb3 = 1;
+  pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3);
+  const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3, sb3);
   const long long U3 = (long long)sc.nseg * ((sc.L + kApplyTile - 1) / kApplyTile);
   const int G3 = (int)(U3 < sms ? U3 : sms);
   auto k3 = a.rope.on ? (gate ? apply_tc<D, true, true> : apply_tc<D, true, false>)
                       : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
   if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
-  k3<<<G3, kTcThreadsApply, p3.total, a.stream>>>(mq, mg, mo, a.rope, sc.L, sc.nblk, U3, s3,
-                                                  a.apply, a.part, sc, direct, a.gtab, a.eps,
-                                                  a.flag);
-  if ((st = tc_check_launch()) != LA_OK) return st;
+  st = launch_pdl(k3, dim3(G3), dim3(kTcThreadsApply), p3.total, a.stream, mq, mg, mo, a.rope,
+                  sc.L, sc.nblk, U3, s3, sb3, reinterpret_cast<const uint8_t*>(a.apply),
+                  (const float2*)a.gtab, a.eps, a.flag);
+  if (st != LA_OK) return st;
   return tc_mark(a, 3);
 }
 
