@@ -44,7 +44,20 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=MAIN, choices=sorted(workloads.WORKLOADS),
+                    help="workload of the timed line (another one than the default is for "
+                         "profiling runs)")
+    ap.add_argument("--mode", default="bidirectional", choices=["bidirectional", "block_causal"])
+    ap.add_argument("--settle", type=int, default=50,
+                    help="untimed forwards before the timed region (clock settling)")
     return ap.parse_args()
+
+
+def launches_per_forward(w, mode) -> int:
+    """Kernels one forward launches: state build (+ reduction when a head has
+    more than one segment) + apply."""
+    one_segment = mode == "bidirectional" or w.block_tokens in (0, w.N)
+    return 2 if one_segment else 3
 
 
 # ---------------------------------------------------------------- dist ----
@@ -428,7 +441,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, "bidirectional", world),
+        "config": config_of(w, mode, world),
         "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -463,20 +476,22 @@ def main():
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     peak, peak_kind = measured_peaks()
-    w = workloads.WORKLOADS[MAIN]
+    w = workloads.WORKLOADS[args.workload]
+    mode = args.mode
 
     t = device_inputs(w, device, seed=w.seed + rank)
     # settle clocks with untimed work, then sample clocks across the timed region
-    _ = time_forward(w, "bidirectional", t, 50, args.warmup, None, device, record_kernels=False)
+    if args.settle > 0:
+        _ = time_forward(w, mode, t, args.settle, args.warmup, None, device, record_kernels=False)
     sampler = ClockSampler(local)
     sampler.start()
-    # the headline: plain forwards back to back (the three launches overlap
-    # through programmatic dependent launch)
-    ms, _, out = time_forward(w, "bidirectional", t, args.steps, 3, pg, device,
+    # the headline: plain forwards back to back (the launches overlap through
+    # programmatic dependent launch)
+    ms, _, out = time_forward(w, mode, t, args.steps, args.warmup, pg, device,
                               record_kernels=False)
     sampler.stop()
     # per-kernel breakdown: a second timed pass with events between the kernels
-    ms_k, kern, out = time_forward(w, "bidirectional", t, min(args.steps, 200), 3, pg, device,
+    ms_k, kern, out = time_forward(w, mode, t, min(args.steps, 200), 3, pg, device,
                                    record_kernels=True)
     del t, out
     torch.cuda.empty_cache()
@@ -497,7 +512,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded torch CUDA generator, N(0,1) -> bf16)",
-        "config": config_of(w, "bidirectional", world),
+        "config": config_of(w, mode, world),
         "hbm_gbs": round(gbs, 1), "hbm_frac_of_peak": round(gbs / peak, 4),
         "peak_hbm_gbs": peak, "peak_source": peak_kind,
         "roofline": dominant,
@@ -505,12 +520,14 @@ def main():
                     "reduce_us": round(sum(kern[1]) / len(kern[1]) * 1e3, 2),
                     "apply": k_apply},
         "ms_per_step_with_kernel_events": ms_k / min(args.steps, 200),
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": launches_per_forward(w, mode) * args.steps,
         "tensor_core_path": bool(la.uses_tensor_cores(w.B, w.H, w.N, w.D, torch.bfloat16,
                                                       grid=w.grid, rope_split=w.rope_split)),
         "clocks": sampler.summary(),
     }
-    if rank == 0:
+    if args.workload != MAIN or mode != "bidirectional":
+        line["metric"] = "linear-attn fwd tokens/s (profiling run: %s, %s)" % (w.name, mode)
+    if rank == 0 and args.e2e_steps > 0:
         line["e2e"] = measure_e2e(w, args.e2e_steps, device, w.seed)
     if not args.no_extra and rank == 0:
         extra = []

@@ -99,6 +99,11 @@ typedef struct {
   int B, H, D;
 } la_state;
 
+/* Size of the control block at the start of every workspace (included in the
+ * sizes below): a flag word and one arrival counter per segment, zero
+ * between calls. */
+#define LA_WORKSPACE_CONTROL_BYTES 65536u
+
 /* Bytes of workspace lin_attn_forward needs for `p` on the current device
  * (the size depends on the device's SM count). Writes *bytes; no launch. */
 LA_API la_status lin_attn_workspace_size(const la_params* p, size_t* bytes);
@@ -114,7 +119,12 @@ LA_API la_status lin_attn_block_step_workspace_size(const la_params* p, size_t* 
  * q, k, v, out: [B,H,N,D] device pointers in p->dtype. gate: NULL or the same
  * shape and dtype (logits; out is multiplied by their sigmoid).
  * workspace: device memory of at least lin_attn_workspace_size bytes, 256-byte
- * aligned; its contents on entry do not matter and are clobbered.
+ * aligned. Its first LA_WORKSPACE_CONTROL_BYTES bytes are a control block (an
+ * error flag and per-segment arrival counters) that must be zero before the
+ * first call that uses the workspace -- allocate it zeroed; every call leaves
+ * the block zero, and lin_attn_device_status re-zeroes it after a call that
+ * gave up a bounded wait. The rest of the workspace may hold anything on entry
+ * and is clobbered.
  * Returns LA_OK once the work is enqueued on `stream`. */
 LA_API la_status lin_attn_forward(const la_params* p, const void* q, const void* k,
                            const void* v, const void* gate, void* out,
@@ -190,7 +200,7 @@ LA_API la_status lin_attn_state_update(const la_params* p, la_state* st, int t_o
 
 /* Synchronise `stream` and report whether any kernel of the last calls that
  * used `workspace` gave up a bounded wait (LA_ERR_DEVICE_TIMEOUT) -- a safety
- * net that should never fire. Clears the flag. */
+ * net that should never fire. Then re-zeroes the control block. */
 LA_API la_status lin_attn_device_status(void* workspace, void* stream);
 
 /* Static description of a status code. */

@@ -19,6 +19,8 @@ LA_ERR_WORKSPACE = 3
 LA_ERR_CUDA = 4
 LA_ERR_DEVICE_TIMEOUT = 5
 
+LA_WORKSPACE_CONTROL_BYTES = 65536   # control block at the start of a workspace
+
 LA_F32 = 0
 LA_BF16 = 1
 LA_BIDIRECTIONAL = 0

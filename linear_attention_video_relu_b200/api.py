@@ -57,7 +57,9 @@ def _check_io(p: C.la_params, *ts):
 
 
 class Workspace:
-    """A device scratch buffer sized by the library (zeroed once)."""
+    """A device scratch buffer sized by the library, zeroed once: its leading
+    control block must be zero before the first call, and every call leaves it
+    zero."""
 
     def __init__(self, nbytes: int, device):
         self.nbytes = max(int(nbytes), 256)
@@ -66,6 +68,10 @@ class Workspace:
     @property
     def ptr(self):
         return self.buf.data_ptr()
+
+    def control_block_is_zero(self) -> bool:
+        n = min(self.nbytes, C.LA_WORKSPACE_CONTROL_BYTES)
+        return int(torch.count_nonzero(self.buf[:n])) == 0
 
     def status(self, stream=None) -> int:
         """Synchronise and read the bounded-wait flag (see lin_attn_device_status)."""

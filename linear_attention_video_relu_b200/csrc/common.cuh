@@ -79,6 +79,8 @@ struct Sched {
   int nblk;   // segments per head
   int nseg;
   int maxc;
+  int fastU;       // U * G < 2^31: divU divides tile products exactly
+  FastDiv divU;
 };
 
 __host__ __device__ inline long long unit_begin(const Sched& s, long long i) {
@@ -88,6 +90,17 @@ __host__ __device__ inline long long unit_begin(const Sched& s, long long i) {
 // The CTA whose range holds tile u: the largest i with unit_begin(i) <= u.
 __host__ __device__ inline int cta_of_unit(const Sched& s, long long u) {
   return (int)(((u + 1) * (long long)s.G - 1) / s.U);
+}
+
+// cta_of_unit with one multiply-shift when U * G < 2^31.
+__device__ __forceinline__ int cta_of_unit_fast(const Sched& s, long long u) {
+  return s.fastU ? fdiv(s.divU, (int)((u + 1) * s.G - 1)) : cta_of_unit(s, u);
+}
+
+// Number of CTAs (= partial slots) that hold tiles of segment seg.
+__device__ __forceinline__ int parts_of(const Sched& s, int seg) {
+  const long long ub = (long long)seg * s.tps;
+  return cta_of_unit_fast(s, ub + s.tps - 1) - cta_of_unit_fast(s, ub) + 1;
 }
 
 __host__ __device__ inline long long slot_index(const Sched& s, int seg, int cta) {

@@ -25,6 +25,10 @@ using namespace la;
 namespace {
 
 constexpr size_t kAlign = 256;
+// Control block at the start of every workspace: the bounded-wait flag word,
+// then one arrival counter per segment (at most kMaxCounters of them).
+constexpr size_t kCounterOffset = 256;
+constexpr int kMaxCounters = (int)((LA_WORKSPACE_CONTROL_BYTES - kCounterOffset) / sizeof(int));
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -155,6 +159,8 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   if (G > sc.U) G = sc.U;
   if (G < 1) G = 1;
   sc.G = (int)G;
+  sc.fastU = sc.U > 0 && sc.U * sc.G < (1LL << 31);
+  sc.divU = make_fastdiv(sc.fastU ? (int)sc.U : 1);
   sc.maxc = 1;
   if (sc.U > 0) {
     for (int s = 0; s < sc.nseg; ++s) {
@@ -167,8 +173,8 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
 
   const size_t dd1 = (size_t)p->D * (p->D + 1);
   size_t off = 0;
-  pl->off_flag = off;
-  off += kAlign;
+  pl->off_flag = off;                     // control block: flag word, then counters
+  off += LA_WORKSPACE_CONTROL_BYTES;
   pl->off_tab = off;
   off += round_up((size_t)(r.on ? r.entries : 0) * sizeof(float2), kAlign);
   pl->off_part = off;
@@ -283,6 +289,8 @@ la_status run(const Launch& L) {
     a.g = L.g;
     a.out = L.out;
     a.flag = reinterpret_cast<int*>(L.ws + L.pl->off_flag);
+    a.counters = reinterpret_cast<int*>(L.ws + L.pl->off_flag + kCounterOffset);
+    a.fused = L.pl->sc.nblk == 1 && L.pl->sc.nseg <= kMaxCounters;
     a.gtab = reinterpret_cast<float2*>(L.ws + L.pl->off_tab);
     a.part = reinterpret_cast<float*>(L.ws + L.pl->off_part);
     a.apply = reinterpret_cast<float*>(L.ws + L.pl->off_apply);
@@ -436,10 +444,11 @@ la_status lin_attn_forward_noalloc(const la_params* p, const void* q, const void
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != LA_OK) return s;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  // the bounded-wait flag word must start at zero; everything else the
-  // kernels read is written earlier in the same call
-  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + pl.off_flag, 0, sizeof(int), cs) !=
-      cudaSuccess) {
+  // the scratch starts zeroed; a call that gave up a bounded wait may leave
+  // its control block dirty, and this path has no status query, so it is
+  // cleared before every call
+  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + pl.off_flag, 0,
+                      LA_WORKSPACE_CONTROL_BYTES, cs) != cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_CUDA;
   }
@@ -497,7 +506,8 @@ la_status lin_attn_device_status(void* workspace, void* stream) {
     return LA_ERR_CUDA;
   }
   if (flag != 0) {
-    if (cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) {
+    // a kernel that gave up may also have left arrival counters behind
+    if (cudaMemset(workspace, 0, LA_WORKSPACE_CONTROL_BYTES) != cudaSuccess) {
       cudaGetLastError();
       return LA_ERR_CUDA;
     }

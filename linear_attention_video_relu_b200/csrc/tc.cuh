@@ -31,7 +31,9 @@
 
 namespace la {
 
-constexpr int kSmemBudget = 227 * 1024; // dynamic shared memory per CTA on sm_100
+// dynamic shared memory per CTA on sm_100 (227 KB), less 1 KB for the
+// kernels' static shared variables
+constexpr int kSmemBudget = 227 * 1024 - 1024;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 enum : int { kFlagStateTimeout = 1, kFlagApplyTimeout = 2 };
@@ -50,6 +52,8 @@ struct TcArgs {
   float* apply;
   float* stS;
   float* stz;
+  int* counters;   // per-segment arrival counters (zero between calls)
+  int fused;       // one segment per head: the state build writes the images
   int use_state, commit, do_apply;
   float eps;
   cudaStream_t stream;
@@ -89,7 +93,7 @@ __host__ __device__ inline StatePlan state_plan(int D, int entries, int stages) 
   p.off_tab = off;
   off = align_up(off + entries * 8u, 32);
   p.off_pos = off;  // per stage: table row offset of each token row, per axis
-  off += entries ? stages * 3u * tc_state_tile_c(D) * 4 : 0;
+  off = align_up(off + (entries ? stages * 3u * tc_state_tile_c(D) * 2 : 0), 16);
   p.off_z = off;
   off += 2u * 16 * 8 * 4;  // z of each math warp (8 values), per accumulator buffer
   p.off_bar = align_up(off, 8);
@@ -116,7 +120,7 @@ __host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, in
   p.off_tab = align_up(off, 32);
   off = p.off_tab + entries * 8u;
   p.off_pos = align_up(off, 16);
-  off = p.off_pos + (entries ? stages * 3u * kApplyTile * 4 : 0);
+  off = p.off_pos + (entries ? stages * 3u * kApplyTile * 2 : 0);
   p.off_bar = align_up(off, 8);
   off = p.off_bar + (4u * stages + 9u) * 8u;
   p.off_tmem = off;
@@ -281,7 +285,7 @@ __device__ __forceinline__ ChunkCol chunk_col(const Rope& r, int chunk) {
 
 // Table row offsets (per axis) of rows [0, rows) of a tile whose first token
 // is n0, written by the 32 lanes of the TMA warp.
-__device__ __forceinline__ void write_row_offsets(const Rope& r, int* pos, int rows, int n0,
+__device__ __forceinline__ void write_row_offsets(const Rope& r, uint16_t* pos, int rows, int n0,
                                                   int lane) {
   for (int row = lane; row < rows; row += 32) {
     const int n = n0 + row;
@@ -289,9 +293,9 @@ __device__ __forceinline__ void write_row_offsets(const Rope& r, int* pos, int r
     const int rem = n - tl * r.div_hw.d;
     const int h = fdiv(r.div_w, rem);
     const int w = rem - h * r.Wg;
-    pos[row] = r.tab_off[0] + min(tl, r.T - 1) * r.stride[0];
-    pos[rows + row] = r.tab_off[1] + h * r.stride[1];
-    pos[2 * rows + row] = r.tab_off[2] + w * r.stride[2];
+    pos[row] = (uint16_t)(r.tab_off[0] + min(tl, r.T - 1) * r.stride[0]);
+    pos[rows + row] = (uint16_t)(r.tab_off[1] + h * r.stride[1]);
+    pos[2 * rows + row] = (uint16_t)(r.tab_off[2] + w * r.stride[2]);
   }
 }
 
@@ -354,6 +358,96 @@ __device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uint32_t* v) {
       : "memory");
 }
 
+// ---- image of one segment ----------------------------------------------------------
+//
+// Partial slots are [D + 1][D] floats: row n < D is column n of S (S[a][n] at
+// n * D + a), row D is z. An apply image is what the apply kernel copies into
+// shared memory: S as bf16 hi/lo K-major rows (row n holds S[0..D-1][n], 128-byte
+// swizzle, one 64-value half after the other) followed by z as floats. The
+// 4 values a0..a0+3 of row n sit at byte image_offset(n, a0) (hi; lo D * 128
+// bytes further), or at 4 (D * D + a0) for z.
+
+template <int D>
+__device__ __forceinline__ uint32_t image_offset(int n, int a0) {
+  constexpr int SHALF = 2 * D * 128;
+  if (n == D) return 4u * (D * D + a0);
+  const int ac = a0 >> 3;
+  return (ac >> 3) * SHALF + n * 128 + (((ac & 7) ^ (n & 7)) << 4) + ((a0 & 4) << 1);
+}
+
+template <int D>
+__device__ __forceinline__ void store_image4(uint8_t* img, bool zrow, float4 v) {
+  if (zrow) {
+    *reinterpret_cast<float4*>(img) = v;
+  } else {
+    const uint32_t h0 = ptx::pack_bf16x2(v.x, v.y);
+    const uint32_t h1 = ptx::pack_bf16x2(v.z, v.w);
+    const uint32_t l0 = ptx::pack_bf16x2(v.x - ptx::bf16_lo(h0), v.y - ptx::bf16_hi(h0));
+    const uint32_t l1 = ptx::pack_bf16x2(v.z - ptx::bf16_lo(h1), v.w - ptx::bf16_hi(h1));
+    *reinterpret_cast<uint2*>(img) = make_uint2(h0, h1);
+    *reinterpret_cast<uint2*>(img + D * 128) = make_uint2(l0, l1);
+  }
+}
+
+__device__ __forceinline__ float4 add4(float4 x, float4 y) {
+  return make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
+}
+
+__device__ __forceinline__ float4 ldcg4(const float* p) {
+  return __ldcg(reinterpret_cast<const float4*>(p));
+}
+
+// Image (and, when committing, the carried state) of segment seg of a call
+// with one segment per head (seg = head): apply = run + blk with blk the
+// segment's partials summed in CTA order and run the carried state or zero --
+// the fp32 operations of reduce_states. Threads tid, tid + nthr, ... each take
+// 4 values of one partial row; loads bypass L1 (other CTAs wrote them).
+template <int D>
+__device__ void reduce_segment(const float* __restrict__ partials, const Sched& sc, int seg,
+                               uint8_t* __restrict__ images, float* __restrict__ stS,
+                               float* __restrict__ stz, int use_state, int commit, int tid,
+                               int nthr) {
+  constexpr int DD = D * D, DD1 = D * (D + 1), QPR = D / 4, ITEMS = (D + 1) * QPR;
+  constexpr int BATCH = 8;
+  const int np = parts_of(sc, seg);
+  const float* base = partials + (long long)seg * sc.maxc * DD1;
+  uint8_t* img = images + (long long)seg * image_bytes(D);
+  for (int item = tid; item < ITEMS; item += nthr) {
+    const int n = item / QPR;
+    const int a0 = 4 * (item - n * QPR);
+    const bool zrow = n == D;
+    const int off = n * D + a0;
+    float4 acc = ldcg4(base + off);
+    for (int i0 = 1; i0 < np; i0 += BATCH) {
+      float4 b[BATCH];
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k)
+        if (i0 + k < np) b[k] = ldcg4(base + (long long)(i0 + k) * DD1 + off);
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k)
+        if (i0 + k < np) acc = add4(acc, b[k]);
+    }
+    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (use_state) {
+      float r[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        r[e] = zrow ? stz[(long long)seg * D + a0 + e] : stS[(long long)seg * DD + (a0 + e) * D + n];
+      run = make_float4(r[0], r[1], r[2], r[3]);
+    }
+    run = add4(run, acc);
+    store_image4<D>(img + image_offset<D>(n, a0), zrow, run);
+    if (use_state && commit) {
+      const float r[4] = {run.x, run.y, run.z, run.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (zrow) stz[(long long)seg * D + a0 + e] = r[e];
+        else stS[(long long)seg * DD + (a0 + e) * D + n] = r[e];
+      }
+    }
+  }
+}
+
 // ---- state build ------------------------------------------------------------------
 
 // warp 0 TMA, warp 1 MMA, warps 2-17 math, warps 18-21 epilogue (one per TMEM
@@ -364,7 +458,9 @@ template <int D, bool ROPE>
 __global__ void __launch_bounds__(kTcThreadsState, 1)
 state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ Rope rope, const __grid_constant__ Sched sc, int stages,
-               float* __restrict__ partials, float2* __restrict__ gtab, int* flag) {
+               float* __restrict__ partials, float2* __restrict__ gtab, int* flag,
+               int* __restrict__ counters, uint8_t* __restrict__ images, float* stS,
+               float* stz, int use_state, int commit) {
   constexpr int TT = tc_state_tile_c(D);      // tokens per tile
   constexpr int HALVES = D / 64;              // 64-column (128-byte) halves
   constexpr int HALF_BYTES = TT * 128;        // one half of one tensor's tile
@@ -385,7 +481,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   uint8_t* sm = smem_raw + (base - raw_addr);
   const StatePlan P = state_plan(D, ROPE ? rope.entries : 0, stages);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
-  int* s_pos = reinterpret_cast<int*>(sm + P.off_pos);
+  uint16_t* s_pos = reinterpret_cast<uint16_t*>(sm + P.off_pos);
   float* s_z = reinterpret_cast<float*>(sm + P.off_z);
   const uint32_t bar0 = base + P.off_bar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -398,6 +494,8 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   const uint32_t done_bar = bar0 + 8u * (3 * stages + 8);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P.off_tmem);
   __shared__ int s_abort;
+  __shared__ int s_red;    // segment the epilogue warps reduce next, or -1
+  __shared__ int s_tail;   // segment all warps reduce after the tile loop, or -1
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int cta = blockIdx.x;
@@ -405,6 +503,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
   if (threadIdx.x == 0) {
     s_abort = 0;
+    s_tail = -1;
     for (int s = 0; s < stages; ++s) {
       ptx::mbar_init(full_bar(s), 1);
       ptx::mbar_init(kready_bar(s), kMath);
@@ -520,7 +619,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                                    &s_abort);
       if (ok) {
         const uint32_t kt = base + it.stage * STAGE_BYTES + half * HALF_BYTES;
-        const int* rowoff = s_pos + (it.stage * 3 + col.ax) * TT;
+        const uint16_t* rowoff = s_pos + (it.stage * 3 + col.ax) * TT;
 #pragma unroll
         for (int i = 0; i < IPW; ++i) {
           const int r = 32 * (rg0 + WPC * i) + lane;
@@ -563,6 +662,8 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
   } else {
     // ---------------- epilogue warps: accumulator and z -> the CTA's partial slot ------
+    // slot layout: [D + 1][D] floats, row n < D = column n of S (S[a][n] at
+    // n * D + a), row D = z
     const int q = warp & 3;             // TMEM lane quadrant of this warp
     const int te = threadIdx.x - (64 + kMath);
     const uint32_t tmem = *s_tmem;
@@ -587,11 +688,10 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tmem_ld_cols<16>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * D + 16 * cj), v);
         ptx::tmem_wait_ld();
         if (ready && has_row) {
-          float4* dst = reinterpret_cast<float4*>(slot + (size_t)row * D + 16 * cj);
+          // column n of S is row n of the slot: lanes store consecutive a
+          float* dst = slot + (size_t)(16 * cj) * D + row;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+          for (int e = 0; e < 16; ++e) dst[(size_t)e * D] = __uint_as_float(v[e]);
         }
       }
       if (te < D && ready) {
@@ -605,6 +705,34 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       ptx::mbar_arrive(acce_bar(b));
       ptx::mbar_arrive(zfree_bar(b));
       ++sidx;
+      if (counters) {
+        // one segment per head: the CTA that completes a segment last turns
+        // its partials into the image (all epilogue warps' slot writes are
+        // fenced before the arrival is counted)
+        __threadfence();
+        const bool all_ready = ptx::bar_all(2, 128, ready);
+        if (te == 0) {
+          int red = -1;
+          if (all_ready) {
+            const int old = atomicAdd(counters + it.seg, 1);
+            if (old == parts_of(sc, it.seg) - 1) {
+              counters[it.seg] = 0;   // every contributor has arrived
+              red = it.seg;
+            }
+          }
+          if (red >= 0 && u + 1 == u1) {
+            s_tail = red;             // the CTA's last tile: reduce with all warps
+            red = -1;
+          }
+          s_red = red;
+        }
+        ptx::bar_sync(2, 128);
+        const int red = s_red;
+        if (red >= 0) {
+          __threadfence();
+          reduce_segment<D>(partials, sc, red, images, stS, stz, use_state, commit, te, 128);
+        }
+      }
     }
   }
   __syncthreads();
@@ -613,184 +741,122 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     ptx::tc_fence_after();
     ptx::tmem_dealloc(*s_tmem, TMEM_COLS);
   }
+  if (s_tail >= 0 && !s_abort) {
+    __threadfence();
+    reduce_segment<D>(partials, sc, s_tail, images, stS, stz, use_state, commit, threadIdx.x,
+                      kTcThreadsState);
+  }
 }
 
 // ---- reduction into B-operand images -------------------------------------------------
+//
+// finalize_images: for every head and every segment of the head in order,
+// blk = the segment's partials summed in CTA order, apply = run + blk,
+// run = apply, with run starting at zero or at the carried state (written back
+// when committing) -- the fp32 operations of reduce_states. Each apply state is
+// written as the image the apply kernel copies into shared memory: S as bf16
+// hi/lo K-major rows (128-byte swizzle) and z as floats.
+//
+// A thread owns 4 consecutive K-values a0..a0+3 of one row n of the
+// column-major partials (n = D is z) of one head, for all of the head's
+// segments. It walks the (segment, partial) pairs of the head in order in
+// batches of kFinBatch: all loads of a batch are issued before the first add,
+// so every thread keeps kFinBatch 16-byte loads in flight.
 
-// Writes the apply state of segment seg as the image the apply kernel copies
-// into shared memory: S as bf16 hi/lo K-major swizzled rows, z as floats.
+constexpr int kFinThreads = 128;
+constexpr int kFinBatch = 16;
+
+// Position in the ordered list of (segment, partial) pairs of one head.
+struct FinCursor {
+  int j;     // segment within the head
+  int i;     // partial within the segment
+  int np;    // partials of segment j
+  int next;  // first CTA of segment j + 1
+};
+
+__device__ __forceinline__ void fin_start(const Sched& sc, int hh, FinCursor& c) {
+  const long long ub = (long long)hh * sc.nblk * sc.tps;
+  const int first = cta_of_unit_fast(sc, ub);
+  c.j = 0;
+  c.i = 0;
+  c.next = ub + sc.tps < sc.U ? cta_of_unit_fast(sc, ub + sc.tps) : sc.G;
+  c.np = cta_of_unit_fast(sc, ub + sc.tps - 1) - first + 1;
+}
+
+__device__ __forceinline__ void fin_advance(const Sched& sc, int hh, FinCursor& c) {
+  if (++c.i < c.np) return;
+  c.i = 0;
+  if (++c.j >= sc.nblk) return;
+  const long long ub = ((long long)hh * sc.nblk + c.j) * sc.tps;
+  const int first = c.next;
+  c.next = ub + sc.tps < sc.U ? cta_of_unit_fast(sc, ub + sc.tps) : sc.G;
+  c.np = cta_of_unit_fast(sc, ub + sc.tps - 1) - first + 1;
+}
+
 template <int D>
-__device__ __forceinline__ void write_image_chunk(uint8_t* images, int seg, bool zitem, int n,
-                                                  int ac, const float (&v)[8]) {
-  constexpr int SHALF = 2 * D * 128;  // one K-half of the image rows
-  uint8_t* img = images + (long long)seg * image_bytes(D);
-  if (zitem) {
-    float4* zdst = reinterpret_cast<float4*>(img + 4u * D * D + 32u * ac);
-    zdst[0] = make_float4(v[0], v[1], v[2], v[3]);
-    zdst[1] = make_float4(v[4], v[5], v[6], v[7]);
-  } else {
-    uint32_t hi[4], lo[4];
+__host__ __device__ constexpr long long fin_items_per_head() {
+  return (long long)(D + 1) * (D / 4);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFinThreads)
+finalize_images(const float* __restrict__ partials, const __grid_constant__ Sched sc,
+                long long items, uint8_t* __restrict__ images, float* __restrict__ stS,
+                float* __restrict__ stz, int use_state, int commit) {
+  constexpr int DD = D * D, DD1 = D * (D + 1), SHALF = 2 * D * 128, QPR = D / 4;
+  ptx::grid_dependency_wait();
+  ptx::launch_dependents();
+  const long long t = (long long)blockIdx.x * kFinThreads + threadIdx.x;
+  if (t >= items) return;
+  const int hh = (int)(t / fin_items_per_head<D>());
+  const int rem = (int)(t - (long long)hh * fin_items_per_head<D>());
+  const int n = rem / QPR;
+  const int a0 = 4 * (rem - n * QPR);
+  const bool zrow = n == D;
+  const int off = n * D + a0;
+  const uint32_t o = image_offset<D>(n, a0);
+  float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (use_state) {
+    float r[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      r[e] = zrow ? stz[(long long)hh * D + a0 + e] : stS[(long long)hh * DD + (a0 + e) * D + n];
+    run = make_float4(r[0], r[1], r[2], r[3]);
+  }
+  const float* pbase = partials + (long long)hh * sc.nblk * sc.maxc * DD1 + off;
+  uint8_t* ibase = images + (long long)hh * sc.nblk * image_bytes(D) + o;
+  FinCursor c;
+  fin_start(sc, hh, c);
+  float4 acc = run;
+  while (c.j < sc.nblk) {
+    float4 buf[kFinBatch];
+    FinCursor l = c;
+#pragma unroll
+    for (int k = 0; k < kFinBatch; ++k) {
+      if (l.j < sc.nblk) {
+        buf[k] = __ldg(reinterpret_cast<const float4*>(
+            pbase + ((long long)l.j * sc.maxc + l.i) * DD1));
+        fin_advance(sc, hh, l);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kFinBatch; ++k) {
+      if (c.j < sc.nblk) {
+        acc = c.i == 0 ? buf[k] : add4(acc, buf[k]);
+        if (c.i + 1 == c.np) {
+          run = add4(run, acc);
+          store_image4<D>(ibase + (long long)c.j * image_bytes(D), zrow, run);
+        }
+        fin_advance(sc, hh, c);
+      }
+    }
+  }
+  if (use_state && commit) {
+    const float r[4] = {run.x, run.y, run.z, run.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      hi[e] = ptx::pack_bf16x2(v[2 * e], v[2 * e + 1]);
-      lo[e] = ptx::pack_bf16x2(v[2 * e] - ptx::bf16_lo(hi[e]), v[2 * e + 1] - ptx::bf16_hi(hi[e]));
-    }
-    const uint32_t o = (ac >> 3) * SHALF + n * 128 + (((ac & 7) ^ (n & 7)) << 4);
-    *reinterpret_cast<uint4*>(img + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(img + o + D * 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-  }
-}
-
-// Sum of the partials of segment seg at the 8 element offsets off[], in CTA
-// order (the order reduce_states uses).
-template <int D>
-__device__ __forceinline__ void segment_sum(const float* __restrict__ partials, const Sched& sc,
-                                            int seg, const int (&off)[8], float (&blk)[8]) {
-  constexpr int DD1 = D * (D + 1);
-  const long long ub = (long long)seg * sc.tps;
-  const int np = cta_of_unit(sc, ub + sc.tps - 1) - cta_of_unit(sc, ub) + 1;
-  const float* base = partials + (long long)seg * sc.maxc * DD1;
-  // all loads of up to 8 partials are issued before the first add
-  float p[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) p[i][e] = i < np ? base[(long long)i * DD1 + off[e]] : 0.f;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) blk[e] = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (i < np) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) blk[e] += p[i][e];
-    }
-  for (int i = 8; i < np; ++i) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) blk[e] += base[(long long)i * DD1 + off[e]];
-  }
-}
-
-// Sums of up to 8 consecutive segments (first..first+count-1) at the 8 element
-// offsets, with every load issued before any add; blk[j] for segment first+j.
-// Used by the block-causal scan, whose block sums have at most 2 partials in
-// the common case (more fall back to segment_sum).
-template <int D>
-__device__ __forceinline__ void segment_sums8(const float* __restrict__ partials,
-                                              const Sched& sc, int first, int count,
-                                              const int (&off)[8], float (&blk)[8][8]) {
-  constexpr int DD1 = D * (D + 1);
-  int np[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const long long ub = (long long)(first + j) * sc.tps;
-    np[j] = j < count ? cta_of_unit(sc, ub + sc.tps - 1) - cta_of_unit(sc, ub) + 1 : 0;
-  }
-  float p0[8][8], p1[8][8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float* base = partials + (long long)(first + j) * sc.maxc * DD1;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      p0[j][e] = np[j] > 0 ? base[off[e]] : 0.f;
-      p1[j][e] = np[j] > 1 ? base[DD1 + off[e]] : 0.f;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      blk[j][e] = 0.f;
-      if (np[j] > 0) blk[j][e] += p0[j][e];
-      if (np[j] > 1) blk[j][e] += p1[j][e];
-    }
-    if (np[j] > 2) {
-      const float* base = partials + (long long)(first + j) * sc.maxc * DD1;
-      for (int i = 2; i < np[j]; ++i) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) blk[j][e] += base[(long long)i * DD1 + off[e]];
-      }
-    }
-  }
-}
-
-// One segment per head (bidirectional, or one block with a carried state):
-// apply = run + blk with run the carried state (or zero), the fp32 operations
-// of reduce_states; committed back when asked. One thread per (head, chunk of
-// 8 values): chunk (column n, K chunk ac) of S, or K chunk ac of z.
-template <int D>
-__global__ void __launch_bounds__(64)
-finalize_single(const float* __restrict__ partials, const __grid_constant__ Sched sc,
-                uint8_t* __restrict__ images, float* __restrict__ stS, float* __restrict__ stz,
-                int use_state, int commit) {
-  constexpr int CPR = D / 8, DD = D * D;
-  constexpr int ITEMS = D * CPR + CPR;
-  ptx::grid_dependency_wait();
-  ptx::launch_dependents();
-  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gid >= (long long)sc.nseg * ITEMS) return;
-  const int hh = (int)(gid / ITEMS), item = (int)(gid - (long long)hh * ITEMS);
-  const bool zitem = item >= D * CPR;
-  const int n = zitem ? 0 : item % D;
-  const int ac = zitem ? item - D * CPR : item / D;
-  int off[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) off[e] = zitem ? DD + 8 * ac + e : (8 * ac + e) * D + n;
-  float blk[8], run[8];
-  segment_sum<D>(partials, sc, hh, off, blk);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float r0 = !use_state ? 0.f
-                                : (zitem ? stz[(long long)hh * D + 8 * ac + e]
-                                         : stS[(long long)hh * DD + off[e]]);
-    run[e] = r0 + blk[e];
-  }
-  write_image_chunk<D>(images, hh, zitem, n, ac, run);
-  if (use_state && commit) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      if (zitem) stz[(long long)hh * D + 8 * ac + e] = run[e];
-      else stS[(long long)hh * DD + off[e]] = run[e];
-    }
-  }
-}
-
-// Several blocks per head (block-causal): the apply state of block b is
-// run + blk(b) with run the sum over blocks 0..b-1, in block order (the same
-// fp32 operations as reduce_states). One thread per (head, 8-value chunk),
-// consecutive threads on consecutive columns so loads coalesce; blocks go in
-// groups of 8 whose partial loads are all issued before the in-order adds.
-template <int D>
-__global__ void __launch_bounds__(64)
-finalize_scan(const float* __restrict__ partials, const __grid_constant__ Sched sc,
-              uint8_t* __restrict__ images) {
-  constexpr int CPR = D / 8, DD = D * D;
-  constexpr int ITEMS = D * CPR + CPR;
-  ptx::grid_dependency_wait();
-  ptx::launch_dependents();
-  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const int heads = sc.nseg / sc.nblk;
-  if (gid >= (long long)heads * ITEMS) return;
-  const int hh = (int)(gid / ITEMS), item = (int)(gid - (long long)hh * ITEMS);
-  const bool zitem = item >= D * CPR;
-  const int n = zitem ? 0 : item % D;
-  const int ac = zitem ? item - D * CPR : item / D;
-  int off[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) off[e] = zitem ? DD + 8 * ac + e : (8 * ac + e) * D + n;
-  float run[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) run[e] = 0.f;
-  for (int b0 = 0; b0 < sc.nblk; b0 += 8) {
-    const int count = min(8, sc.nblk - b0);
-    float blk[8][8];
-    segment_sums8<D>(partials, sc, hh * sc.nblk + b0, count, off, blk);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < count) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) run[e] = run[e] + blk[j][e];
-        write_image_chunk<D>(images, hh * sc.nblk + b0 + j, zitem, n, ac, run);
-      }
+      if (zrow) stz[(long long)hh * D + a0 + e] = r[e];
+      else stS[(long long)hh * DD + (a0 + e) * D + n] = r[e];
     }
   }
 }
@@ -833,7 +899,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   float* s_den = reinterpret_cast<float*>(sm + P.off_den);   // [stage][chunk][row]
   constexpr uint32_t IMG = image_bytes(D);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
-  int* s_pos = reinterpret_cast<int*>(sm + P.off_pos);
+  uint16_t* s_pos = reinterpret_cast<uint16_t*>(sm + P.off_pos);
   const uint32_t bar0 = base + P.off_bar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto qready_bar = [&](int s) { return bar0 + 8u * (stages + s); };
@@ -1098,7 +1164,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                                    &s_abort);
       if (ok) {
         const uint32_t qt = base + it.stage * TILE_BYTES + half * HALF_BYTES;
-        const int* rowoff = s_pos + (it.stage * 3 + col.ax) * TM;
+        const uint16_t* rowoff = s_pos + (it.stage * 3 + col.ax) * TM;
         float* dst_den = s_den + (it.stage * CPR + c) * TM;
 #pragma unroll
         for (int i = 0; i < IPW; ++i) {
@@ -1238,23 +1304,19 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   auto k1 = a.rope.on ? state_build_tc<D, true> : state_build_tc<D, false>;
   if ((st = tc_smem_attr(k1, p1.total)) != LA_OK) return st;
   if ((st = tc_mark(a, 0)) != LA_OK) return st;
+  uint8_t* images = reinterpret_cast<uint8_t*>(a.apply);
   k1<<<sc.G, kTcThreadsState, p1.total, a.stream>>>(mk, mv, a.rope, sc, s1, a.part, a.gtab,
-                                                    a.flag);
+                                                    a.flag, a.fused ? a.counters : nullptr,
+                                                    images, a.stS, a.stz, a.use_state, a.commit);
   if ((st = tc_check_launch()) != LA_OK) return st;
   if ((st = tc_mark(a, 1)) != LA_OK) return st;
-  {
+  if (!a.fused) {
     // the reduction and the apply kernel are launched programmatically
     // dependent: they start early and wait in griddepcontrol.wait
-    const long long items = a.heads * (long long)(D * (D / 8) + D / 8);
-    uint8_t* images = reinterpret_cast<uint8_t*>(a.apply);
-    if (sc.nblk == 1) {
-      st = launch_pdl(finalize_single<D>, dim3((unsigned)((items + 63) / 64)), dim3(64), 0,
-                      a.stream, (const float*)a.part, sc, images, a.stS, a.stz, a.use_state,
-                      a.commit);
-    } else {
-      st = launch_pdl(finalize_scan<D>, dim3((unsigned)((items + 63) / 64)), dim3(64), 0,
-                      a.stream, (const float*)a.part, sc, images);
-    }
+    const long long items = a.heads * fin_items_per_head<D>();
+    st = launch_pdl(finalize_images<D>, dim3((unsigned)((items + kFinThreads - 1) / kFinThreads)),
+                    dim3(kFinThreads), 0, a.stream, (const float*)a.part, sc, items, images,
+                    a.stS, a.stz, a.use_state, a.commit);
     if (st != LA_OK) return st;
   }
   if ((st = tc_mark(a, 2)) != LA_OK) return st;

@@ -34,7 +34,9 @@ def run_forward(w: workloads.Workload, t: dict, mode: str, **kw) -> torch.Tensor
                      grid=w.grid, rope_split=w.rope_split, theta=w.rope_theta, eps=w.eps,
                      workspace=ws, **kw)
     torch.cuda.synchronize()
-    # no kernel may have given up a bounded wait
+    # the arrival counters and the flag are back at zero, and no kernel gave
+    # up a bounded wait
+    assert ws.control_block_is_zero()
     assert ws.status() == la._native.LA_OK
     return out
 

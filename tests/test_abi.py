@@ -137,3 +137,9 @@ def test_tensor_core_path_selection_is_host_logic():
     assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=20, rope_dh=22, rope_dw=22)) == 0
     assert C.lin_attn_uses_tensor_cores(_params(D=128, rope_dt=32, rope_dh=48, rope_dw=48)) == 1
     assert C.lin_attn_uses_tensor_cores(_params(D=64, rope=0)) == 1
+
+
+def test_control_block_size_matches_the_header():
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+LA_WORKSPACE_CONTROL_BYTES\s+(\d+)u?", text)
+    assert m and int(m.group(1)) == C.LA_WORKSPACE_CONTROL_BYTES

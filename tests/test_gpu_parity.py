@@ -144,6 +144,7 @@ def test_block_steps_match_forward_and_oracle():
         outs.append(o)
     seq = torch.cat(outs, dim=2)
     torch.cuda.synchronize()
+    assert all(ws.control_block_is_zero() for ws in st._ws.values())
     ref = oracle.forward(oracle.params_for(w, "block_causal"), x["q"], x["k"], x["v"])
     assert_parity(to64(seq), ref, w.dtype, "block steps")
     rel, _ = errors(to64(seq), to64(fwd))
