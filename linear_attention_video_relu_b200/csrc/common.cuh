@@ -47,15 +47,13 @@ struct Rope {
   int T, Hg, Wg;
   int t_offset;
   int half[3];       // pairs per axis (d_axis / 2)
-  int stride[3];     // table entries per position (half, padded so that a
-                     // position step is an odd number of 16-byte units)
+  int stride[3];     // table row length per position (rope_stride(half))
   int pair_base[3];  // first pair index of each axis
   int tab_off[3];    // first table entry of each axis
   int entries;       // table size in float2
   double theta;
   FastDiv div_hw;    // by Hg * Wg
   FastDiv div_w;     // by Wg
-  float rcp_stride[3];  // 1 / stride[a] (exact position recovery for entry < 2^20)
   // theta^(-2m/d) / pi of every pair (pair order) as an unevaluated float sum
   // hi + lo, so that position * frequency / pi is formed to ~2^-48 relative
   float inv_pi_hi[64];
@@ -108,57 +106,79 @@ __host__ __device__ inline long long slot_index(const Sched& s, int seg, int cta
 }
 
 // ---- RoPE table ----------------------------------------------------------
+//
+// One row per (axis, position); a row of an axis with `half` rotation pairs
+// holds G = ceil(half / 4) groups of 8 floats -- cos of pairs 4g .. 4g+3, then
+// their sin -- and 4 padding floats, so that a row spans an odd number of
+// 16-byte units (conflict-free 16-byte loads of consecutive positions). Pairs
+// past `half` in the last group read cos 1, sin 0. Sizes and offsets (stride,
+// tab_off, entries) count float2 units of 8 bytes.
 
-// Table stride for an axis with `half` pairs: half rounded up so that one
-// position step spans an odd number of 16-byte units (conflict-free loads of
-// consecutive positions). Zero-width axes keep stride 0.
+// Row length in float2 units for an axis with `half` pairs (0 for none).
 __host__ __device__ inline int rope_stride(int half) {
-  if (half == 0) return 0;
-  int units = (half + 1) / 2;
-  if ((units & 1) == 0) ++units;
-  return 2 * units;
+  return half == 0 ? 0 : 4 * ((half + 3) / 4) + 2;
 }
 
-// (cos, sin) of table entry e: the angle pos * theta^(-2m/d) of its axis
-// position and pair. With x = angle / pi carried as x_hi + x_lo (the product
-// error of x_hi recovered exactly by an FMA), x_hi - 2 rint(x_hi / 2) is exact,
-// so the reduced argument r in [-1, 1] is accurate to a few ulp and
-// sincospif(r) gives cos(angle), sin(angle) to float precision. Padding
-// entries get (1, 0). ih / il are copies of r.inv_pi_hi / r.inv_pi_lo in shared
-// memory (lanes read different pairs; a parameter-space read of a per-lane
+// cos, sin of pair m at position pos on axis a: the angle pos * theta^(-2m/d)
+// with x = angle / pi carried as x_hi + x_lo (the product error of x_hi
+// recovered exactly by an FMA); x_hi - 2 rint(x_hi / 2) is exact, so the
+// reduced argument in [-1, 1] is accurate to a few ulp and sincospif gives
+// cos, sin to float precision. ih / il: theta^(-2m/d) / pi of every pair as a
+// float sum hi + lo, in shared memory (a parameter-space read of a per-lane
 // index would be serialised).
-__device__ inline float2 rope_entry(const Rope& r, const float* ih_tab, const float* il_tab,
-                                    int e) {
-  int base = 0, stride = r.stride[0], half = r.half[0], pb = 0, toff = r.t_offset;
-  float rcp = r.rcp_stride[0];
-  if (e >= r.tab_off[2]) {
-    base = r.tab_off[2]; stride = r.stride[2]; half = r.half[2]; pb = r.pair_base[2];
-    toff = 0; rcp = r.rcp_stride[2];
-  } else if (e >= r.tab_off[1]) {
-    base = r.tab_off[1]; stride = r.stride[1]; half = r.half[1]; pb = r.pair_base[1];
-    toff = 0; rcp = r.rcp_stride[1];
-  }
-  const int local = e - base;
-  const int pos = (int)(((float)local + 0.5f) * rcp);
-  const int m = local - pos * stride;
-  if (m >= half) return make_float2(1.f, 0.f);
-  const float P = (float)(pos + toff);                // exact: positions < 2^24
-  const float ih = ih_tab[pb + m], il = il_tab[pb + m];
-  const float x_hi = P * ih;
-  const float x_lo = fmaf(P, ih, -x_hi) + P * il;
+__device__ inline void rope_angle_cs(int pos, int pair, const float* ih, const float* il,
+                                     float& c, float& s) {
+  const float P = (float)pos;                         // exact: positions < 2^24
+  const float x_hi = P * ih[pair];
+  const float x_lo = fmaf(P, ih[pair], -x_hi) + P * il[pair];
   const float red = (x_hi - 2.f * rintf(0.5f * x_hi)) + x_lo;
-  float s, c;
   sincospif(red, &s, &c);
-  return make_float2(c, s);
 }
 
-// Table entry of pair p (0 .. D/2-1) for a token at local frame tl, row h,
+// Fills the whole table (threads tid, tid + nthr, ...): one work item per
+// (axis, position, group), the item g == G writing the row's padding.
+__device__ inline void rope_fill(const Rope& r, const float* ih, const float* il, float* tab,
+                                 int tid, int nthr) {
+  const int G0 = (r.half[0] + 3) / 4, G1 = (r.half[1] + 3) / 4, G2 = (r.half[2] + 3) / 4;
+  const int n0 = r.half[0] ? r.T * (G0 + 1) : 0;
+  const int n1 = r.half[1] ? r.Hg * (G1 + 1) : 0;
+  const int n2 = r.half[2] ? r.Wg * (G2 + 1) : 0;
+  for (int it = tid; it < n0 + n1 + n2; it += nthr) {
+    const int a = it < n0 ? 0 : (it < n0 + n1 ? 1 : 2);
+    const int local = it - (a == 0 ? 0 : (a == 1 ? n0 : n0 + n1));
+    const int Ga = a == 0 ? G0 : (a == 1 ? G1 : G2);
+    const int half = a == 0 ? r.half[0] : (a == 1 ? r.half[1] : r.half[2]);
+    const int pos = local / (Ga + 1);
+    const int g = local - pos * (Ga + 1);
+    const int toff = a == 0 ? r.tab_off[0] : (a == 1 ? r.tab_off[1] : r.tab_off[2]);
+    const int stride = a == 0 ? r.stride[0] : (a == 1 ? r.stride[1] : r.stride[2]);
+    const int pbase = a == 0 ? r.pair_base[0] : (a == 1 ? r.pair_base[1] : r.pair_base[2]);
+    float* row = tab + 2 * (toff + pos * stride);
+    if (g == Ga) {
+      *reinterpret_cast<float4*>(row + 8 * g) = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    float cv[4], sv[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int m = 4 * g + w;
+      cv[w] = 1.f;
+      sv[w] = 0.f;
+      if (m < half) rope_angle_cs(pos + (a == 0 ? r.t_offset : 0), pbase + m, ih, il, cv[w], sv[w]);
+    }
+    *reinterpret_cast<float4*>(row + 8 * g) = make_float4(cv[0], cv[1], cv[2], cv[3]);
+    *reinterpret_cast<float4*>(row + 8 * g + 4) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+  }
+}
+
+// (cos, sin) of pair p (0 .. D/2-1) for a token at local frame tl, row h,
 // column w.
-__device__ inline int rope_index(const Rope& r, int p, int tl, int h, int w) {
-  int ax = p < r.pair_base[1] ? 0 : (p < r.pair_base[2] ? 1 : 2);
-  int m = p - r.pair_base[ax];
-  int pos = ax == 0 ? tl : (ax == 1 ? h : w);
-  return r.tab_off[ax] + pos * r.stride[ax] + m;
+__device__ inline float2 rope_cs(const Rope& r, const float* tab, int p, int tl, int h, int w) {
+  const int ax = p < r.pair_base[1] ? 0 : (p < r.pair_base[2] ? 1 : 2);
+  const int m = p - r.pair_base[ax];
+  const int pos = ax == 0 ? tl : (ax == 1 ? h : w);
+  const int i = 2 * (r.tab_off[ax] + pos * r.stride[ax]) + 8 * (m >> 2) + (m & 3);
+  return make_float2(tab[i], tab[i + 4]);
 }
 
 // ---- element access --------------------------------------------------------

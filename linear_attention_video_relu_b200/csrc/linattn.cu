@@ -136,7 +136,6 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
     // constants of the rotary parameterisation: theta^(-2m/d) / pi per pair,
     // split into float hi + lo
     for (int a = 0; a < 3; ++a) {
-      r.rcp_stride[a] = r.stride[a] ? 1.f / (float)r.stride[a] : 0.f;
       for (int m = 0; m < r.half[a]; ++m) {
         const double v = pow(r.theta, -(double)m / (double)r.half[a]) / M_PI;
         r.inv_pi_hi[r.pair_base[a] + m] = (float)v;

@@ -52,8 +52,7 @@ state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N
       s_il[tid] = rope.inv_pi_lo[tid];
     }
     __syncthreads();
-    for (int e = tid; e < rope.entries; e += kSimtThreads)
-      s_tab[e] = rope_entry(rope, s_ih, s_il, e);
+    rope_fill(rope, s_ih, s_il, reinterpret_cast<float*>(s_tab), tid, kSimtThreads);
     __syncthreads();
     int e0 = (int)((long long)cta * rope.entries / gridDim.x);
     int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);
@@ -109,7 +108,7 @@ state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N
       if (rope.on && r < rows) {
         int tl, h, w;
         token_pos(rope, nbase + r, tl, h, w);
-        const float2 cs = s_tab[rope_index(rope, pr, tl, h, w)];
+        const float2 cs = rope_cs(rope, reinterpret_cast<const float*>(s_tab), pr, tl, h, w);
         y0 = x0 * cs.x - x1 * cs.y;
         y1 = x0 * cs.y + x1 * cs.x;
       }
@@ -212,7 +211,7 @@ apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out
     if (rope.on && r < rows) {
       int tl, h, w;
       token_pos(rope, nbase + r, tl, h, w);
-      const float2 cs = gtab[rope_index(rope, pr, tl, h, w)];
+      const float2 cs = rope_cs(rope, reinterpret_cast<const float*>(gtab), pr, tl, h, w);
       y0 = x0 * cs.x - x1 * cs.y;
       y1 = x0 * cs.y + x1 * cs.x;
     }

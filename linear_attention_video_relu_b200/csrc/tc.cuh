@@ -299,11 +299,12 @@ __device__ __forceinline__ void write_row_offsets(const Rope& r, uint16_t* pos, 
   }
 }
 
-// phi = ReLU on 8 bf16 values (packed max with 0, exact in bf16), then, with
-// ROPE, the rotation of the 4 pairs by the (cos, sin) at cs. The un-rotated
-// phi values come back as 4 packed fp32 pairs.
+// phi = ReLU of one 16-byte chunk of bf16 values (4 rotation pairs (x_j, y_j)),
+// rotated by the pairs' cos, sin: cs[0] holds the cos of the 4 pairs, cs[1]
+// their sin; x' = x cos - y sin, y' = x sin + y cos in fp32, rounded once to
+// bf16. xy returns phi as packed float pairs {(x0,x1), (x2,x3), (y0,y1), (y2,y3)}.
 template <bool ROPE>
-__device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, uint64_t (&f)[4]) {
+__device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, uint64_t (&xy)[4]) {
   const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
   uint32_t m[4];
   float x[4], y[4];
@@ -312,17 +313,22 @@ __device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, uint64_t 
     asm("max.bf16x2 %0, %1, %2;" : "=r"(m[j]) : "r"(w4[j]), "r"(0u));
     x[j] = ptx::bf16_lo(m[j]);
     y[j] = ptx::bf16_hi(m[j]);
-    f[j] = ptx::f2(x[j], y[j]);
   }
+  xy[0] = ptx::f2(x[0], x[1]);
+  xy[1] = ptx::f2(x[2], x[3]);
+  xy[2] = ptx::f2(y[0], y[1]);
+  xy[3] = ptx::f2(y[2], y[3]);
   if (!ROPE) return make_uint4(m[0], m[1], m[2], m[3]);
-  const float4 c01 = cs[0], c23 = cs[1];
-  const float cv[4] = {c01.x, c01.z, c23.x, c23.z};
-  const float sv[4] = {c01.y, c01.w, c23.y, c23.w};
-  uint32_t o[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    o[j] = ptx::pack_bf16x2(fmaf(x[j], cv[j], -y[j] * sv[j]), fmaf(x[j], sv[j], y[j] * cv[j]));
-  return make_uint4(o[0], o[1], o[2], o[3]);
+  const float4 C = cs[0], S = cs[1];
+  const uint64_t c01 = ptx::f2(C.x, C.y), c23 = ptx::f2(C.z, C.w);
+  const uint64_t s01 = ptx::f2(S.x, S.y), s23 = ptx::f2(S.z, S.w);
+  float ox[4], oy[4];
+  ptx::f2_split(ptx::sub2(ptx::mul2(xy[0], c01), ptx::mul2(xy[2], s01)), ox[0], ox[1]);
+  ptx::f2_split(ptx::sub2(ptx::mul2(xy[1], c23), ptx::mul2(xy[3], s23)), ox[2], ox[3]);
+  ptx::f2_split(ptx::fma2(xy[0], s01, ptx::mul2(xy[2], c01)), oy[0], oy[1]);
+  ptx::f2_split(ptx::fma2(xy[1], s23, ptx::mul2(xy[3], c23)), oy[2], oy[3]);
+  return make_uint4(ptx::pack_bf16x2(ox[0], oy[0]), ptx::pack_bf16x2(ox[1], oy[1]),
+                    ptx::pack_bf16x2(ox[2], oy[2]), ptx::pack_bf16x2(ox[3], oy[3]));
 }
 
 // Builds the CTA's cos/sin table in shared memory (all math threads), then
@@ -334,7 +340,7 @@ __device__ __forceinline__ void build_rope_table(const Rope& r, float2* tab, int
     s_il[tt] = r.inv_pi_lo[tt];
   }
   ptx::bar_sync(1, kMath);
-  for (int e = tt; e < r.entries; e += kMath) tab[e] = rope_entry(r, s_ih, s_il, e);
+  rope_fill(r, s_ih, s_il, reinterpret_cast<float*>(tab), tt, kMath);
   ptx::bar_sync(1, kMath);
 }
 
@@ -642,12 +648,14 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int b = sidx & 1;
         wait_bounded(zfree_bar(b), (uint32_t)(((sidx >> 1) & 1) ^ 1), flag, kFlagStateTimeout,
                      &s_abort);
+        // z2 = {(d0,d2), (d4,d6), (d1,d3), (d5,d7)} of the chunk's 8 dims
         float zz[8];
+        ptx::f2_split(z2[0], zz[0], zz[2]);
+        ptx::f2_split(z2[1], zz[4], zz[6]);
+        ptx::f2_split(z2[2], zz[1], zz[3]);
+        ptx::f2_split(z2[3], zz[5], zz[7]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          ptx::f2_split(z2[e], zz[2 * e], zz[2 * e + 1]);
-          z2[e] = ptx::f2(0.f, 0.f);
-        }
+        for (int e = 0; e < 4; ++e) z2[e] = ptx::f2(0.f, 0.f);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float t = zz[e];
@@ -753,105 +761,86 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 // finalize_images: for every head and every segment of the head in order,
 // blk = the segment's partials summed in CTA order, apply = run + blk,
 // run = apply, with run starting at zero or at the carried state (written back
-// when committing) -- the fp32 operations of reduce_states. Each apply state is
-// written as the image the apply kernel copies into shared memory: S as bf16
-// hi/lo K-major rows (128-byte swizzle) and z as floats.
+// when committing) -- the fp32 operations of reduce_states -- and apply
+// written as the segment's image.
 //
-// A thread owns 4 consecutive K-values a0..a0+3 of one row n of the
-// column-major partials (n = D is z) of one head, for all of the head's
-// segments. It walks the (segment, partial) pairs of the head in order in
-// batches of kFinBatch: all loads of a batch are issued before the first add,
-// so every thread keeps kFinBatch 16-byte loads in flight.
+// Grid (heads, row groups): a thread owns 4 consecutive K-values a0..a0+3 of
+// one row n of the column-major partials (n = D is z) of one head, for all of
+// the head's segments. The CTA first tabulates the partial count of up to
+// kFinSegs segments in shared memory; threads then take the segments in
+// batches of kFinBatch, issuing the loads of the first two partials of every
+// segment of a batch before the first add (more than two is rare and loops).
 
 constexpr int kFinThreads = 128;
 constexpr int kFinBatch = 16;
-
-// Position in the ordered list of (segment, partial) pairs of one head.
-struct FinCursor {
-  int j;     // segment within the head
-  int i;     // partial within the segment
-  int np;    // partials of segment j
-  int next;  // first CTA of segment j + 1
-};
-
-__device__ __forceinline__ void fin_start(const Sched& sc, int hh, FinCursor& c) {
-  const long long ub = (long long)hh * sc.nblk * sc.tps;
-  const int first = cta_of_unit_fast(sc, ub);
-  c.j = 0;
-  c.i = 0;
-  c.next = ub + sc.tps < sc.U ? cta_of_unit_fast(sc, ub + sc.tps) : sc.G;
-  c.np = cta_of_unit_fast(sc, ub + sc.tps - 1) - first + 1;
-}
-
-__device__ __forceinline__ void fin_advance(const Sched& sc, int hh, FinCursor& c) {
-  if (++c.i < c.np) return;
-  c.i = 0;
-  if (++c.j >= sc.nblk) return;
-  const long long ub = ((long long)hh * sc.nblk + c.j) * sc.tps;
-  const int first = c.next;
-  c.next = ub + sc.tps < sc.U ? cta_of_unit_fast(sc, ub + sc.tps) : sc.G;
-  c.np = cta_of_unit_fast(sc, ub + sc.tps - 1) - first + 1;
-}
+constexpr int kFinSegs = 1024;
 
 template <int D>
-__host__ __device__ constexpr long long fin_items_per_head() {
-  return (long long)(D + 1) * (D / 4);
+__host__ __device__ constexpr int fin_items_per_head() {
+  return (D + 1) * (D / 4);
 }
 
 template <int D>
 __global__ void __launch_bounds__(kFinThreads)
 finalize_images(const float* __restrict__ partials, const __grid_constant__ Sched sc,
-                long long items, uint8_t* __restrict__ images, float* __restrict__ stS,
+                uint8_t* __restrict__ images, float* __restrict__ stS,
                 float* __restrict__ stz, int use_state, int commit) {
-  constexpr int DD = D * D, DD1 = D * (D + 1), SHALF = 2 * D * 128, QPR = D / 4;
+  constexpr int DD = D * D, DD1 = D * (D + 1), QPR = D / 4;
+  __shared__ int s_np[kFinSegs];
   ptx::grid_dependency_wait();
   ptx::launch_dependents();
-  const long long t = (long long)blockIdx.x * kFinThreads + threadIdx.x;
-  if (t >= items) return;
-  const int hh = (int)(t / fin_items_per_head<D>());
-  const int rem = (int)(t - (long long)hh * fin_items_per_head<D>());
-  const int n = rem / QPR;
-  const int a0 = 4 * (rem - n * QPR);
+  const int hh = blockIdx.x;
+  const int item = blockIdx.y * kFinThreads + threadIdx.x;
+  const bool valid = item < fin_items_per_head<D>();
+  const int n = item / QPR;
+  const int a0 = 4 * (item - n * QPR);
   const bool zrow = n == D;
   const int off = n * D + a0;
-  const uint32_t o = image_offset<D>(n, a0);
   float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (use_state) {
+  if (use_state && valid) {
     float r[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e)
       r[e] = zrow ? stz[(long long)hh * D + a0 + e] : stS[(long long)hh * DD + (a0 + e) * D + n];
     run = make_float4(r[0], r[1], r[2], r[3]);
   }
-  const float* pbase = partials + (long long)hh * sc.nblk * sc.maxc * DD1 + off;
-  uint8_t* ibase = images + (long long)hh * sc.nblk * image_bytes(D) + o;
-  FinCursor c;
-  fin_start(sc, hh, c);
-  float4 acc = run;
-  while (c.j < sc.nblk) {
-    float4 buf[kFinBatch];
-    FinCursor l = c;
+  const long long seg0 = (long long)hh * sc.nblk;
+  const float* pbase = partials + seg0 * sc.maxc * DD1 + off;
+  uint8_t* ibase = images + seg0 * image_bytes(D) + (valid ? image_offset<D>(n, a0) : 0);
+  const long long pstride = (long long)sc.maxc * DD1;
+  for (int j0 = 0; j0 < sc.nblk; j0 += kFinSegs) {
+    const int cnt = min(kFinSegs, sc.nblk - j0);
+    for (int jj = threadIdx.x; jj < cnt; jj += kFinThreads)
+      s_np[jj] = parts_of(sc, (int)(seg0 + j0 + jj));
+    __syncthreads();
+    if (valid) {
+      for (int jb = 0; jb < cnt; jb += kFinBatch) {
+        float4 b0[kFinBatch], b1[kFinBatch];
+        int np[kFinBatch];
 #pragma unroll
-    for (int k = 0; k < kFinBatch; ++k) {
-      if (l.j < sc.nblk) {
-        buf[k] = __ldg(reinterpret_cast<const float4*>(
-            pbase + ((long long)l.j * sc.maxc + l.i) * DD1));
-        fin_advance(sc, hh, l);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kFinBatch; ++k) {
-      if (c.j < sc.nblk) {
-        acc = c.i == 0 ? buf[k] : add4(acc, buf[k]);
-        if (c.i + 1 == c.np) {
-          run = add4(run, acc);
-          store_image4<D>(ibase + (long long)c.j * image_bytes(D), zrow, run);
+        for (int k = 0; k < kFinBatch; ++k) {
+          np[k] = jb + k < cnt ? s_np[jb + k] : 0;
+          const float* p = pbase + (j0 + jb + k) * pstride;
+          if (np[k] > 0) b0[k] = __ldg(reinterpret_cast<const float4*>(p));
+          if (np[k] > 1) b1[k] = __ldg(reinterpret_cast<const float4*>(p + DD1));
         }
-        fin_advance(sc, hh, c);
+#pragma unroll
+        for (int k = 0; k < kFinBatch; ++k) {
+          if (np[k] > 0) {
+            float4 blk = b0[k];
+            if (np[k] > 1) blk = add4(blk, b1[k]);
+            const float* p = pbase + (j0 + jb + k) * pstride;
+            for (int i = 2; i < np[k]; ++i)
+              blk = add4(blk, __ldg(reinterpret_cast<const float4*>(p + (long long)i * DD1)));
+            run = add4(run, blk);
+            store_image4<D>(ibase + (long long)(j0 + jb + k) * image_bytes(D), zrow, run);
+          }
+        }
       }
     }
+    __syncthreads();
   }
-  if (use_state && commit) {
+  if (use_state && commit && valid) {
     const float r[4] = {run.x, run.y, run.z, run.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -875,15 +864,13 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   constexpr int HALVES = D / 64;
   constexpr int HALF_BYTES = TM * 128;
   constexpr int TILE_BYTES = HALVES * HALF_BYTES;
-  constexpr int NB = 2 * D;                  // B operand rows: S_hi^T then S_lo^T
-  constexpr int SHALF = NB * 128;            // one K-half of the B operand
+  constexpr int SHALF = 2 * D * 128;         // one K-half of an image: S_hi^T, S_lo^T rows
   constexpr int CPR = D / 8;
   constexpr int WPC = kMathWarps / CPR;      // warps per chunk column
   constexpr int IPW = TM / 32 / WPC;         // 32-row groups per warp and tile
   constexpr int KSTEPS = D / 16;
-  constexpr int DD1 = D * (D + 1);
-  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, NB, 0, 0);
-  constexpr uint32_t TMEM_COLS = 2 * NB;
+  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, D, 0, 0);
+  constexpr uint32_t TMEM_COLS = 2 * D;      // two accumulators of D columns
   constexpr uint32_t TX = (GATE ? 2 : 1) * TILE_BYTES;
   constexpr int EC = D / 4;                  // epilogue columns per thread
   static_assert(WPC >= 1 && IPW * WPC * 32 == TM, "tile must split over the math warps");
@@ -895,7 +882,6 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   uint8_t* sm = smem_raw + (base - raw_addr);
   const ApplyPlan P = apply_plan(D, ROPE ? rope.entries : 0, GATE ? 1 : 0, stages, sbuf);
   const uint32_t gbase = base + P.off_g;
-  const uint32_t Sb = base + P.off_S;
   float* s_den = reinterpret_cast<float*>(sm + P.off_den);   // [stage][chunk][row]
   constexpr uint32_t IMG = image_bytes(D);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
@@ -997,7 +983,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                      &s_abort);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer: acc[b] = RoPE(phi q) [S_hi | S_lo] ----------------
+    // ---------------- MMA issuer: acc[b] = RoPE(phi q) S_hi + RoPE(phi q) S_lo ----------
     if (lane == 0) {
       const uint32_t tmem = *s_tmem;
       TileIter it;
@@ -1021,13 +1007,17 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           break;
         ptx::tc_fence_after();
         const uint32_t qt = base + it.stage * TILE_BYTES;
-        const uint32_t acc = tmem + (uint32_t)(b * NB);
+        const uint32_t acc = tmem + (uint32_t)(b * D);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
+          // the hi and lo halves of S accumulate into the same columns
           const uint32_t aoff = (kk / 4) * HALF_BYTES + (kk % 4) * 32;
           const uint32_t boff = (kk / 4) * SHALF + (kk % 4) * 32;
-          ptx::mma_bf16(acc, ptx::smem_desc_sw128(qt + aoff, 16, 1024),
-                        ptx::smem_desc_sw128(Sb + boff, 16, 1024), IDESC, kk == 0 ? 0u : 1u);
+          const uint64_t adesc = ptx::smem_desc_sw128(qt + aoff, 16, 1024);
+          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(Sb + boff, 16, 1024), IDESC,
+                        kk == 0 ? 0u : 1u);
+          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(Sb + boff + D * 128, 16, 1024), IDESC,
+                        1u);
         }
         ptx::mma_commit(accf_bar(b));
         // the slot is free for the next image once this segment's MMAs are done
@@ -1080,7 +1070,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     int b = 0;
     uint32_t bph = 0;
 
-    // out = (acc_hi + acc_lo) / den (* sigmoid(g)) as bf16, over the q tile
+    // out = acc / den (* sigmoid(g)) as bf16, over the q tile
     auto epilogue = [&](int s, uint32_t sph, int eb, uint32_t ebph) {
       // all den partials of the tile are in shared memory once every math
       // thread has arrived on the tile's qready barrier
@@ -1096,11 +1086,10 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       const uint64_t inv2 = ptx::f2(inv, inv);
       const uint32_t qt = base + s * TILE_BYTES;
       const uint32_t gt = gbase + s * TILE_BYTES;
-      const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(eb * NB);
+      const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(eb * D);
       const int col0 = quarter * EC;
-      uint32_t vh[EC], vl[EC];
+      uint32_t vh[EC];
       tmem_ld_cols<EC>(lane_base + col0, vh);
-      tmem_ld_cols<EC>(lane_base + D + col0, vl);
       ptx::tmem_wait_ld();
       if (ready) {
         const int h = col0 / 64;
@@ -1113,9 +1102,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           for (int e = 0; e < 4; ++e) {
             const uint64_t hv = ptx::f2(__uint_as_float(vh[8 * k4 + 2 * e]),
                                         __uint_as_float(vh[8 * k4 + 2 * e + 1]));
-            const uint64_t lv = ptx::f2(__uint_as_float(vl[8 * k4 + 2 * e]),
-                                        __uint_as_float(vl[8 * k4 + 2 * e + 1]));
-            ptx::f2_split(ptx::mul2(ptx::add2(hv, lv), inv2), o[2 * e], o[2 * e + 1]);
+            ptx::f2_split(ptx::mul2(hv, inv2), o[2 * e], o[2 * e + 1]);
           }
           if (GATE) {
             const uint4 gr = ptx::ld_shared_v4(gt + off);
@@ -1152,10 +1139,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           const float4* zsrc = reinterpret_cast<const float4*>(
               sm + P.off_S + (uint32_t)k * image_slot(D) + 4u * D * D + 32u * c);
           const float4 za = zsrc[0], zb = zsrc[1];
-          zc2[0] = ptx::f2(za.x, za.y);
-          zc2[1] = ptx::f2(za.z, za.w);
-          zc2[2] = ptx::f2(zb.x, zb.y);
-          zc2[3] = ptx::f2(zb.z, zb.w);
+          // in the packing of phi_rope's xy: (d0,d2), (d4,d6), (d1,d3), (d5,d7)
+          zc2[0] = ptx::f2(za.x, za.z);
+          zc2[1] = ptx::f2(zb.x, zb.z);
+          zc2[2] = ptx::f2(za.y, za.w);
+          zc2[3] = ptx::f2(zb.y, zb.w);
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(sempty_bar(k));
@@ -1313,10 +1301,9 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   if (!a.fused) {
     // the reduction and the apply kernel are launched programmatically
     // dependent: they start early and wait in griddepcontrol.wait
-    const long long items = a.heads * fin_items_per_head<D>();
-    st = launch_pdl(finalize_images<D>, dim3((unsigned)((items + kFinThreads - 1) / kFinThreads)),
-                    dim3(kFinThreads), 0, a.stream, (const float*)a.part, sc, items, images,
-                    a.stS, a.stz, a.use_state, a.commit);
+    const dim3 grid((unsigned)a.heads, (fin_items_per_head<D>() + kFinThreads - 1) / kFinThreads);
+    st = launch_pdl(finalize_images<D>, grid, dim3(kFinThreads), 0, a.stream,
+                    (const float*)a.part, sc, images, a.stS, a.stz, a.use_state, a.commit);
     if (st != LA_OK) return st;
   }
   if ((st = tc_mark(a, 2)) != LA_OK) return st;
