@@ -178,8 +178,9 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   off += round_up((size_t)(r.on ? r.entries : 0) * sizeof(float2), kAlign);
   pl->off_part = off;
   off += round_up((size_t)sc.nseg * sc.maxc * dd1 * sizeof(float), kAlign);
-  pl->off_apply = off;
-  off += round_up((size_t)sc.nseg * dd1 * sizeof(float), kAlign);
+  pl->off_apply = off;   // fp32 apply states (SIMT) or B-operand images (tensor cores)
+  const size_t per_seg = pl->tc ? (size_t)image_bytes(p->D) : dd1 * sizeof(float);
+  off += round_up((size_t)sc.nseg * per_seg, kAlign);
   pl->total = off;
   return LA_OK;
 }

@@ -74,13 +74,16 @@ struct StatePlan {
 
 struct ApplyPlan {
   int stages, sbuf;
-  uint32_t off_g, off_S, off_den, off_tab, off_pos, off_bar, off_tmem, total;
+  uint32_t off_g, off_S, off_tab, off_pos, off_bar, off_tmem, total;
 };
 
-// Bytes of one segment's B-operand image: S as bf16 hi and lo rows (K-major,
-// 128-byte swizzle, 2D rows of D values) followed by z as D floats. This is
-// exactly the size of a D x (D + 1) fp32 state.
-__host__ __device__ constexpr uint32_t image_bytes(int D) { return 4u * D * (D + 1); }
+// Bytes of one segment's B-operand image (K-major, 128-byte swizzle): per
+// 64-value K half, D rows of S_hi^T then D rows of S_lo^T (bf16); then per K
+// half a 16-row block whose row 0 is z_hi, row 1 z_lo and rows 2-15 zero.
+__host__ __device__ constexpr uint32_t image_zoff(int D) { return 4u * D * D; }
+__host__ __device__ constexpr uint32_t image_bytes(int D) {
+  return image_zoff(D) + (uint32_t)(D / 64) * 2048u;
+}
 __host__ __device__ constexpr uint32_t image_slot(int D) { return (image_bytes(D) + 1023u) / 1024u * 1024u; }
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -115,8 +118,6 @@ __host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, in
   off += gate ? stages * tile : 0;
   p.off_S = align_up(off, 1024);
   off = p.off_S + sbuf * image_slot(D);  // B-operand images, one per S slot
-  p.off_den = off;
-  off += stages * (D / 8) * kApplyTile * 4u;
   p.off_tab = align_up(off, 32);
   off = p.off_tab + entries * 8u;
   p.off_pos = align_up(off, 16);
@@ -173,12 +174,15 @@ inline bool tc_supported(bool bf16, int D, int rope, int dt, int dh, int dw, int
 
 // Bounded mbarrier wait: false after kWaitLimitNs (then the flag records it
 // and *abort tells the other roles to stop), or as soon as *abort is set.
+// Longest sleep of one try_wait; the thread wakes when the phase completes.
+constexpr uint32_t kWaitSleepNs = 1000000;
+
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, int* flag, int code,
                                              volatile int* abort_flag) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+  if (ptx::mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
   const uint64_t t0 = ptx::globaltimer();
   for (uint32_t n = 1;; ++n) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if ((n & 15u) == 0) {
       if (*abort_flag) return false;
       if (ptx::globaltimer() - t0 > kWaitLimitNs) {
@@ -302,11 +306,12 @@ __device__ __forceinline__ void write_row_offsets(const Rope& r, uint16_t* pos, 
 // phi = ReLU of one 16-byte chunk of bf16 values (4 rotation pairs (x_j, y_j)),
 // rotated by the pairs' cos, sin: cs[0] holds the cos of the 4 pairs, cs[1]
 // their sin; x' = x cos - y sin, y' = x sin + y cos in fp32, rounded once to
-// bf16. xy returns phi as packed float pairs {(x0,x1), (x2,x3), (y0,y1), (y2,y3)}.
+// bf16. xy returns phi as packed float pairs {(x0,x1), (x2,x3), (y0,y1), (y2,y3)},
+// m as the 4 bf16x2 words.
 template <bool ROPE>
-__device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, uint64_t (&xy)[4]) {
+__device__ __forceinline__ uint4 phi_rope(uint4 raw, const float4* cs, uint64_t (&xy)[4],
+                                          uint32_t (&m)[4]) {
   const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-  uint32_t m[4];
   float x[4], y[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -367,32 +372,39 @@ __device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uint32_t* v) {
 // ---- image of one segment ----------------------------------------------------------
 //
 // Partial slots are [D + 1][D] floats: row n < D is column n of S (S[a][n] at
-// n * D + a), row D is z. An apply image is what the apply kernel copies into
-// shared memory: S as bf16 hi/lo K-major rows (row n holds S[0..D-1][n], 128-byte
-// swizzle, one 64-value half after the other) followed by z as floats. The
-// 4 values a0..a0+3 of row n sit at byte image_offset(n, a0) (hi; lo D * 128
-// bytes further), or at 4 (D * D + a0) for z.
+// n * D + a), row D is z. An apply image (layout at image_bytes) is what the
+// apply kernel copies into shared memory as its B operands. The 4 values
+// a0..a0+3 of row n (< D) go to byte image_offset(n, a0) as hi, D * 128 bytes
+// further as lo; those of z to rows 0 (hi) and 1 (lo) of the z block.
 
 template <int D>
 __device__ __forceinline__ uint32_t image_offset(int n, int a0) {
   constexpr int SHALF = 2 * D * 128;
-  if (n == D) return 4u * (D * D + a0);
   const int ac = a0 >> 3;
+  if (n == D) return image_zoff(D) + (ac >> 3) * 2048u + (((ac & 7)) << 4) + ((a0 & 4) << 1);
   return (ac >> 3) * SHALF + n * 128 + (((ac & 7) ^ (n & 7)) << 4) + ((a0 & 4) << 1);
 }
 
 template <int D>
-__device__ __forceinline__ void store_image4(uint8_t* img, bool zrow, float4 v) {
-  if (zrow) {
-    *reinterpret_cast<float4*>(img) = v;
-  } else {
-    const uint32_t h0 = ptx::pack_bf16x2(v.x, v.y);
-    const uint32_t h1 = ptx::pack_bf16x2(v.z, v.w);
-    const uint32_t l0 = ptx::pack_bf16x2(v.x - ptx::bf16_lo(h0), v.y - ptx::bf16_hi(h0));
-    const uint32_t l1 = ptx::pack_bf16x2(v.z - ptx::bf16_lo(h1), v.w - ptx::bf16_hi(h1));
-    *reinterpret_cast<uint2*>(img) = make_uint2(h0, h1);
+__device__ __forceinline__ void store_image4(uint8_t* img, bool zrow, int a0, float4 v) {
+  const uint32_t h0 = ptx::pack_bf16x2(v.x, v.y);
+  const uint32_t h1 = ptx::pack_bf16x2(v.z, v.w);
+  const uint32_t l0 = ptx::pack_bf16x2(v.x - ptx::bf16_lo(h0), v.y - ptx::bf16_hi(h0));
+  const uint32_t l1 = ptx::pack_bf16x2(v.z - ptx::bf16_lo(h1), v.w - ptx::bf16_hi(h1));
+  *reinterpret_cast<uint2*>(img) = make_uint2(h0, h1);
+  if (!zrow) {
     *reinterpret_cast<uint2*>(img + D * 128) = make_uint2(l0, l1);
+    return;
   }
+  // z block: img is row 0 of chunk ac (unswizzled there); row r holds that
+  // chunk at 16-byte position (ac ^ r) & 7 within its 128 bytes
+  const int ac = (a0 >> 3) & 7;
+  uint8_t* blk = img - ((ac << 4) + ((a0 & 4) << 1));
+  const int sub = (a0 & 4) << 1;
+  *reinterpret_cast<uint2*>(blk + 128 + (((ac ^ 1) & 7) << 4) + sub) = make_uint2(l0, l1);
+#pragma unroll
+  for (int r = 2; r < 16; ++r)
+    *reinterpret_cast<uint2*>(blk + r * 128 + (((ac ^ r) & 7) << 4) + sub) = make_uint2(0u, 0u);
 }
 
 __device__ __forceinline__ float4 add4(float4 x, float4 y) {
@@ -442,7 +454,7 @@ __device__ void reduce_segment(const float* __restrict__ partials, const Sched& 
       run = make_float4(r[0], r[1], r[2], r[3]);
     }
     run = add4(run, acc);
-    store_image4<D>(img + image_offset<D>(n, a0), zrow, run);
+    store_image4<D>(img + image_offset<D>(n, a0), zrow, a0, run);
     if (use_state && commit) {
       const float r[4] = {run.x, run.y, run.z, run.w};
 #pragma unroll
@@ -632,9 +644,10 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           const uint32_t addr = kt + r * 128 + ((cc ^ (r & 7)) << 4);
           const uint4 raw = ptx::ld_shared_v4(addr);
           uint64_t f[4];
+          uint32_t mw4[4];
           const float4* cs =
               ROPE ? reinterpret_cast<const float4*>(s_tab + rowoff[r] + col.pair_off) : nullptr;
-          const uint4 o = phi_rope<ROPE>(raw, cs, f);
+          const uint4 o = phi_rope<ROPE>(raw, cs, f, mw4);
 #pragma unroll
           for (int e = 0; e < 4; ++e) z2[e] = ptx::add2(z2[e], f[e]);
           ptx::st_shared_v4(addr, o);
@@ -833,7 +846,7 @@ finalize_images(const float* __restrict__ partials, const __grid_constant__ Sche
             for (int i = 2; i < np[k]; ++i)
               blk = add4(blk, __ldg(reinterpret_cast<const float4*>(p + (long long)i * DD1)));
             run = add4(run, blk);
-            store_image4<D>(ibase + (long long)(j0 + jb + k) * image_bytes(D), zrow, run);
+            store_image4<D>(ibase + (long long)(j0 + jb + k) * image_bytes(D), zrow, a0, run);
           }
         }
       }
@@ -851,8 +864,22 @@ finalize_images(const float* __restrict__ partials, const __grid_constant__ Sche
 }
 
 // ---- apply ---------------------------------------------------------------------------
+//
+// Per 128-token tile of q (TMA, 128-byte swizzle) the math warps write
+// A = RoPE(phi(q)) in place over the tile (bf16: the MMA's A operand in shared
+// memory) and phi(q) into tensor memory. The MMA warp accumulates, in
+// accumulator buffer b,
+//   columns [0, D)      A S_hi + A S_lo        (numerator, S in two bf16 halves)
+//   columns [D, D + 16) phi(q) [z_hi, z_lo, 0 ...]   (denominator parts)
+// and the epilogue (the math warps, one tile behind their transform) writes
+// out = acc / (eps + den) (* sigmoid(g)) as bf16 over the tile, which the store
+// warp sends out with TMA.
 
 constexpr int kTcThreadsApply = 96 + kMath;  // warp 0 load, 1 MMA, 2-17 math, 18 store
+
+__host__ __device__ constexpr uint32_t tmem_cols_pow2(uint32_t n) {
+  return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : (n <= 256 ? 256 : 512)));
+}
 
 template <int D, bool ROPE, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
@@ -865,15 +892,17 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   constexpr int HALF_BYTES = TM * 128;
   constexpr int TILE_BYTES = HALVES * HALF_BYTES;
   constexpr int SHALF = 2 * D * 128;         // one K-half of an image: S_hi^T, S_lo^T rows
-  constexpr int CPR = D / 8;
-  constexpr int WPC = kMathWarps / CPR;      // warps per chunk column
-  constexpr int IPW = TM / 32 / WPC;         // 32-row groups per warp and tile
+  constexpr int CPR = D / 8;                 // 16-byte chunks per row
+  constexpr int CPW = CPR / 4;               // chunks per math warp (4 warps per row group)
   constexpr int KSTEPS = D / 16;
-  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, D, 0, 0);
-  constexpr uint32_t TMEM_COLS = 2 * D;      // two accumulators of D columns
+  constexpr uint32_t ACC_COLS = D + 16;      // numerator + denominator block
+  constexpr uint32_t PHI0 = 2 * ACC_COLS;    // phi(q) buffers: D / 2 columns each
+  constexpr uint32_t TMEM_COLS = tmem_cols_pow2(PHI0 + D);
+  constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(TM, D, 0, 0);
+  constexpr uint32_t IDESC_Z = ptx::idesc_bf16_f32(TM, 16, 0, 0);
   constexpr uint32_t TX = (GATE ? 2 : 1) * TILE_BYTES;
   constexpr int EC = D / 4;                  // epilogue columns per thread
-  static_assert(WPC >= 1 && IPW * WPC * 32 == TM, "tile must split over the math warps");
+  static_assert(CPW >= 1 && CPW * 4 == CPR, "chunks must split over 4 warps per row group");
   const int tps = (L + TM - 1) / TM;
 
   extern __shared__ uint8_t smem_raw[];
@@ -882,7 +911,6 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   uint8_t* sm = smem_raw + (base - raw_addr);
   const ApplyPlan P = apply_plan(D, ROPE ? rope.entries : 0, GATE ? 1 : 0, stages, sbuf);
   const uint32_t gbase = base + P.off_g;
-  float* s_den = reinterpret_cast<float*>(sm + P.off_den);   // [stage][chunk][row]
   constexpr uint32_t IMG = image_bytes(D);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
   uint16_t* s_pos = reinterpret_cast<uint16_t*>(sm + P.off_pos);
@@ -916,7 +944,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       ptx::mbar_init(accf_bar(b), 1);
       ptx::mbar_init(acce_bar(b), kMath);
       ptx::mbar_init(sfull_bar(b), 1);
-      ptx::mbar_init(sempty_bar(b), 1 + kMathWarps);
+      ptx::mbar_init(sempty_bar(b), 1);
     }
     ptx::mbar_init(done_bar, 1);
     ptx::fence_mbar_init();
@@ -930,6 +958,53 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   // table are read only after the kernels that write them have completed
   ptx::grid_dependency_wait();
 
+  // out = acc / (eps + den) (* sigmoid(g)) as bf16, over the q tile
+  auto epilogue = [&](int s, int eb, uint32_t ebph, int row, uint32_t lane_bits, int col0) {
+    const bool ready = wait_bounded(accf_bar(eb), ebph, flag, kFlagApplyTimeout, &s_abort);
+    ptx::tc_fence_after();
+    const uint32_t lane_base = *s_tmem + lane_bits + (uint32_t)eb * ACC_COLS;
+    uint32_t vh[EC], dz[2];
+    tmem_ld_cols<EC>(lane_base + col0, vh);
+    ptx::tmem_ld_32x32_x2(lane_base + D, dz);
+    ptx::tmem_wait_ld();
+    if (ready) {
+      const float inv = 1.f / (eps + (__uint_as_float(dz[0]) + __uint_as_float(dz[1])));
+      const uint64_t inv2 = ptx::f2(inv, inv);
+      const uint32_t qt = base + s * TILE_BYTES;
+      const uint32_t gt = gbase + s * TILE_BYTES;
+      const int h = col0 / 64;
+#pragma unroll
+      for (int k4 = 0; k4 < EC / 8; ++k4) {
+        const int chunk = (col0 % 64) / 8 + k4;
+        const uint32_t off = h * HALF_BYTES + row * 128 + ((chunk ^ (row & 7)) << 4);
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint64_t hv = ptx::f2(__uint_as_float(vh[8 * k4 + 2 * e]),
+                                      __uint_as_float(vh[8 * k4 + 2 * e + 1]));
+          ptx::f2_split(ptx::mul2(hv, inv2), o[2 * e], o[2 * e + 1]);
+        }
+        if (GATE) {
+          const uint4 gr = ptx::ld_shared_v4(gt + off);
+          const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o[2 * e] *= 1.f / (1.f + __expf(-ptx::bf16_lo(gw[e])));
+            o[2 * e + 1] *= 1.f / (1.f + __expf(-ptx::bf16_hi(gw[e])));
+          }
+        }
+        ptx::st_shared_v4(qt + off, make_uint4(ptx::pack_bf16x2(o[0], o[1]),
+                                                ptx::pack_bf16x2(o[2], o[3]),
+                                                ptx::pack_bf16x2(o[4], o[5]),
+                                                ptx::pack_bf16x2(o[6], o[7])));
+      }
+    }
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(acce_bar(eb));
+    ptx::fence_proxy_async();
+    ptx::mbar_arrive(oready_bar(s));
+  };
+
   if (warp == 0) {
     // ---------------- TMA loads: S images per segment, q (and gate) tiles ----------------
     TileIter it;
@@ -939,7 +1014,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     for (long long u = u0; u < u1; ++u, it.next()) {
       int ok = 1;
       if (it.seg != cur_seg) {
-        // the segment's S image into the next slot, once its last user is done
+        // the segment's image into the next slot, once its last user is done
         cur_seg = it.seg;
         ++ss;
         if (lane == 0) {
@@ -983,7 +1058,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                      &s_abort);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer: acc[b] = RoPE(phi q) S_hi + RoPE(phi q) S_lo ----------
+    // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t tmem = *s_tmem;
       TileIter it;
@@ -1007,17 +1082,25 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           break;
         ptx::tc_fence_after();
         const uint32_t qt = base + it.stage * TILE_BYTES;
-        const uint32_t acc = tmem + (uint32_t)(b * D);
+        const uint32_t acc = tmem + (uint32_t)b * ACC_COLS;
+        const uint32_t phi = tmem + PHI0 + (uint32_t)b * (D / 2);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
           // the hi and lo halves of S accumulate into the same columns
           const uint32_t aoff = (kk / 4) * HALF_BYTES + (kk % 4) * 32;
           const uint32_t boff = (kk / 4) * SHALF + (kk % 4) * 32;
           const uint64_t adesc = ptx::smem_desc_sw128(qt + aoff, 16, 1024);
-          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(Sb + boff, 16, 1024), IDESC,
+          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(Sb + boff, 16, 1024), IDESC_S,
                         kk == 0 ? 0u : 1u);
-          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(Sb + boff + D * 128, 16, 1024), IDESC,
-                        1u);
+          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(Sb + boff + D * 128, 16, 1024),
+                        IDESC_S, 1u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          // denominator: phi(q) from tensor memory (8 columns per K step)
+          const uint32_t zoff = image_zoff(D) + (kk / 4) * 2048 + (kk % 4) * 32;
+          ptx::mma_bf16_ta(acc + D, phi + 8u * kk, ptx::smem_desc_sw128(Sb + zoff, 16, 1024),
+                           IDESC_Z, kk == 0 ? 0u : 1u);
         }
         ptx::mma_commit(accf_bar(b));
         // the slot is free for the next image once this segment's MMAs are done
@@ -1048,135 +1131,59 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       }
       ptx::bulk_wait<0>();
     }
-  } else {
-    // ---------------- math warps: phi(q), den, RoPE; epilogue ----------------
+  } else if (warp < 2 + kMathWarps) {
+    // ---------------- math warps: phi(q), RoPE; epilogue ----------------
+    // A warp owns the 32 rows of its TMEM lane quadrant and CPW chunk columns.
     const int tt = threadIdx.x - 64;
-    const int mw = warp - 2;
-    const int c = mw % CPR, rg0 = mw / CPR;      // chunk column, first row group
-    const int half = c >> 3, cc = c & 7;
-    const int q4 = warp & 3, quarter = mw >> 2;  // TMEM lane quadrant, column quarter
-    const int erow = 32 * q4 + lane;             // epilogue row = TMEM lane
+    const int q4 = warp & 3;                     // TMEM lane quadrant = row group
+    const int jw = (warp - 2) >> 2;              // warp within the quadrant, 0..3
+    const int row = 32 * q4 + lane;              // tile row of this thread
+    const uint32_t lane_bits = (uint32_t)(32 * q4) << 16;
     if (ROPE)
       for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = gtab[e];
-    ChunkCol col{};
-    if (ROPE) col = chunk_col(rope, c);
-    const uint32_t tmem = *s_tmem;
-    uint64_t zc2[4];
+    ChunkCol col[CPW];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) zc2[e] = ptx::f2(0.f, 0.f);
-    int cur_seg = -1, ss = -1;
+    for (int i = 0; i < CPW; ++i) col[i] = ROPE ? chunk_col(rope, jw * CPW + i) : ChunkCol{};
+    if (ROPE) ptx::bar_sync(1, kMath);           // table complete before the first lookup
+    const uint32_t tmem = *s_tmem;
     int pend_stage = -1, pend_b = 0;
-    uint32_t pend_bph = 0, pend_ph = 0;
+    uint32_t pend_bph = 0;
     int b = 0;
     uint32_t bph = 0;
-
-    // out = acc / den (* sigmoid(g)) as bf16, over the q tile
-    auto epilogue = [&](int s, uint32_t sph, int eb, uint32_t ebph) {
-      // all den partials of the tile are in shared memory once every math
-      // thread has arrived on the tile's qready barrier
-      const bool seen = wait_bounded(qready_bar(s), sph, flag, kFlagApplyTimeout, &s_abort);
-      const bool ready =
-          wait_bounded(accf_bar(eb), ebph, flag, kFlagApplyTimeout, &s_abort) && seen;
-      ptx::tc_fence_after();
-      float den = eps;
-      const float* dp = s_den + s * CPR * TM + erow;
-#pragma unroll
-      for (int ch = 0; ch < CPR; ++ch) den += dp[ch * TM];
-      const float inv = 1.f / den;
-      const uint64_t inv2 = ptx::f2(inv, inv);
-      const uint32_t qt = base + s * TILE_BYTES;
-      const uint32_t gt = gbase + s * TILE_BYTES;
-      const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(eb * D);
-      const int col0 = quarter * EC;
-      uint32_t vh[EC];
-      tmem_ld_cols<EC>(lane_base + col0, vh);
-      ptx::tmem_wait_ld();
-      if (ready) {
-        const int h = col0 / 64;
-#pragma unroll
-        for (int k4 = 0; k4 < EC / 8; ++k4) {
-          const int chunk = (col0 % 64) / 8 + k4;
-          const uint32_t off = h * HALF_BYTES + erow * 128 + ((chunk ^ (erow & 7)) << 4);
-          float o[8];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint64_t hv = ptx::f2(__uint_as_float(vh[8 * k4 + 2 * e]),
-                                        __uint_as_float(vh[8 * k4 + 2 * e + 1]));
-            ptx::f2_split(ptx::mul2(hv, inv2), o[2 * e], o[2 * e + 1]);
-          }
-          if (GATE) {
-            const uint4 gr = ptx::ld_shared_v4(gt + off);
-            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              o[2 * e] *= 1.f / (1.f + __expf(-ptx::bf16_lo(gw[e])));
-              o[2 * e + 1] *= 1.f / (1.f + __expf(-ptx::bf16_hi(gw[e])));
-            }
-          }
-          ptx::st_shared_v4(qt + off, make_uint4(ptx::pack_bf16x2(o[0], o[1]),
-                                                  ptx::pack_bf16x2(o[2], o[3]),
-                                                  ptx::pack_bf16x2(o[4], o[5]),
-                                                  ptx::pack_bf16x2(o[6], o[7])));
-        }
-      }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(acce_bar(eb));
-      ptx::fence_proxy_async();
-      ptx::mbar_arrive(oready_bar(s));
-    };
 
     TileIter it;
     it.init(u0, tps, stages);
     for (long long u = u0; u < u1; ++u, it.next()) {
-      if (it.seg != cur_seg) {
-        // the segment's image is in slot k: take z of this warp's chunk
-        cur_seg = it.seg;
-        ++ss;
-        const int k = ss % sbuf;
-        const bool got = wait_bounded(sfull_bar(k), (uint32_t)((ss / sbuf) & 1), flag,
-                                      kFlagApplyTimeout, &s_abort);
-        if (got) {
-          const float4* zsrc = reinterpret_cast<const float4*>(
-              sm + P.off_S + (uint32_t)k * image_slot(D) + 4u * D * D + 32u * c);
-          const float4 za = zsrc[0], zb = zsrc[1];
-          // in the packing of phi_rope's xy: (d0,d2), (d4,d6), (d1,d3), (d5,d7)
-          zc2[0] = ptx::f2(za.x, za.z);
-          zc2[1] = ptx::f2(zb.x, zb.z);
-          zc2[2] = ptx::f2(za.y, za.w);
-          zc2[3] = ptx::f2(zb.y, zb.w);
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(sempty_bar(k));
-      }
       const bool ok = wait_bounded(full_bar(it.stage), it.phase, flag, kFlagApplyTimeout,
                                    &s_abort);
       if (ok) {
-        const uint32_t qt = base + it.stage * TILE_BYTES + half * HALF_BYTES;
-        const uint16_t* rowoff = s_pos + (it.stage * 3 + col.ax) * TM;
-        float* dst_den = s_den + (it.stage * CPR + c) * TM;
+        // A = RoPE(phi q) in place; phi q into the tensor memory of buffer b,
+        // whose last reader (the MMAs of two tiles ago) the epilogue of the
+        // previous tile has waited for
+        const uint32_t tphi = tmem + lane_bits + PHI0 + (uint32_t)b * (D / 2);
 #pragma unroll
-        for (int i = 0; i < IPW; ++i) {
-          const int r = 32 * (rg0 + WPC * i) + lane;
-          const uint32_t addr = qt + r * 128 + ((cc ^ (r & 7)) << 4);
+        for (int i = 0; i < CPW; ++i) {
+          const int c = jw * CPW + i;
+          const uint32_t addr = base + it.stage * TILE_BYTES + (c >> 3) * HALF_BYTES +
+                                row * 128 + (((c & 7) ^ (row & 7)) << 4);
           const uint4 raw = ptx::ld_shared_v4(addr);
-          uint64_t f[4];
+          uint64_t xy[4];
+          uint32_t m[4];
           const float4* cs =
-              ROPE ? reinterpret_cast<const float4*>(s_tab + rowoff[r] + col.pair_off) : nullptr;
-          const uint4 o = phi_rope<ROPE>(raw, cs, f);
-          uint64_t d2 = ptx::mul2(f[0], zc2[0]);
-#pragma unroll
-          for (int e = 1; e < 4; ++e) d2 = ptx::fma2(f[e], zc2[e], d2);
-          float dlo, dhi;
-          ptx::f2_split(d2, dlo, dhi);
-          dst_den[r] = dlo + dhi;
+              ROPE ? reinterpret_cast<const float4*>(
+                         s_tab + s_pos[(it.stage * 3 + col[i].ax) * TM + row] + col[i].pair_off)
+                   : nullptr;
+          const uint4 o = phi_rope<ROPE>(raw, cs, xy, m);
           ptx::st_shared_v4(addr, o);
+          ptx::tmem_st_32x32_x4(tphi + 4u * c, m);
         }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
         ptx::fence_proxy_async();
         ptx::mbar_arrive(qready_bar(it.stage));
       }
-      if (pend_stage >= 0) epilogue(pend_stage, pend_ph, pend_b, pend_bph);
+      if (pend_stage >= 0) epilogue(pend_stage, pend_b, pend_bph, row, lane_bits, jw * EC);
       pend_stage = it.stage;
-      pend_ph = it.phase;
       pend_b = b;
       pend_bph = bph;
       if (++b == 2) {
@@ -1184,7 +1191,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         bph ^= 1u;
       }
     }
-    if (pend_stage >= 0) epilogue(pend_stage, pend_ph, pend_b, pend_bph);
+    if (pend_stage >= 0) epilogue(pend_stage, pend_b, pend_bph, row, lane_bits, jw * EC);
   }
   __syncthreads();
   if (warp == 1) {
