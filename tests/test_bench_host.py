@@ -1,0 +1,115 @@
+"""Host-side logic of bench.py on the CPU: the reference arm's JSON line, the
+max-over-ranks timing and barrier over a two-rank gloo group, the launch
+count and the committed-profile traffic lookup."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import workloads  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _json_lines(text):
+    return [json.loads(l) for l in text.splitlines() if l.startswith("{")]
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1
+    d = lines[0]
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["value"] > 0
+    assert d["config"]["workload"] == "480p_bidir"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_under_two_ranks_prints_once():
+    port = _free_port()
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1", "--master-port",
+                        str(port), "bench.py", "--impl", "reference", "--gpus", "2", "--steps",
+                        "1", "--warmup", "0"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1 and lines[0]["n_gpus"] == 2
+
+
+def _rank_main(rank, port, values, out):
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank,
+                            world_size=2)
+    bench.barrier(dist)
+    out[rank] = bench.reduce_max(values[rank], dist)
+    bench.barrier(dist)
+    dist.destroy_process_group()
+
+
+def test_reduce_max_and_barrier_over_gloo():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank_main, args=(port, [1.5, 4.25], out), nprocs=2, join=True)
+        assert dict(out) == {0: 4.25, 1: 4.25}
+
+
+def test_reduce_max_without_group_is_identity():
+    assert bench.reduce_max(3.0, None) == 3.0
+
+
+def test_launches_per_forward():
+    W = workloads.WORKLOADS
+    assert bench.launches_per_forward(W["480p_bidir"], "bidirectional") == 2
+    assert bench.launches_per_forward(W["480p_block_causal"], "block_causal") == 3
+    assert bench.launches_per_forward(W["720p_long"], "block_causal") == 3
+
+
+def test_profile_traffic_lookup_is_tied_to_the_sources(tmp_path, monkeypatch):
+    # a committed line counts only while its source hash matches the kernels
+    h = bench.kernel_source_hash()
+    assert len(h) == 12
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    csrc = tmp_path / "linear_attention_video_relu_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("// kernel\n")
+    h2 = bench.kernel_source_hash()
+    (tmp_path / "profiles" / "x.txt").write_text(
+        "# bench-traffic apply 480p_bidir 123 %s\n# bench-traffic apply 720p_long 9 %s\n"
+        "# bench-traffic state_build 480p_bidir 77 000000000000\n" % (h2, h2))
+    assert bench.ncu_traffic("apply", "480p_bidir") == 123
+    assert bench.ncu_traffic("apply", "720p_long") == 9
+    assert bench.ncu_traffic("state_build", "480p_bidir") is None
+
+
+def test_committed_profiles_name_their_command():
+    pdir = os.path.join(ROOT, "profiles")
+    names = [n for n in os.listdir(pdir) if n.endswith((".txt", ".md"))]
+    assert names
+    for n in names:
+        text = open(os.path.join(pdir, n)).read()
+        assert "ncu " in text and "bench.py" in text, n
+        assert len(text) < 8192, n
