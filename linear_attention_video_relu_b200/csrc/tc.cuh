@@ -73,7 +73,7 @@ struct StatePlan {
 };
 
 struct ApplyPlan {
-  int stages, sbuf;
+  int stages, sbuf, gst;
   uint32_t off_g, off_S, off_tab, off_pos, off_bar, off_tmem, total;
 };
 
@@ -108,14 +108,15 @@ __host__ __device__ inline StatePlan state_plan(int D, int entries, int stages) 
 }
 
 __host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, int stages,
-                                                int sbuf) {
+                                                int sbuf, int gst) {
   ApplyPlan p;
   const uint32_t tile = (uint32_t)kApplyTile * D * 2;
   p.stages = stages;
   p.sbuf = sbuf;
-  uint32_t off = stages * tile;
-  p.off_g = off;
-  off += gate ? stages * tile : 0;
+  p.gst = gate ? gst : 0;
+  uint32_t off = stages * tile;   // q stages
+  p.off_g = off;                  // gate tiles: one per stage, or a ring of their own
+  off += p.gst * tile;
   p.off_S = align_up(off, 1024);
   off = p.off_S + sbuf * image_slot(D);  // B-operand images, one per S slot
   p.off_tab = align_up(off, 32);
@@ -123,7 +124,7 @@ __host__ __device__ inline ApplyPlan apply_plan(int D, int entries, int gate, in
   p.off_pos = align_up(off, 16);
   off = p.off_pos + (entries ? stages * 3u * kApplyTile * 2 : 0);
   p.off_bar = align_up(off, 8);
-  off = p.off_bar + (4u * stages + 9u) * 8u;
+  off = p.off_bar + (4u * stages + 9u + 2u * p.gst) * 8u;
   p.off_tmem = off;
   off += 16;
   p.total = off + 1024;
@@ -136,27 +137,37 @@ inline int pick_state_stages(int D, int entries) {
   return 0;
 }
 
+// The apply kernel's output path: at D = 64 the epilogue writes out over the
+// q tile and a TMA store sends it (the stage is freed after the store); at
+// D = 128 (larger tiles, fewer stages fit) the epilogue stores straight from
+// registers, the MMAs free the q stage, and gate tiles have a ring of their own.
+__host__ __device__ constexpr bool apply_direct_out(int D) { return D == 128; }
+
 // Two S slots (the next segment's image prefetched while the current one is
-// in use) when at least 4 stages still fit, else one slot and the most stages.
-inline void pick_apply_plan(int D, int entries, int gate, int* stages, int* sbuf) {
+// in use) when at least 4 q stages still fit, else one slot and the most
+// stages.
+inline void pick_apply_plan(int D, int entries, int gate, int* stages, int* sbuf, int* gst) {
   *stages = 0;
   *sbuf = 1;
+  auto g = [&](int s) { return gate ? (apply_direct_out(D) ? 2 : s) : 0; };
   for (int s = 8; s >= 4; --s)
-    if (apply_plan(D, entries, gate, s, 2).total <= (uint32_t)kSmemBudget) {
+    if (apply_plan(D, entries, gate, s, 2, g(s)).total <= (uint32_t)kSmemBudget) {
       *stages = s;
       *sbuf = 2;
+      *gst = g(s);
       return;
     }
   for (int s = 8; s >= 2; --s)
-    if (apply_plan(D, entries, gate, s, 1).total <= (uint32_t)kSmemBudget) {
+    if (apply_plan(D, entries, gate, s, 1, g(s)).total <= (uint32_t)kSmemBudget) {
       *stages = s;
+      *gst = g(s);
       return;
     }
 }
 
 inline int pick_apply_stages(int D, int entries, int gate) {
-  int st, sb;
-  pick_apply_plan(D, entries, gate, &st, &sb);
+  int st, sb, gs;
+  pick_apply_plan(D, entries, gate, &st, &sb, &gs);
   return st;
 }
 
@@ -871,11 +882,14 @@ finalize_images(const float* __restrict__ partials, const __grid_constant__ Sche
 // accumulator buffer b,
 //   columns [0, D)      A S_hi + A S_lo        (numerator, S in two bf16 halves)
 //   columns [D, D + 16) phi(q) [z_hi, z_lo, 0 ...]   (denominator parts)
-// and the epilogue (the math warps, one tile behind their transform) writes
-// out = acc / (eps + den) (* sigmoid(g)) as bf16 over the tile, which the store
-// warp sends out with TMA.
+// and the epilogue (the math warps, one tile behind their transform) forms
+// out = acc / (eps + den) (* sigmoid(g)) as bf16. Output path (apply_direct_out):
+// either over the q tile, sent by warp 18 with a TMA store that then frees the
+// stage; or stored from registers, with the stage freed by the MMAs and gate
+// tiles brought by warp 18 into a ring of their own.
 
-constexpr int kTcThreadsApply = 96 + kMath;  // warp 0 load, 1 MMA, 2-17 math, 18 store
+// warp 0 q (+ gate) tiles and images, 1 MMA, 2-17 math, 18 store or gate loads
+constexpr int kTcThreadsApply = 96 + kMath;
 
 __host__ __device__ constexpr uint32_t tmem_cols_pow2(uint32_t n) {
   return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : (n <= 256 ? 256 : 512)));
@@ -884,8 +898,9 @@ __host__ __device__ constexpr uint32_t tmem_cols_pow2(uint32_t n) {
 template <int D, bool ROPE, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
-         const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ Rope rope, int L,
-         int nblk, long long U, int stages, int sbuf, const uint8_t* __restrict__ images,
+         const __grid_constant__ CUtensorMap tm_o, __nv_bfloat16* __restrict__ out,
+         const __grid_constant__ Rope rope, int L, int nblk,
+         long long U, int stages, int sbuf, int gst, const uint8_t* __restrict__ images,
          const float2* __restrict__ gtab, float eps, int* flag) {
   constexpr int TM = kApplyTile;
   constexpr int HALVES = D / 64;
@@ -900,8 +915,9 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   constexpr uint32_t TMEM_COLS = tmem_cols_pow2(PHI0 + D);
   constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(TM, D, 0, 0);
   constexpr uint32_t IDESC_Z = ptx::idesc_bf16_f32(TM, 16, 0, 0);
-  constexpr uint32_t TX = (GATE ? 2 : 1) * TILE_BYTES;
   constexpr int EC = D / 4;                  // epilogue columns per thread
+  constexpr bool DIRECT = apply_direct_out(D);
+  constexpr uint32_t TX = (!DIRECT && GATE ? 2 : 1) * TILE_BYTES;
   static_assert(CPW >= 1 && CPW * 4 == CPR, "chunks must split over 4 warps per row group");
   const int tps = (L + TM - 1) / TM;
 
@@ -909,7 +925,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
   const uint32_t base = align_up(raw_addr, 1024);
   uint8_t* sm = smem_raw + (base - raw_addr);
-  const ApplyPlan P = apply_plan(D, ROPE ? rope.entries : 0, GATE ? 1 : 0, stages, sbuf);
+  const ApplyPlan P = apply_plan(D, ROPE ? rope.entries : 0, GATE ? 1 : 0, stages, sbuf, gst);
   const uint32_t gbase = base + P.off_g;
   constexpr uint32_t IMG = image_bytes(D);
   float2* s_tab = reinterpret_cast<float2*>(sm + P.off_tab);
@@ -919,11 +935,14 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   auto qready_bar = [&](int s) { return bar0 + 8u * (stages + s); };
   auto empty_bar = [&](int s) { return bar0 + 8u * (2 * stages + s); };
   auto oready_bar = [&](int s) { return bar0 + 8u * (3 * stages + s); };
-  auto accf_bar = [&](int b) { return bar0 + 8u * (4 * stages + b); };
-  auto acce_bar = [&](int b) { return bar0 + 8u * (4 * stages + 2 + b); };
-  auto sfull_bar = [&](int k) { return bar0 + 8u * (4 * stages + 4 + k); };
-  auto sempty_bar = [&](int k) { return bar0 + 8u * (4 * stages + 6 + k); };
-  const uint32_t done_bar = bar0 + 8u * (4 * stages + 8);
+  const uint32_t bar1 = bar0 + 8u * (4 * stages);
+  auto accf_bar = [&](int b) { return bar1 + 8u * b; };
+  auto acce_bar = [&](int b) { return bar1 + 8u * (2 + b); };
+  auto sfull_bar = [&](int k) { return bar1 + 8u * (4 + k); };
+  auto sempty_bar = [&](int k) { return bar1 + 8u * (6 + k); };
+  const uint32_t done_bar = bar1 + 8u * 8;
+  auto gfull_bar = [&](int k) { return bar1 + 8u * (9 + k); };
+  auto gempty_bar = [&](int k) { return bar1 + 8u * (9 + gst + k); };
   auto s_slot = [&](int k) { return base + P.off_S + (uint32_t)k * image_slot(D); };
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P.off_tmem);
   __shared__ int s_abort;
@@ -947,6 +966,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       ptx::mbar_init(sempty_bar(b), 1);
     }
     ptx::mbar_init(done_bar, 1);
+    if (DIRECT)
+      for (int k = 0; k < gst; ++k) {
+        ptx::mbar_init(gfull_bar(k), 1);
+        ptx::mbar_init(gempty_bar(k), kMath);
+      }
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
@@ -957,53 +981,6 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   // launched early (programmatic dependent launch): the images and the RoPE
   // table are read only after the kernels that write them have completed
   ptx::grid_dependency_wait();
-
-  // out = acc / (eps + den) (* sigmoid(g)) as bf16, over the q tile
-  auto epilogue = [&](int s, int eb, uint32_t ebph, int row, uint32_t lane_bits, int col0) {
-    const bool ready = wait_bounded(accf_bar(eb), ebph, flag, kFlagApplyTimeout, &s_abort);
-    ptx::tc_fence_after();
-    const uint32_t lane_base = *s_tmem + lane_bits + (uint32_t)eb * ACC_COLS;
-    uint32_t vh[EC], dz[2];
-    tmem_ld_cols<EC>(lane_base + col0, vh);
-    ptx::tmem_ld_32x32_x2(lane_base + D, dz);
-    ptx::tmem_wait_ld();
-    if (ready) {
-      const float inv = 1.f / (eps + (__uint_as_float(dz[0]) + __uint_as_float(dz[1])));
-      const uint64_t inv2 = ptx::f2(inv, inv);
-      const uint32_t qt = base + s * TILE_BYTES;
-      const uint32_t gt = gbase + s * TILE_BYTES;
-      const int h = col0 / 64;
-#pragma unroll
-      for (int k4 = 0; k4 < EC / 8; ++k4) {
-        const int chunk = (col0 % 64) / 8 + k4;
-        const uint32_t off = h * HALF_BYTES + row * 128 + ((chunk ^ (row & 7)) << 4);
-        float o[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint64_t hv = ptx::f2(__uint_as_float(vh[8 * k4 + 2 * e]),
-                                      __uint_as_float(vh[8 * k4 + 2 * e + 1]));
-          ptx::f2_split(ptx::mul2(hv, inv2), o[2 * e], o[2 * e + 1]);
-        }
-        if (GATE) {
-          const uint4 gr = ptx::ld_shared_v4(gt + off);
-          const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            o[2 * e] *= 1.f / (1.f + __expf(-ptx::bf16_lo(gw[e])));
-            o[2 * e + 1] *= 1.f / (1.f + __expf(-ptx::bf16_hi(gw[e])));
-          }
-        }
-        ptx::st_shared_v4(qt + off, make_uint4(ptx::pack_bf16x2(o[0], o[1]),
-                                                ptx::pack_bf16x2(o[2], o[3]),
-                                                ptx::pack_bf16x2(o[4], o[5]),
-                                                ptx::pack_bf16x2(o[6], o[7])));
-      }
-    }
-    ptx::tc_fence_before();
-    ptx::mbar_arrive(acce_bar(eb));
-    ptx::fence_proxy_async();
-    ptx::mbar_arrive(oready_bar(s));
-  };
 
   if (warp == 0) {
     // ---------------- TMA loads: S images per segment, q (and gate) tiles ----------------
@@ -1042,7 +1019,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         for (int h = 0; h < HALVES; ++h) {
           ptx::tma_load_3d(base + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_q, 64 * h,
                            it.tile * TM, it.seg, full_bar(it.stage));
-          if (GATE)
+          if (!DIRECT && GATE)
             ptx::tma_load_3d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h,
                              it.tile * TM, it.seg, full_bar(it.stage));
         }
@@ -1103,7 +1080,9 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                            IDESC_Z, kk == 0 ? 0u : 1u);
         }
         ptx::mma_commit(accf_bar(b));
-        // the slot is free for the next image once this segment's MMAs are done
+        // (direct output) the q stage and, after a segment's last tile, the
+        // image slot are free once these MMAs have read them
+        if (DIRECT) ptx::mma_commit(empty_bar(it.stage));
         if (it.last_of_segment(u, u1)) ptx::mma_commit(sempty_bar(ss % sbuf));
         if (++b == 2) {
           b = 0;
@@ -1114,8 +1093,8 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       wait_bounded(done_bar, 0, flag, kFlagApplyTimeout, &s_abort);
     }
   } else if (warp == 2 + kMathWarps) {
-    // ---------------- TMA stores: out tiles, then free the stage ----------------
-    if (lane == 0) {
+    if (!DIRECT && lane == 0) {
+      // ---------------- TMA stores: out tiles, then free the stage ----------------
       TileIter it;
       it.init(u0, tps, stages);
       for (long long u = u0; u < u1; ++u, it.next()) {
@@ -1131,7 +1110,27 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       }
       ptx::bulk_wait<0>();
     }
-  } else if (warp < 2 + kMathWarps) {
+    if (DIRECT && GATE && lane == 0) {
+      // ---------------- TMA loads of gate tiles into their own ring ----------------
+      TileIter it;
+      it.init(u0, tps, gst);
+      long long issued = 0;
+      for (long long u = u0; u < u1; ++u, it.next()) {
+        if (!wait_bounded(gempty_bar(it.stage), it.phase ^ 1u, flag, kFlagApplyTimeout,
+                          &s_abort))
+          break;
+        ptx::mbar_expect_tx(gfull_bar(it.stage), TILE_BYTES);
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h)
+          ptx::tma_load_3d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h,
+                           it.tile * TM, it.seg, gfull_bar(it.stage));
+        ++issued;
+      }
+      for (long long i = issued - gst < 0 ? 0 : issued - gst; i < issued; ++i)
+        wait_bounded(gfull_bar((int)(i % gst)), (uint32_t)((i / gst) & 1), flag,
+                     kFlagApplyTimeout, &s_abort);
+    }
+  } else {
     // ---------------- math warps: phi(q), RoPE; epilogue ----------------
     // A warp owns the 32 rows of its TMEM lane quadrant and CPW chunk columns.
     const int tt = threadIdx.x - 64;
@@ -1139,18 +1138,77 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     const int jw = (warp - 2) >> 2;              // warp within the quadrant, 0..3
     const int row = 32 * q4 + lane;              // tile row of this thread
     const uint32_t lane_bits = (uint32_t)(32 * q4) << 16;
-    if (ROPE)
+    const int col0 = jw * EC;                    // epilogue columns of this thread
+    if (ROPE) {
       for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = gtab[e];
+      ptx::bar_sync(1, kMath);                   // table complete before the first lookup
+    }
     ChunkCol col[CPW];
 #pragma unroll
     for (int i = 0; i < CPW; ++i) col[i] = ROPE ? chunk_col(rope, jw * CPW + i) : ChunkCol{};
-    if (ROPE) ptx::bar_sync(1, kMath);           // table complete before the first lookup
     const uint32_t tmem = *s_tmem;
-    int pend_stage = -1, pend_b = 0;
-    uint32_t pend_bph = 0;
+
+    // out rows of tile (seg, tile) in stage s: acc / (eps + den) (* sigmoid(g))
+    // as bf16, over the q tile or (direct) from registers to global memory,
+    // where rows past the segment's end are not stored
+    auto epilogue = [&](int s, int seg, int tile, int eb, uint32_t ebph, int gs, uint32_t gph) {
+      const bool ready = wait_bounded(accf_bar(eb), ebph, flag, kFlagApplyTimeout, &s_abort);
+      const bool gready = !(DIRECT && GATE) ||
+                          wait_bounded(gfull_bar(gs), gph, flag, kFlagApplyTimeout, &s_abort);
+      ptx::tc_fence_after();
+      const uint32_t lane_base = tmem + lane_bits + (uint32_t)eb * ACC_COLS;
+      uint32_t vh[EC], dz[2];
+      tmem_ld_cols<EC>(lane_base + col0, vh);
+      ptx::tmem_ld_32x32_x2(lane_base + D, dz);
+      ptx::tmem_wait_ld();
+      const int r = tile * TM + row;
+      if (ready && gready && (!DIRECT || r < L)) {
+        const float inv = 1.f / (eps + (__uint_as_float(dz[0]) + __uint_as_float(dz[1])));
+        const uint64_t inv2 = ptx::f2(inv, inv);
+        uint4* dst = reinterpret_cast<uint4*>(out + ((long long)seg * L + r) * D + col0);
+        const uint32_t gt = gbase + (DIRECT ? gs : s) * TILE_BYTES;
+        const int h = col0 / 64;
+#pragma unroll
+        for (int k4 = 0; k4 < EC / 8; ++k4) {
+          float o[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint64_t hv = ptx::f2(__uint_as_float(vh[8 * k4 + 2 * e]),
+                                        __uint_as_float(vh[8 * k4 + 2 * e + 1]));
+            ptx::f2_split(ptx::mul2(hv, inv2), o[2 * e], o[2 * e + 1]);
+          }
+          const int chunk = (col0 % 64) / 8 + k4;
+          const uint32_t off = h * HALF_BYTES + row * 128 + ((chunk ^ (row & 7)) << 4);
+          if (GATE) {
+            const uint4 gr = ptx::ld_shared_v4(gt + off);
+            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              o[2 * e] *= __frcp_rn(1.f + __expf(-ptx::bf16_lo(gw[e])));
+              o[2 * e + 1] *= __frcp_rn(1.f + __expf(-ptx::bf16_hi(gw[e])));
+            }
+          }
+          const uint4 ov = make_uint4(ptx::pack_bf16x2(o[0], o[1]), ptx::pack_bf16x2(o[2], o[3]),
+                                      ptx::pack_bf16x2(o[4], o[5]), ptx::pack_bf16x2(o[6], o[7]));
+          if (DIRECT) dst[k4] = ov;
+          else ptx::st_shared_v4(base + s * TILE_BYTES + off, ov);
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(acce_bar(eb));
+      if (DIRECT && GATE) ptx::mbar_arrive(gempty_bar(gs));
+      if (!DIRECT) {
+        ptx::fence_proxy_async();
+        ptx::mbar_arrive(oready_bar(s));
+      }
+    };
+
+    int pend_stage = -1, pend_seg = 0, pend_tile = 0, pend_b = 0, pend_g = 0;
+    uint32_t pend_bph = 0, pend_gph = 0;
     int b = 0;
     uint32_t bph = 0;
-
+    int gslot = 0;
+    uint32_t gphase = 0;
     TileIter it;
     it.init(u0, tps, stages);
     for (long long u = u0; u < u1; ++u, it.next()) {
@@ -1182,16 +1240,26 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         ptx::fence_proxy_async();
         ptx::mbar_arrive(qready_bar(it.stage));
       }
-      if (pend_stage >= 0) epilogue(pend_stage, pend_b, pend_bph, row, lane_bits, jw * EC);
+      if (pend_stage >= 0)
+        epilogue(pend_stage, pend_seg, pend_tile, pend_b, pend_bph, pend_g, pend_gph);
       pend_stage = it.stage;
+      pend_seg = it.seg;
+      pend_tile = it.tile;
       pend_b = b;
       pend_bph = bph;
+      pend_g = gslot;
+      pend_gph = gphase;
       if (++b == 2) {
         b = 0;
         bph ^= 1u;
       }
+      if (DIRECT && GATE && ++gslot == gst) {
+        gslot = 0;
+        gphase ^= 1u;
+      }
     }
-    if (pend_stage >= 0) epilogue(pend_stage, pend_b, pend_bph, row, lane_bits, jw * EC);
+    if (pend_stage >= 0)
+      epilogue(pend_stage, pend_seg, pend_tile, pend_b, pend_bph, pend_g, pend_gph);
   }
   __syncthreads();
   if (warp == 1) {
@@ -1321,17 +1389,18 @@ la_status tc_run_d(const TcArgs& a, int sms) {
       !make_map(&mo, a.out, D, sc.L, sc.nseg, kApplyTile) ||
       !make_map(&mg, gate ? a.g : a.q, D, sc.L, sc.nseg, kApplyTile))
     return LA_ERR_CUDA;
-  int s3 = 0, sb3 = 1;
-  pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3);
-  const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3, sb3);
+  int s3 = 0, sb3 = 1, gs3 = 0;
+  pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3, &gs3);
+  const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3, sb3, gs3);
   const long long U3 = (long long)sc.nseg * ((sc.L + kApplyTile - 1) / kApplyTile);
   const int G3 = (int)(U3 < sms ? U3 : sms);
   auto k3 = a.rope.on ? (gate ? apply_tc<D, true, true> : apply_tc<D, true, false>)
                       : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
   if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
-  st = launch_pdl(k3, dim3(G3), dim3(kTcThreadsApply), p3.total, a.stream, mq, mg, mo, a.rope,
-                  sc.L, sc.nblk, U3, s3, sb3, reinterpret_cast<const uint8_t*>(a.apply),
-                  (const float2*)a.gtab, a.eps, a.flag);
+  st = launch_pdl(k3, dim3(G3), dim3(kTcThreadsApply), p3.total, a.stream, mq, mg, mo,
+                  static_cast<__nv_bfloat16*>(a.out), a.rope, sc.L, sc.nblk, U3, s3, sb3, gs3,
+                  reinterpret_cast<const uint8_t*>(a.apply), (const float2*)a.gtab, a.eps,
+                  a.flag);
   if (st != LA_OK) return st;
   return tc_mark(a, 3);
 }
