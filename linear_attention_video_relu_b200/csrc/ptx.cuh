@@ -118,6 +118,12 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Orders this thread's view of global memory (including writes of other CTAs
+// it has acquired) before its later async-proxy (bulk copy) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---- programmatic dependent launch -------------------------------------------------
 
 // Blocks until the grids this one depends on have completed and their memory

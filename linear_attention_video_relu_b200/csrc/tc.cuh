@@ -100,7 +100,7 @@ __host__ __device__ inline StatePlan state_plan(int D, int entries, int stages) 
   p.off_z = off;
   off += 2u * 16 * 8 * 4;  // z of each math warp (8 values), per accumulator buffer
   p.off_bar = align_up(off, 8);
-  off = p.off_bar + (3u * stages + 9u) * 8u;
+  off = p.off_bar + (3u * stages + 10u) * 8u;
   p.off_tmem = off;
   off += 16;
   p.total = off + 1024;  // slack to align the base to 1024 bytes
@@ -477,11 +477,50 @@ __device__ void reduce_segment(const float* __restrict__ partials, const Sched& 
   }
 }
 
+// reduce_segment over np partial slots already copied to shared memory
+// (slot i at sp + i * D(D + 1)): the same fp32 operations in the same order.
+template <int D>
+__device__ void reduce_segment_smem(const float* sp, int np, int seg,
+                                    uint8_t* __restrict__ images, float* __restrict__ stS,
+                                    float* __restrict__ stz, int use_state, int commit, int tid,
+                                    int nthr) {
+  constexpr int DD = D * D, DD1 = D * (D + 1), QPR = D / 4, ITEMS = (D + 1) * QPR;
+  uint8_t* img = images + (long long)seg * image_bytes(D);
+  for (int item = tid; item < ITEMS; item += nthr) {
+    const int n = item / QPR;
+    const int a0 = 4 * (item - n * QPR);
+    const bool zrow = n == D;
+    const int off = n * D + a0;
+    float4 acc = *reinterpret_cast<const float4*>(sp + off);
+    for (int i = 1; i < np; ++i)
+      acc = add4(acc, *reinterpret_cast<const float4*>(sp + (long long)i * DD1 + off));
+    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (use_state) {
+      float r[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        r[e] = zrow ? stz[(long long)seg * D + a0 + e] : stS[(long long)seg * DD + (a0 + e) * D + n];
+      run = make_float4(r[0], r[1], r[2], r[3]);
+    }
+    run = add4(run, acc);
+    store_image4<D>(img + image_offset<D>(n, a0), zrow, a0, run);
+    if (use_state && commit) {
+      const float r[4] = {run.x, run.y, run.z, run.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (zrow) stz[(long long)seg * D + a0 + e] = r[e];
+        else stS[(long long)seg * DD + (a0 + e) * D + n] = r[e];
+      }
+    }
+  }
+}
+
 // ---- state build ------------------------------------------------------------------
 
 // warp 0 TMA, warp 1 MMA, warps 2-17 math, warps 18-21 epilogue (one per TMEM
 // lane quadrant)
 constexpr int kTcThreadsState = 64 + kMath + 128;
+constexpr int kTailSegs = 32;   // segments a CTA can leave to its tail
 
 template <int D, bool ROPE>
 __global__ void __launch_bounds__(kTcThreadsState, 1)
@@ -521,10 +560,12 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   auto zrdy_bar = [&](int b) { return bar0 + 8u * (3 * stages + 4 + b); };
   auto zfree_bar = [&](int b) { return bar0 + 8u * (3 * stages + 6 + b); };
   const uint32_t done_bar = bar0 + 8u * (3 * stages + 8);
+  const uint32_t tail_bar = bar0 + 8u * (3 * stages + 9);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P.off_tmem);
   __shared__ int s_abort;
-  __shared__ int s_red;    // segment the epilogue warps reduce next, or -1
-  __shared__ int s_tail;   // segment all warps reduce after the tile loop, or -1
+  __shared__ int s_red;    // segment the epilogue warps reduce at once, or -1
+  __shared__ int s_npend;  // segments all warps reduce after the tile loop
+  __shared__ int s_pend[kTailSegs];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int cta = blockIdx.x;
@@ -532,7 +573,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    s_tail = -1;
+    s_npend = 0;
     for (int s = 0; s < stages; ++s) {
       ptx::mbar_init(full_bar(s), 1);
       ptx::mbar_init(kready_bar(s), kMath);
@@ -545,6 +586,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       ptx::mbar_init(zfree_bar(b), 128);
     }
     ptx::mbar_init(done_bar, 1);
+    ptx::mbar_init(tail_bar, 1);
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
@@ -740,7 +782,8 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       if (counters) {
         // one segment per head: the CTA that completes a segment last turns
         // its partials into the image (all epilogue warps' slot writes are
-        // fenced before the arrival is counted)
+        // fenced before the arrival is counted) -- after its tile loop with
+        // all warps, or here when its list of pending segments is full
         __threadfence();
         const bool all_ready = ptx::bar_all(2, 128, ready);
         if (te == 0) {
@@ -752,8 +795,8 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
               red = it.seg;
             }
           }
-          if (red >= 0 && u + 1 == u1) {
-            s_tail = red;             // the CTA's last tile: reduce with all warps
+          if (red >= 0 && s_npend < kTailSegs) {
+            s_pend[s_npend++] = red;  // reduce with all warps after the tile loop
             red = -1;
           }
           s_red = red;
@@ -773,10 +816,37 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     ptx::tc_fence_after();
     ptx::tmem_dealloc(*s_tmem, TMEM_COLS);
   }
-  if (s_tail >= 0 && !s_abort) {
+  if (s_npend > 0 && !s_abort) {
+    // At D = 128 (six partial rows per thread) the drained stage ring takes
+    // up to `cap` partial slots: bulk-copy a segment's partials there at once
+    // and reduce them from shared memory. At D = 64 the register path, with
+    // fewer rows per thread, is as fast.
+    constexpr uint32_t SLOT = DD1 * 4;
+    const int cap = D == 128 ? (int)(P.off_bar / SLOT) : 0;
     __threadfence();
-    reduce_segment<D>(partials, sc, s_tail, images, stS, stz, use_state, commit, threadIdx.x,
-                      kTcThreadsState);
+    uint32_t tph = 0;
+    for (int k = 0; k < s_npend; ++k) {
+      const int seg = s_pend[k];
+      const int np = parts_of(sc, seg);
+      if (np > cap) {
+        reduce_segment<D>(partials, sc, seg, images, stS, stz, use_state, commit, threadIdx.x,
+                          kTcThreadsState);
+        continue;
+      }
+      if (threadIdx.x == 0) {
+        ptx::fence_proxy_async_global();
+        ptx::mbar_expect_tx(tail_bar, (uint32_t)np * SLOT);
+        for (int i = 0; i < np; ++i)
+          ptx::bulk_load(base + (uint32_t)i * SLOT,
+                         partials + ((long long)seg * sc.maxc + i) * DD1, SLOT, tail_bar);
+      }
+      const bool got = wait_bounded(tail_bar, tph, flag, kFlagStateTimeout, &s_abort);
+      if (!__syncthreads_and(got)) break;   // every thread leaves together
+      tph ^= 1u;
+      reduce_segment_smem<D>(reinterpret_cast<const float*>(sm), np, seg, images, stS, stz,
+                             use_state, commit, threadIdx.x, kTcThreadsState);
+      __syncthreads();   // before the next segment's copies overwrite the slots
+    }
   }
 }
 
