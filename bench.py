@@ -389,9 +389,10 @@ def oracle_sample(w, budget_s: float, max_heads=None):
     cores = oracle.threads(0)
     heads = min(w.B * w.H, max_heads or w.B * w.H)
     T, Hg, Wg = w.grid
-    # about 0.5 us of CPU per token-head at D = 64 (scaled by D^2): size frames to the budget
+    # about 10 us of one core per token-head at D = 64 (scaled by D^2), as measured on
+    # the hosts: size frames to the budget
     frames = T
-    est = lambda f: heads * f * Hg * Wg * (w.D * w.D / 4096.0) * 0.5e-6 / min(cores, heads)
+    est = lambda f: heads * f * Hg * Wg * (w.D * w.D / 4096.0) * 10e-6 / min(cores, heads)
     while frames > 1 and est(frames) > budget_s:
         frames -= 1
     sw = workloads.Workload(name=w.name + "_sample", B=1, H=heads, N=frames * Hg * Wg, D=w.D,

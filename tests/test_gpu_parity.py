@@ -61,6 +61,21 @@ def edge_cases():
             rope_split=(20, 22, 22)), "bidirectional"),
         # no RoPE in bf16
         (mk("no_rope_bf16", B=1, H=2, N=300, D=64, dtype="bf16", seed=20), "bidirectional"),
+        # D = 128 without a gate (output stored from registers), several tiles and a
+        # ragged tail, bidirectional and in blocks that split tiles
+        (mk("d128_ragged_tiles", B=1, H=3, N=3 * 7 * 13, D=128, dtype="bf16", seed=21,
+            grid=(3, 7, 13), rope_split=(32, 48, 48)), "bidirectional"),
+        (mk("d128_blocks", B=1, H=3, N=3 * 7 * 13, D=128, dtype="bf16", seed=22,
+            grid=(3, 7, 13), rope_split=(32, 48, 48), gate=True, modes=("block_causal",),
+            block_tokens=91), "block_causal"),
+        # thousands of one-tile heads: a CTA completes more heads than it can
+        # leave to its tail and reduces the rest on the spot
+        (mk("many_small_heads", B=64, H=128, N=16, D=64, dtype="bf16", seed=23,
+            grid=(1, 4, 4), rope_split=(16, 24, 24)), "bidirectional"),
+        # more heads than the workspace has arrival counters: the separate
+        # reduction kernel takes over
+        (mk("counter_overflow", B=136, H=128, N=8, D=64, dtype="bf16", seed=24,
+            grid=(1, 2, 4), rope_split=(16, 24, 24)), "bidirectional"),
     ]
 
 
@@ -125,6 +140,26 @@ def test_one_block_equals_bidirectional():
 
 def _block_view(x, b, bt):
     return x[:, :, b * bt:(b + 1) * bt].contiguous()
+
+
+def test_block_steps_d128_gated_match_oracle():
+    # the carried state at D = 128 with the gate: two blocks, committed in turn
+    w = workloads.Workload("d128_steps", B=1, H=2, N=4 * 6 * 8, D=128, dtype="bf16",
+                           seed=25, grid=(4, 6, 8), rope_split=(32, 48, 48), gate=True,
+                           modes=("block_causal",), block_tokens=2 * 6 * 8)
+    x = workloads.make_inputs(w)
+    t = upload(w, x)
+    bt = w.block_tokens
+    st = la.BlockState(w.B, w.H, w.D)
+    outs = [st.step(_block_view(t["q"], b, bt), _block_view(t["k"], b, bt),
+                    _block_view(t["v"], b, bt), _block_view(t["g"], b, bt), t_offset=2 * b,
+                    commit=True, grid=(2, 6, 8), rope_split=w.rope_split, eps=w.eps)
+            for b in range(2)]
+    seq = torch.cat(outs, dim=2)
+    torch.cuda.synchronize()
+    ref = oracle.forward(oracle.params_for(w, "block_causal"), x["q"], x["k"], x["v"],
+                         g=x["g"])
+    assert_parity(to64(seq), ref, w.dtype, "d128 block steps")
 
 
 def test_block_steps_match_forward_and_oracle():
