@@ -1150,8 +1150,8 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                            IDESC_Z, kk == 0 ? 0u : 1u);
         }
         ptx::mma_commit(accf_bar(b));
-        // (direct output) the q stage and, after a segment's last tile, the
-        // image slot are free once these MMAs have read them
+        // once these MMAs have read them, the q stage (with direct output) and,
+        // after a segment's last tile, the image slot are free
         if (DIRECT) ptx::mma_commit(empty_bar(it.stage));
         if (it.last_of_segment(u, u1)) ptx::mma_commit(sempty_bar(ss % sbuf));
         if (++b == 2) {
