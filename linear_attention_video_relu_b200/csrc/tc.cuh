@@ -595,9 +595,14 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   }
   __syncthreads();
   if (threadIdx.x == 0) ptx::launch_dependents();
+  // Launched early (programmatic dependent launch) behind the previous
+  // kernel of the stream: k and v are read, and the workspace is written,
+  // only after griddepcontrol.wait (by the TMA warp before its loads, by the
+  // math warps before the table goes out; everything else follows the loads).
 
   if (warp == 0) {
     // ---------------- TMA producer (+ row offsets of the RoPE table) ----------------
+    ptx::grid_dependency_wait();
     TileIter it;
     it.init(u0, sc.tps, stages);
     long long issued = 0;
@@ -673,6 +678,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     const int half = c >> 3, cc = c & 7;
     if (ROPE) {
       build_rope_table(rope, s_tab, tt);
+      ptx::grid_dependency_wait();
       const int e0 = (int)((long long)cta * rope.entries / gridDim.x);
       const int e1 = (int)((long long)(cta + 1) * rope.entries / gridDim.x);
       for (int e = e0 + tt; e < e1; e += kMath) gtab[e] = s_tab[e];
@@ -1048,6 +1054,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     ptx::tmem_relinquish();
   }
   __syncthreads();
+  if (threadIdx.x == 0) ptx::launch_dependents();
   // launched early (programmatic dependent launch): the images and the RoPE
   // table are read only after the kernels that write them have completed
   ptx::grid_dependency_wait();
@@ -1438,10 +1445,10 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   if ((st = tc_smem_attr(k1, p1.total)) != LA_OK) return st;
   if ((st = tc_mark(a, 0)) != LA_OK) return st;
   uint8_t* images = reinterpret_cast<uint8_t*>(a.apply);
-  k1<<<sc.G, kTcThreadsState, p1.total, a.stream>>>(mk, mv, a.rope, sc, s1, a.part, a.gtab,
-                                                    a.flag, a.fused ? a.counters : nullptr,
-                                                    images, a.stS, a.stz, a.use_state, a.commit);
-  if ((st = tc_check_launch()) != LA_OK) return st;
+  st = launch_pdl(k1, dim3(sc.G), dim3(kTcThreadsState), p1.total, a.stream, mk, mv, a.rope,
+                  sc, s1, a.part, a.gtab, a.flag, a.fused ? a.counters : nullptr, images,
+                  a.stS, a.stz, a.use_state, a.commit);
+  if (st != LA_OK) return st;
   if ((st = tc_mark(a, 1)) != LA_OK) return st;
   if (!a.fused) {
     // the reduction and the apply kernel are launched programmatically
