@@ -47,7 +47,8 @@ def parse_args():
     ap.add_argument("--workload", default=MAIN, choices=sorted(workloads.WORKLOADS),
                     help="workload of the timed line (another one than the default is for "
                          "profiling runs)")
-    ap.add_argument("--mode", default="bidirectional", choices=["bidirectional", "block_causal"])
+    ap.add_argument("--mode", default="bidirectional",
+                    choices=["bidirectional", "block_causal", "token_causal"])
     ap.add_argument("--settle", type=int, default=50,
                     help="untimed forwards before the timed region (clock settling)")
     return ap.parse_args()
@@ -56,6 +57,8 @@ def parse_args():
 def launches_per_forward(w, mode) -> int:
     """Kernels one forward launches: state build (+ reduction when a head has
     more than one segment) + apply."""
+    if mode == "token_causal":
+        return 3   # CUDA-core kernels: state partials, scan, chunked apply
     one_segment = mode == "bidirectional" or w.block_tokens in (0, w.N)
     return 2 if one_segment else 3
 
@@ -540,7 +543,8 @@ def main():
         extra = []
         K = max(20, args.steps // 5)
         for name, mode in (("480p_block_causal", "block_causal"), ("720p_long", "bidirectional"),
-                           ("720p_long", "block_causal"), ("gated_d128", "bidirectional")):
+                           ("720p_long", "block_causal"), ("gated_d128", "bidirectional"),
+                           ("480p_bidir", "token_causal")):
             ww = workloads.WORKLOADS[name]
             extra.append(measure_workload(ww, mode, K, 3, None, device, peak, peak_kind,
                                           ww.seed))

@@ -74,16 +74,16 @@ typedef enum {
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;   /* I/O dtype; state is fp32 */
 
-typedef enum { LA_BIDIRECTIONAL = 0, LA_BLOCK_CAUSAL = 1 } la_mode;
+typedef enum { LA_BIDIRECTIONAL = 0, LA_BLOCK_CAUSAL = 1, LA_TOKEN_CAUSAL = 2 } la_mode;
 
 typedef struct {
   int B, H, N, D;        /* batch, heads, tokens per head, head dim.
                             D in {32, 64, 128}; N >= 0 (N = 0: no work). */
   la_dtype dtype;        /* dtype of q, k, v, gate and out */
-  la_mode mode;          /* bidirectional or block-causal */
+  la_mode mode;          /* bidirectional, block-causal or token-causal */
   int block_tokens;      /* block-causal: tokens per block, N % block_tokens == 0.
                             A token of block b sees blocks 0..b (its own block
-                            whole). Ignored in bidirectional mode. */
+                            whole). Ignored in the other modes. */
   int rope;              /* 0: no rotation (then the grid fields are ignored) */
   int grid_t, grid_h, grid_w;     /* latent grid; N == grid_t*grid_h*grid_w */
   int rope_dt, rope_dh, rope_dw;  /* even widths with sum D (t, h, w order) */
@@ -116,6 +116,11 @@ LA_API la_status lin_attn_block_step_workspace_size(const la_params* p, size_t* 
  *   bidirectional: out_i uses S, z summed over all N tokens of its head.
  *   block-causal:  out_i of block b uses S, z summed over blocks 0..b, which
  *                  is Algorithm 1 run with an empty initial cache.
+ *   token-causal:  out_i uses S, z summed over tokens 0..i of its head (the
+ *                  causal form, Eq. 3 of "Block Linear Attention with
+ *                  Constant-Memory KV Cache"). Runs on the CUDA-core
+ *                  kernels: chunks of 32 tokens, the running sums over
+ *                  earlier chunks plus the masked sums inside the chunk.
  * q, k, v, out: [B,H,N,D] device pointers in p->dtype. gate: NULL or the same
  * shape and dtype (logits; out is multiplied by their sigmoid).
  * workspace: device memory of at least lin_attn_workspace_size bytes, 256-byte
@@ -208,7 +213,8 @@ LA_API const char* lin_attn_status_string(la_status s);
 
 /* Which kernel family lin_attn_forward would use for `p` on the current
  * device: 1 = tensor-core (tcgen05 + TMA, bf16 I/O, D in {64, 128}),
- * 0 = CUDA-core (fp32 I/O, or shapes outside the tensor-core path). */
+ * 0 = CUDA-core (fp32 I/O, token-causal mode, or shapes outside the
+ * tensor-core path). */
 LA_API int lin_attn_uses_tensor_cores(const la_params* p);
 
 #ifdef __cplusplus

@@ -25,6 +25,7 @@ LA_F32 = 0
 LA_BF16 = 1
 LA_BIDIRECTIONAL = 0
 LA_BLOCK_CAUSAL = 1
+LA_TOKEN_CAUSAL = 2
 
 
 class la_params(ctypes.Structure):

@@ -14,7 +14,8 @@ import torch
 from . import _native as C
 
 _DTYPES = {torch.bfloat16: C.LA_BF16, torch.float32: C.LA_F32}
-_MODES = {"bidirectional": C.LA_BIDIRECTIONAL, "block_causal": C.LA_BLOCK_CAUSAL}
+_MODES = {"bidirectional": C.LA_BIDIRECTIONAL, "block_causal": C.LA_BLOCK_CAUSAL,
+          "token_causal": C.LA_TOKEN_CAUSAL}
 
 
 def make_params(B: int, H: int, N: int, D: int, dtype: torch.dtype, mode: str = "bidirectional",

@@ -34,6 +34,7 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
   bool tc;             // tensor-core kernels
+  bool causal;         // token-causal mode (CUDA-core kernels, chunked)
   Rope rope;
   Sched sc;
   long long heads;
@@ -67,7 +68,8 @@ la_status check_params(const la_params* p, bool one_block) {
   if (p->D != 32 && p->D != 64 && p->D != 128) return LA_ERR_INVALID_ARG;
   if (p->dtype != LA_F32 && p->dtype != LA_BF16) return LA_ERR_INVALID_ARG;
   if (!one_block) {
-    if (p->mode != LA_BIDIRECTIONAL && p->mode != LA_BLOCK_CAUSAL) return LA_ERR_INVALID_ARG;
+    if (p->mode != LA_BIDIRECTIONAL && p->mode != LA_BLOCK_CAUSAL && p->mode != LA_TOKEN_CAUSAL)
+      return LA_ERR_INVALID_ARG;
     if (p->mode == LA_BLOCK_CAUSAL &&
         (p->block_tokens < 1 || (p->N > 0 && p->N % p->block_tokens != 0)))
       return LA_ERR_INVALID_ARG;
@@ -90,7 +92,8 @@ la_status check_params(const la_params* p, bool one_block) {
   return LA_OK;
 }
 
-bool want_tc(const la_params* p) {
+bool want_tc(const la_params* p, bool one_block) {
+  if (!one_block && p->mode == LA_TOKEN_CAUSAL) return false;   // CUDA-core kernels only
   const int entries = p->rope ? p->grid_t * rope_stride(p->rope_dt / 2) +
                                     p->grid_h * rope_stride(p->rope_dh / 2) +
                                     p->grid_w * rope_stride(p->rope_dw / 2)
@@ -108,7 +111,7 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   st = device_sms(&sms);
   if (st != LA_OK) return st;
   memset(pl, 0, sizeof(*pl));
-  pl->tc = want_tc(p);
+  pl->tc = want_tc(p, one_block);
   pl->sms = sms;
   pl->heads = (long long)p->B * p->H;
 
@@ -146,9 +149,12 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
 
   Sched& sc = pl->sc;
   const int N = p->N;
-  sc.L = (!one_block && p->mode == LA_BLOCK_CAUSAL) ? p->block_tokens : N;
+  // token-causal: chunks of kCausalChunk tokens (the last one ragged)
+  pl->causal = !one_block && p->mode == LA_TOKEN_CAUSAL;
+  sc.L = pl->causal ? kCausalChunk
+                    : ((!one_block && p->mode == LA_BLOCK_CAUSAL) ? p->block_tokens : N);
   if (sc.L < 1) sc.L = 1;
-  sc.nblk = N / sc.L;
+  sc.nblk = (N + sc.L - 1) / sc.L;
   if (sc.nblk < 1) sc.nblk = 1;
   sc.nseg = (int)(pl->heads * sc.nblk);
   sc.TT = pl->tc ? tc_state_tile(p->D) : kSimtTileState;
@@ -253,6 +259,19 @@ la_status run_simt(const Launch& L) {
   if ((st = last_error()) != LA_OK) return st;
   if ((st = mark(L, 2)) != LA_OK) return st;
   if (!L.do_apply) return LA_OK;
+  if (pl.causal) {
+    const int C = kCausalChunk;
+    size_t smemc = ((size_t)D * (D + 1) + 5 * (size_t)C * D + 2 * (size_t)C * C + C) *
+                   sizeof(float);
+    if ((st = set_smem(apply_causal_simt<D, T>, smemc)) != LA_OK) return st;
+    const int gc = pl.sc.nseg < (1 << 20) ? pl.sc.nseg : (1 << 20);
+    apply_causal_simt<D, T><<<gc, kSimtThreads, smemc, L.stream>>>(
+        static_cast<const T*>(L.q), static_cast<const T*>(L.k), static_cast<const T*>(L.v),
+        static_cast<const T*>(L.g), static_cast<T*>(L.out), N, pl.rope, pl.sc.nblk,
+        pl.sc.nseg, apply, gtab, L.p->eps);
+    if ((st = last_error()) != LA_OK) return st;
+    return mark(L, 3);
+  }
   const int TA = kSimtTileApply;
   size_t smem3 = ((size_t)D * (D + 1) + 2 * (size_t)TA * D + TA) * sizeof(float);
   st = set_smem(apply_simt<D, T>, smem3);
@@ -530,7 +549,7 @@ const char* lin_attn_status_string(la_status s) {
 
 int lin_attn_uses_tensor_cores(const la_params* p) {
   if (check_params(p, false) != LA_OK) return 0;
-  return want_tc(p) ? 1 : 0;
+  return want_tc(p, false) ? 1 : 0;
 }
 
 }  // extern "C"

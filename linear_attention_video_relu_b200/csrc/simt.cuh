@@ -15,6 +15,10 @@ namespace la {
 constexpr int kSimtThreads = 256;
 constexpr int kSimtTileState = 32;   // tokens per tile of the state build
 constexpr int kSimtTileApply = 32;   // tokens per tile of the apply step
+// Token-causal mode: segments (chunks) of this many tokens, one tile each.
+constexpr int kCausalChunk = 32;
+static_assert(kCausalChunk == kSimtTileState && kCausalChunk == kSimtTileApply,
+              "a causal chunk is one tile of each kernel");
 
 // Position (local frame, row, column) of token n of a head.
 __device__ inline void token_pos(const Rope& r, long long n, int& tl, int& h, int& w) {
@@ -91,7 +95,9 @@ state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N
     }
     const int head = seg / sc.nblk, blk = seg - head * sc.nblk;
     const int r0 = tile * TT;
-    const int rows = min(TT, sc.L - r0);
+    // segments hold L tokens, except a ragged last chunk in token-causal mode
+    const int seglen = (int)min((long long)sc.L, N - (long long)blk * sc.L);
+    const int rows = min(TT, seglen - r0);
     const long long nbase = (long long)blk * sc.L + r0;
     const T* kh = k + ((long long)head * N + nbase) * D;
     const T* vh = v + ((long long)head * N + nbase) * D;
@@ -241,6 +247,120 @@ apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out
     out[ebase + idx] = from_f32<T>(o);
   }
   __syncthreads();
+  }
+}
+
+// Token-causal apply (Eq. 3 of "Block Linear Attention with Constant-Memory KV
+// Cache"): one CTA per chunk of kCausalChunk tokens. With S_<c, z_<c the sums
+// over earlier chunks of the head (the inclusive state of the previous chunk,
+// written by reduce_states) and P_ij = RoPE(phi q_i) . RoPE(phi k_j),
+// Q_ij = phi q_i . phi k_j inside the chunk,
+//   out_i = (RoPE(phi q_i) S_<c + sum_{j <= i} P_ij v_j)
+//           / (phi q_i . z_<c + sum_{j <= i} Q_ij + eps)   (times sigmoid(g_i)).
+template <int D, typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+apply_causal_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                  const T* __restrict__ g, T* __restrict__ out, long long N, Rope rope, int nblk,
+                  int nseg, const float* __restrict__ apply, const float2* __restrict__ gtab,
+                  float eps) {
+  constexpr int C = kCausalChunk;
+  constexpr int DD1 = D * (D + 1);
+  static_assert(C == 32, "the denominator adds one masked weight per lane");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* s_S = reinterpret_cast<float*>(smem_raw);  // [D][D], then z [D]
+  float* s_z = s_S + D * D;
+  float* s_qphi = s_z + D;                           // [C][D]
+  float* s_qr = s_qphi + C * D;
+  float* s_kphi = s_qr + C * D;
+  float* s_kr = s_kphi + C * D;
+  float* s_v = s_kr + C * D;
+  float* s_P = s_v + C * D;                          // [C][C] numerator weights
+  float* s_Q = s_P + C * C;                          // [C][C] denominator weights
+  float* s_den = s_Q + C * C;                        // [C]
+  const int tid = threadIdx.x;
+  for (int seg = blockIdx.x; seg < nseg; seg += gridDim.x) {
+    const int head = seg / nblk, blk = seg - head * nblk;
+    const long long nbase = (long long)blk * C;
+    const int rows = (int)min((long long)C, N - nbase);
+    const long long ebase = ((long long)head * N + nbase) * D;
+    // the state of the chunks before this one (zero for the first)
+    if (blk > 0) {
+      const float4* src = reinterpret_cast<const float4*>(apply + (long long)(seg - 1) * DD1);
+      for (int i = tid; i < DD1 / 4; i += kSimtThreads) reinterpret_cast<float4*>(s_S)[i] = src[i];
+    } else {
+      for (int i = tid; i < DD1; i += kSimtThreads) s_S[i] = 0.f;
+    }
+    for (int idx = tid; idx < C * (D / 2); idx += kSimtThreads) {
+      const int r = idx / (D / 2), pr = idx - r * (D / 2);
+      float qx = 0.f, qy = 0.f, kx = 0.f, ky = 0.f, v0 = 0.f, v1 = 0.f;
+      if (r < rows) {
+        const long long e = ebase + r * D + 2 * pr;
+        qx = relu(to_f32(q[e]));
+        qy = relu(to_f32(q[e + 1]));
+        kx = relu(to_f32(k[e]));
+        ky = relu(to_f32(k[e + 1]));
+        v0 = to_f32(v[e]);
+        v1 = to_f32(v[e + 1]);
+      }
+      float qrx = qx, qry = qy, krx = kx, kry = ky;
+      if (rope.on && r < rows) {
+        int tl, h, w;
+        token_pos(rope, nbase + r, tl, h, w);
+        const float2 cs = rope_cs(rope, reinterpret_cast<const float*>(gtab), pr, tl, h, w);
+        qrx = qx * cs.x - qy * cs.y;
+        qry = qx * cs.y + qy * cs.x;
+        krx = kx * cs.x - ky * cs.y;
+        kry = kx * cs.y + ky * cs.x;
+      }
+      const int o = r * D + 2 * pr;
+      s_qphi[o] = qx;
+      s_qphi[o + 1] = qy;
+      s_qr[o] = qrx;
+      s_qr[o + 1] = qry;
+      s_kphi[o] = kx;
+      s_kphi[o + 1] = ky;
+      s_kr[o] = krx;
+      s_kr[o + 1] = kry;
+      s_v[o] = v0;
+      s_v[o + 1] = v1;
+    }
+    __syncthreads();
+    // masked weights inside the chunk (j <= i)
+    for (int idx = tid; idx < C * C; idx += kSimtThreads) {
+      const int i = idx / C, j = idx - i * C;
+      float p = 0.f, qq = 0.f;
+      if (j <= i) {
+        for (int a = 0; a < D; ++a) {
+          p = fmaf(s_qr[i * D + a], s_kr[j * D + a], p);
+          qq = fmaf(s_qphi[i * D + a], s_kphi[j * D + a], qq);
+        }
+      }
+      s_P[idx] = p;
+      s_Q[idx] = qq;
+    }
+    __syncthreads();
+    const int warp = tid / 32, lane = tid % 32;
+    for (int r = warp; r < C; r += kSimtThreads / 32) {
+      float d = 0.f;
+      for (int a = lane; a < D; a += 32) d = fmaf(s_qphi[r * D + a], s_z[a], d);
+      d += s_Q[r * C + lane];   // C == 32: one masked weight per lane
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      if (lane == 0) s_den[r] = d + eps;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * D; idx += kSimtThreads) {
+      const int r = idx / D, c = idx - r * D;
+      if (r >= rows) continue;
+      float num = 0.f;
+#pragma unroll 8
+      for (int a = 0; a < D; ++a) num = fmaf(s_qr[r * D + a], s_S[a * D + c], num);
+      for (int j = 0; j <= r; ++j) num = fmaf(s_P[r * C + j], s_v[j * D + c], num);
+      float o = num / s_den[r];
+      if (g) o *= sigmoid(to_f32(g[ebase + idx]));
+      out[ebase + idx] = from_f32<T>(o);
+    }
+    __syncthreads();
   }
 }
 

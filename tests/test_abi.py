@@ -137,6 +137,18 @@ def test_tensor_core_path_selection_is_host_logic():
     assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=20, rope_dh=22, rope_dw=22)) == 0
     assert C.lin_attn_uses_tensor_cores(_params(D=128, rope_dt=32, rope_dh=48, rope_dw=48)) == 1
     assert C.lin_attn_uses_tensor_cores(_params(D=64, rope=0)) == 1
+    # token-causal runs on the CUDA-core kernels
+    assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=16, rope_dh=24, rope_dw=24,
+                                                mode=C.LA_TOKEN_CAUSAL)) == 0
+
+
+def test_token_causal_mode_is_accepted_and_ignores_block_tokens():
+    # passes the host checks (the fake pointers then fail only at the device
+    # query, never as an argument error), for any block_tokens
+    for bt in (0, 7):
+        rc = C.lin_attn_forward(_params(mode=C.LA_TOKEN_CAUSAL, block_tokens=bt), Q, K, V, None,
+                                O, WS, 1 << 20, None)
+        assert rc != C.LA_ERR_INVALID_ARG
 
 
 def test_control_block_size_matches_the_header():

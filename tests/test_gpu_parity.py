@@ -79,6 +79,23 @@ def edge_cases():
     ]
 
 
+def token_causal_cases():
+    """Per-token causal attention (Eq. 3): chunks of 32 tokens, ragged tails."""
+    mk = workloads.Workload
+    return [
+        mk("tc_one_token", B=1, H=2, N=1, D=64, dtype="bf16", seed=31, grid=(1, 1, 1),
+           rope_split=(16, 24, 24), modes=("token_causal",)),
+        mk("tc_ragged_105", B=2, H=2, N=3 * 5 * 7, D=64, dtype="bf16", seed=32, grid=(3, 5, 7),
+           rope_split=(16, 24, 24), modes=("token_causal",)),
+        mk("tc_f32_gate", B=1, H=3, N=100, D=32, dtype="f32", seed=33, gate=True,
+           modes=("token_causal",)),
+        mk("tc_d128_gate", B=1, H=2, N=2 * 4 * 6, D=128, dtype="bf16", seed=34, grid=(2, 4, 6),
+           rope_split=(32, 48, 48), gate=True, modes=("token_causal",)),
+        dataclasses.replace(W["480p_bidir"].scaled(1), name="tc_480p_1frame",
+                            modes=("token_causal",)),
+    ]
+
+
 def _check_against_oracle(w, mode):
     x = workloads.make_inputs(w)
     t = upload(w, x)
@@ -95,6 +112,11 @@ def test_small_workloads_match_oracle(w, mode):
 @pytest.mark.parametrize("w,mode", edge_cases(), ids=lambda c: getattr(c, "name", c))
 def test_edge_cases_match_oracle(w, mode):
     _check_against_oracle(w, mode)
+
+
+@pytest.mark.parametrize("w", token_causal_cases(), ids=lambda c: c.name)
+def test_token_causal_matches_oracle(w):
+    _check_against_oracle(w, "token_causal")
 
 
 FULL = [("480p_bidir", "bidirectional"), ("480p_block_causal", "block_causal"),
