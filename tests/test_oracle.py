@@ -320,6 +320,22 @@ def test_causality_future_tokens_do_not_change_the_past(mode):
     assert not np.array_equal(out[:, :, cut:], base[:, :, cut:])
 
 
+def test_token_causal_equals_blocks_of_one_token():
+    # blocks of one token see exactly the tokens 0..i: the block-causal form
+    # with block_tokens = 1 and the per-token causal form are the same sums
+    B, H, N, D = 1, 2, 60, 32
+    q, k, v = _qkv(B, H, N, D, 85)
+    g = _rand(q.shape, 86)
+    kw = dict(grid=(3, 4, 5), rope_split=(8, 12, 12))
+    a = oracle.forward(oracle.make_params(B, H, N, D, mode="token_causal", **kw), q, k, v, g=g)
+    b = oracle.forward(oracle.make_params(B, H, N, D, mode="block_causal", block_tokens=1, **kw),
+                       q, k, v, g=g)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+    # and the last token sees the whole head: the bidirectional output there
+    c = oracle.forward(oracle.make_params(B, H, N, D, **kw), q, k, v, g=g)
+    np.testing.assert_allclose(a[:, :, -1], c[:, :, -1], rtol=1e-12, atol=1e-14)
+
+
 def test_rows_match_full_output():
     B, H, N, D = 2, 2, 60, 32
     q, k, v = _qkv(B, H, N, D, 90)
