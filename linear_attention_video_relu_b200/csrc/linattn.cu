@@ -1,14 +1,18 @@
 // linattn.cu -- host side of the C ABI declared in include/linattn.h:
 // argument checks, the work plan, the workspace carve-up and the launches.
 //
-// One forward is three launches on the caller's stream:
+// A forward follows the factorised form of Eq. 2 and the block recursion of
+// Eq. 3 / Algorithm 1 (SANA-Video paper-graph page, section 3.4) in up to
+// three launches on the caller's stream:
 //   1. state build  (per contiguous tile range: partial S, z of every segment
 //                    the range touches; also the RoPE cos/sin table)
 //   2. reduce       (fixed-order sum of the partials per segment, then the
-//                    block-causal running sum, or the carried state)
+//                    block-causal running sum, or the carried state) -- on
+//                    the tensor-core path folded into the state build when
+//                    every head is one segment
 //   3. apply        (out = RoPE(phi q) S / (phi q . z + eps), gate)
-// following the factorised form of Eq. 2 and the block recursion of Eq. 3 /
-// Algorithm 1 (SANA-Video paper-graph page, section 3.4).
+// The token-causal mode runs on the CUDA-core kernels with 32-token chunks
+// as segments and a chunked apply step.
 #include "linattn.h"
 
 #include <math.h>

@@ -1,11 +1,13 @@
-// simt.cuh -- CUDA-core kernels: the fp32 I/O path and every shape the
-// tensor-core path does not take (D = 32, rope widths not multiples of 8).
+// simt.cuh -- CUDA-core kernels: the fp32 I/O path, the token-causal mode
+// and every shape the tensor-core path does not take (D = 32, rope widths
+// not multiples of 8).
 //
 // Three launches per call, each a step of the factorised form of Eq. 2
 // (SANA-Video paper-graph page, section 3.4):
 //   state_partial_simt  per tile range: S_part = sum RoPE(phi k)^T v, z_part = sum phi k
 //   reduce_states       fixed-order sum of the partials (+ carried state, + block scan)
 //   apply_simt          out = RoPE(phi q) S / (phi q . z + eps), times sigmoid(g)
+//   (apply_causal_simt in token-causal mode)
 #pragma once
 
 #include "common.cuh"

@@ -2,18 +2,21 @@
 // for bf16 I/O with D in {64, 128}.
 //
 // state_build_tc: per CTA a contiguous range of token tiles. TMA brings the k
-//   and v tiles (128-byte swizzle) into a ring of stages; four warps apply
+//   and v tiles (128-byte swizzle) into a ring of stages; 16 math warps apply
 //   phi = ReLU and the 3D RoPE to the k tile in place and sum phi(k) for z;
 //   one thread issues tcgen05.mma with A = RoPE(phi k)^T (MN-major) and
 //   B = v (MN-major) into an fp32 TMEM accumulator, one per segment (double
-//   buffered); the four warps copy the finished accumulator and z to the
-//   CTA's partial slot. Eq. 2's numerator state and denominator sum.
+//   buffered); 4 epilogue warps copy the finished accumulator and z to the
+//   CTA's partial slot. When every head is one segment, the CTA that
+//   completes a segment last also sums its partials into the apply image.
+// finalize_images: the same reduction for heads of several blocks, with the
+//   running sum over blocks.
 // apply_tc: per CTA a contiguous range of 128-token tiles. TMA brings q (and
-//   the gate logits); four warps form phi(q) . z + eps and RoPE(phi q) in
-//   place; one thread issues A = RoPE(phi q) (K-major) x B = S (K-major, as
-//   bf16 hi + lo so S keeps ~16 bits) into TMEM; the same warps divide by the
-//   denominator, apply the gate, round to bf16 and TMA-store the tile (rows
-//   past the segment are clipped by the tensor map).
+//   the gate logits); 16 math warps write RoPE(phi q) in place and phi(q)
+//   into TMEM; one thread issues A = RoPE(phi q) x B = S (K-major, as bf16
+//   hi + lo so S keeps ~16 bits) and phi(q) x [z_hi z_lo] into TMEM; the math
+//   warps divide by the denominator, apply the gate, round to bf16 and send
+//   the tile out (see the apply section for the two output paths).
 //
 // (SANA-Video paper-graph page, section 3.4: the unnumbered ReLU linear
 // attention equation and Eq. 2.) No wait here is unbounded: every mbarrier
