@@ -18,6 +18,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import math
 import os
 import statistics
@@ -110,12 +111,18 @@ def measured_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the CUDA sources with comments and whitespace removed, so that a
+    committed traffic figure stays tied to the code, not to its comments."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_video_relu_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name)) as f:
+                text = f.read()
+            text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+            text = re.sub(r"//[^\n]*", " ", text)
+            text = " ".join(text.split())
+            h.update(name.encode() + b"\0" + text.encode())
     return h.hexdigest()[:12]
 
 

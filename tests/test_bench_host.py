@@ -103,6 +103,12 @@ def test_profile_traffic_lookup_is_tied_to_the_sources(tmp_path, monkeypatch):
     assert bench.ncu_traffic("apply", "480p_bidir") == 123
     assert bench.ncu_traffic("apply", "720p_long") == 9
     assert bench.ncu_traffic("state_build", "480p_bidir") is None
+    # comments do not count; code does
+    (csrc / "k.cu").write_text("/* a\n note */ // kernel, reworded\n")
+    assert bench.kernel_source_hash() == h2
+    (csrc / "k.cu").write_text("// kernel\nint x;\n")
+    assert bench.kernel_source_hash() != h2
+    assert bench.ncu_traffic("apply", "480p_bidir") is None
 
 
 def test_committed_profiles_name_their_command():
