@@ -265,8 +265,8 @@ la_status run_simt(const Launch& L) {
   if (!L.do_apply) return LA_OK;
   if (pl.causal) {
     const int C = kCausalChunk;
-    size_t smemc = ((size_t)D * (D + 1) + 5 * (size_t)C * D + 2 * (size_t)C * C + C) *
-                   sizeof(float);
+    size_t smemc = ((size_t)D * (D + 1) + 3 * (size_t)C * D + 2 * (size_t)C * (D + 1) +
+                    2 * (size_t)C * C + C) * sizeof(float);
     if ((st = set_smem(apply_causal_simt<D, T>, smemc)) != LA_OK) return st;
     const int gc = pl.sc.nseg < (1 << 20) ? pl.sc.nseg : (1 << 20);
     apply_causal_simt<D, T><<<gc, kSimtThreads, smemc, L.stream>>>(

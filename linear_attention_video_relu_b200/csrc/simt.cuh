@@ -161,16 +161,21 @@ reduce_states(const float* __restrict__ partials, Sched sc, float* __restrict__ 
   for (int hh = blockIdx.y; hh < heads; hh += gridDim.y) {
   float run = 0.f;
   if (use_state) run = e < DD ? stS[(long long)hh * DD + e] : stz[(long long)hh * D + (e - DD)];
+  // software pipelined over the segments: the first partial of segment b + 1
+  // is requested before segment b is summed (same additions, same order)
+  const float* base0 = partials + (long long)hh * sc.nblk * sc.maxc * DD1 + e;
+  float first = base0[0];
   for (int b = 0; b < sc.nblk; ++b) {
     const int seg = hh * sc.nblk + b;
-    const long long ubeg = (long long)seg * sc.tps;
-    const int i0 = cta_of_unit(sc, ubeg), i1 = cta_of_unit(sc, ubeg + sc.tps - 1);
-    const float* base = partials + (long long)seg * sc.maxc * DD1 + e;
-    float blk = 0.f;
-    for (int i = i0; i <= i1; ++i) blk += base[(long long)(i - i0) * DD1];
+    const float* base = base0 + (long long)b * sc.maxc * DD1;
+    const int np = parts_of(sc, seg);
+    const float next = b + 1 < sc.nblk ? base[(long long)sc.maxc * DD1] : 0.f;
+    float blk = 0.f + first;
+    for (int i = 1; i < np; ++i) blk += base[(long long)i * DD1];
     const float ap = run + blk;
     apply[(long long)seg * DD1 + e] = ap;
     run = ap;
+    first = next;
   }
   if (use_state && commit) {
     if (e < DD) stS[(long long)hh * DD + e] = run;
@@ -271,11 +276,12 @@ apply_causal_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* s_S = reinterpret_cast<float*>(smem_raw);  // [D][D], then z [D]
   float* s_z = s_S + D * D;
-  float* s_qphi = s_z + D;                           // [C][D]
+  constexpr int KS = D + 1;                          // k row stride: rows j of a warp
+  float* s_qphi = s_z + D;                           // [C][D]   fall in distinct banks
   float* s_qr = s_qphi + C * D;
-  float* s_kphi = s_qr + C * D;
-  float* s_kr = s_kphi + C * D;
-  float* s_v = s_kr + C * D;
+  float* s_kphi = s_qr + C * D;                      // [C][KS]
+  float* s_kr = s_kphi + C * KS;
+  float* s_v = s_kr + C * KS;                        // [C][D]
   float* s_P = s_v + C * D;                          // [C][C] numerator weights
   float* s_Q = s_P + C * C;                          // [C][C] denominator weights
   float* s_den = s_Q + C * C;                        // [C]
@@ -314,15 +320,15 @@ apply_causal_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         krx = kx * cs.x - ky * cs.y;
         kry = kx * cs.y + ky * cs.x;
       }
-      const int o = r * D + 2 * pr;
+      const int o = r * D + 2 * pr, ok = r * KS + 2 * pr;
       s_qphi[o] = qx;
       s_qphi[o + 1] = qy;
       s_qr[o] = qrx;
       s_qr[o + 1] = qry;
-      s_kphi[o] = kx;
-      s_kphi[o + 1] = ky;
-      s_kr[o] = krx;
-      s_kr[o + 1] = kry;
+      s_kphi[ok] = kx;
+      s_kphi[ok + 1] = ky;
+      s_kr[ok] = krx;
+      s_kr[ok + 1] = kry;
       s_v[o] = v0;
       s_v[o + 1] = v1;
     }
@@ -333,8 +339,8 @@ apply_causal_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
       float p = 0.f, qq = 0.f;
       if (j <= i) {
         for (int a = 0; a < D; ++a) {
-          p = fmaf(s_qr[i * D + a], s_kr[j * D + a], p);
-          qq = fmaf(s_qphi[i * D + a], s_kphi[j * D + a], qq);
+          p = fmaf(s_qr[i * D + a], s_kr[j * KS + a], p);
+          qq = fmaf(s_qphi[i * D + a], s_kphi[j * KS + a], qq);
         }
       }
       s_P[idx] = p;

@@ -30,7 +30,6 @@
 #include "common.cuh"
 #include "linattn.h"
 #include "ptx.cuh"
-#include "simt.cuh"
 
 namespace la {
 
