@@ -37,7 +37,10 @@
  *     S[a][c] = sum_j RoPE(phi(k_j))_a v_j,c, and z [B, H, D].
  *   - Asynchrony. A call checks its arguments on the host, enqueues kernels on
  *     `stream` (a cudaStream_t passed as void*, NULL = legacy default stream)
- *     and returns; results are valid once the stream reaches that point.
+ *     and returns; results are valid once the stream reaches that point. The
+ *     tensor-core kernels use programmatic dependent launch: each may start
+ *     behind the kernel before it on the stream, but reads its inputs and
+ *     writes memory only after that kernel has completed.
  *   - Errors. Every call returns la_status; nothing aborts, prints or throws.
  *     Invalid arguments are rejected before any launch and leave memory
  *     untouched. A launch failure returns LA_ERR_CUDA.
@@ -137,8 +140,9 @@ LA_API la_status lin_attn_forward(const la_params* p, const void* q, const void*
 
 /* lin_attn_forward that also records four caller-created CUDA events (as
  * void*, e.g. cudaEvent_t) on `stream`: events[0] before the state build,
- * events[1] after it, events[2] after the reduction, events[3] after the
- * apply step, so a caller can time each kernel on the launching stream.
+ * events[1] after it, events[2] after the reduction (at once when the state
+ * build performs it), events[3] after the apply step, so a caller can time
+ * each kernel on the launching stream.
  * events may be NULL (then this is lin_attn_forward). */
 LA_API la_status lin_attn_forward_timed(const la_params* p, const void* q, const void* k,
                                         const void* v, const void* gate, void* out,
