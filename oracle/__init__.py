@@ -3,7 +3,8 @@
 TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
 baseline of ``bench.py`` use it; the CUDA library and its binding never do.
 The arithmetic lives in ``oracle.c`` (plain C, fp64, index-order sums); this
-file only compiles it with gcc and marshals numpy arrays.
+file compiles it with gcc and marshals numpy arrays, and holds the plain fp64
+numpy form of linear cross-attention at its end.
 
 Every function here is pinned by ``tests/test_oracle.py`` against the brute
 force O(N^2) form, closed forms, invariants of the SANA-Video equations and
@@ -196,4 +197,50 @@ def bruteforce(p: Params, q, k, v, g=None, nthreads: int = 0) -> np.ndarray:
     _check(lib().orc_bruteforce(ctypes.byref(p), qp, kp, vp, gp,
                                 out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
                                 nthreads), "bruteforce")
+    return out
+
+
+# ---- linear cross-attention -------------------------------------------------
+#
+# Queries of one sequence read the keys and values of another (N_q != N_kv,
+# e.g. video tokens attending to text tokens), with the same ReLU kernel and
+# no rotation (the two sequences share no positions): the linear
+# cross-attention the SANA-Video paper-graph page names beside its
+# self-attention. Plain fp64 numpy, written from the definition.
+
+def cross_forward(q, k, v, g=None, eps: float = 1e-6) -> np.ndarray:
+    """out[b,h,i] = phi(q_i) S / (phi(q_i) . z + eps) (* sigmoid(g_i)), with
+    S = sum_j phi(k_j)^T v_j and z = sum_j phi(k_j) over the N_kv keys of the
+    same (b, h). q, g: [B,H,Nq,D]; k, v: [B,H,Nkv,D]."""
+    q = np.maximum(np.asarray(q, dtype=np.float64), 0.0)
+    k = np.maximum(np.asarray(k, dtype=np.float64), 0.0)
+    v = np.asarray(v, dtype=np.float64)
+    S = np.einsum("bhja,bhjc->bhac", k, v)
+    z = k.sum(axis=2)
+    num = np.einsum("bhia,bhac->bhic", q, S)
+    den = np.einsum("bhia,bha->bhi", q, z) + eps
+    out = num / den[..., None]
+    if g is not None:
+        out = out / (1.0 + np.exp(-np.asarray(g, dtype=np.float64)))
+    return out
+
+
+def cross_bruteforce(q, k, v, g=None, eps: float = 1e-6) -> np.ndarray:
+    """The attention-weight form: out_i = sum_j w_ij v_j / (sum_j w_ij + eps)
+    with w_ij = phi(q_i) . phi(k_j); tiny inputs only."""
+    q = np.maximum(np.asarray(q, dtype=np.float64), 0.0)
+    k = np.maximum(np.asarray(k, dtype=np.float64), 0.0)
+    v = np.asarray(v, dtype=np.float64)
+    B, H, Nq, D = q.shape
+    out = np.zeros((B, H, Nq, D))
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nq):
+                w = [float(np.dot(q[b, h, i], k[b, h, j])) for j in range(k.shape[2])]
+                acc = np.zeros(D)
+                for j, wj in enumerate(w):
+                    acc += wj * v[b, h, j]
+                out[b, h, i] = acc / (sum(w) + eps)
+    if g is not None:
+        out = out / (1.0 + np.exp(-np.asarray(g, dtype=np.float64)))
     return out

@@ -355,3 +355,46 @@ def test_bad_arguments_are_rejected():
     p = oracle.make_params(1, 1, 12, 8, grid=(1, 3, 4), rope_split=(2, 2, 2))
     with pytest.raises(ValueError):
         oracle.forward(p, *_qkv(1, 1, 12, 8, 1))
+
+
+# ---- linear cross-attention (numpy fp64 form) --------------------------------
+
+def test_cross_matches_bruteforce_with_gate():
+    rng = np.random.default_rng(301)
+    q = rng.standard_normal((2, 2, 9, 8))
+    k = rng.standard_normal((2, 2, 5, 8))
+    v = rng.standard_normal((2, 2, 5, 8))
+    g = rng.standard_normal((2, 2, 9, 8))
+    np.testing.assert_allclose(oracle.cross_forward(q, k, v, g), oracle.cross_bruteforce(q, k, v, g),
+                               rtol=1e-12, atol=1e-14)
+
+
+def test_cross_with_equal_lengths_is_the_self_attention_oracle():
+    # the C oracle's bidirectional form without RoPE is an independent
+    # implementation of the same sums when queries and keys share a length
+    B, H, N, D = 1, 3, 40, 32
+    q, k, v = _qkv(B, H, N, D, 302)
+    g = _rand(q.shape, 303)
+    ref = oracle.forward(oracle.make_params(B, H, N, D), q, k, v, g=g)
+    got = oracle.cross_forward(q, k, v, g)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_cross_closed_forms():
+    # a hand-worked case: phi(q) = (1, 0) meets k_0 = (2, 1) with weight 2 and
+    # k_1 = (0, 3) with weight 0, so out = 2 v_0 / (2 + eps)
+    q = np.array([[[[1.0, 0.0]]]])
+    k = np.array([[[[2.0, 1.0], [0.0, 3.0]]]])
+    v = np.array([[[[1.0, 2.0], [3.0, 4.0]]]])
+    out = oracle.cross_forward(q, k, v, eps=1e-6)
+    np.testing.assert_allclose(out[0, 0, 0], np.array([1.0, 2.0]) * 2.0 / (2.0 + 1e-6), rtol=1e-15)
+    # constant values come back (up to eps) whatever the queries and keys
+    rng = np.random.default_rng(304)
+    q = rng.standard_normal((1, 2, 7, 4))
+    k = np.abs(rng.standard_normal((1, 2, 3, 4))) + 0.5
+    v = np.broadcast_to(np.array([0.5, -1.0, 2.0, 3.0]), (1, 2, 3, 4))
+    out = oracle.cross_forward(q, k, v, eps=0.0)
+    rows = (np.maximum(q, 0).sum(-1) > 0)
+    np.testing.assert_allclose(out[rows], np.broadcast_to(v[0, 0, 0], out[rows].shape), rtol=1e-12)
+    # queries with no positive entry give exactly zero
+    assert np.array_equal(oracle.cross_forward(-np.abs(q), k, v), np.zeros_like(q))
