@@ -149,6 +149,25 @@ LA_API la_status lin_attn_forward_timed(const la_params* p, const void* q, const
                                         void* workspace, size_t workspace_bytes, void* stream,
                                         void* const* events);
 
+/* Linear cross-attention: the p->N queries of each (b, h) read S, z summed
+ * over n_kv keys and values of the same (b, h), e.g. video tokens attending
+ * to text tokens (the linear cross-attention the SANA-Video paper-graph page
+ * lists beside self-attention):
+ *     out_i = phi(q_i) . S / (phi(q_i) . z + eps) (* sigmoid(g_i)),
+ *     S = sum_j phi(k_j)^T v_j,   z = sum_j phi(k_j),   j < n_kv.
+ * q, gate, out: [B,H,N,D]; k, v: [B,H,n_kv,D], all in p->dtype. The two
+ * sequences share no positions: p->rope must be 0 and p->mode bidirectional
+ * (else LA_ERR_INVALID_ARG); n_kv >= 1 (N = 0: no work).
+ * workspace: at least lin_attn_cross_workspace_size bytes, as in
+ * lin_attn_forward. */
+LA_API la_status lin_attn_cross_forward(const la_params* p, int n_kv, const void* q,
+                                        const void* k, const void* v, const void* gate,
+                                        void* out, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
+/* Bytes of workspace lin_attn_cross_forward needs for `p` and n_kv. */
+LA_API la_status lin_attn_cross_workspace_size(const la_params* p, int n_kv, size_t* bytes);
+
 /* Size of the fixed scratch area that lin_attn_forward_noalloc uses. */
 #define LA_NOALLOC_SCRATCH_BYTES (32u << 20)
 

@@ -55,6 +55,10 @@ SIGNATURES = {
     "lin_attn_forward_timed": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, ctypes.c_size_t, _V,
                                               ctypes.POINTER(ctypes.c_void_p)]),
     "lin_attn_forward_noalloc": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
+    "lin_attn_cross_forward": (ctypes.c_int, [_P, ctypes.c_int, _V, _V, _V, _V, _V, _V,
+                                              ctypes.c_size_t, _V]),
+    "lin_attn_cross_workspace_size": (ctypes.c_int, [_P, ctypes.c_int,
+                                                     ctypes.POINTER(ctypes.c_size_t)]),
     "lin_attn_state_init": (ctypes.c_int, [_ST, ctypes.c_int, ctypes.c_int, ctypes.c_int, _V, _V]),
     "lin_attn_state_reset": (ctypes.c_int, [_ST, _V]),
     "lin_attn_block_step": (ctypes.c_int, [_P, _ST, ctypes.c_int, _V, _V, _V, _V, _V, ctypes.c_int,
@@ -129,6 +133,19 @@ def lin_attn_forward_timed(p, q, k, v, gate, out, workspace, workspace_bytes, st
 
 def lin_attn_forward_noalloc(p, q, k, v, gate, out, stream) -> int:
     return load().lin_attn_forward_noalloc(ctypes.byref(p), q, k, v, gate, out, stream)
+
+
+def lin_attn_cross_forward(p, n_kv, q, k, v, gate, out, workspace, workspace_bytes,
+                           stream) -> int:
+    return load().lin_attn_cross_forward(ctypes.byref(p), n_kv, q, k, v, gate, out, workspace,
+                                         workspace_bytes, stream)
+
+
+def lin_attn_cross_workspace_size(p: la_params, n_kv: int) -> int:
+    n = ctypes.c_size_t(0)
+    check(load().lin_attn_cross_workspace_size(ctypes.byref(p), n_kv, ctypes.byref(n)),
+          "lin_attn_cross_workspace_size")
+    return n.value
 
 
 def lin_attn_state_init(st: la_state, B, H, D, S, z) -> int:

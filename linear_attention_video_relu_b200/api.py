@@ -106,6 +106,36 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[to
     return out
 
 
+def cross_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                  gate: Optional[torch.Tensor] = None, *, eps: float = 1e-6,
+                  out: Optional[torch.Tensor] = None, workspace: Optional[Workspace] = None,
+                  stream=None) -> torch.Tensor:
+    """Linear cross-attention: q, gate, out [B, H, N, D] read the state of
+    k, v [B, H, M, D] (no RoPE; every query sees every key)."""
+    B, H, N, D = q.shape
+    if k.dim() != 4 or tuple(k.shape[:2]) != (B, H) or k.shape[3] != D:
+        raise ValueError("k must be [B, H, M, D] with q's B, H, D; got %s" % (tuple(k.shape),))
+    M = int(k.shape[2])
+    p = make_params(B, H, N, D, q.dtype, eps=eps)
+    pk = make_params(B, H, M, D, q.dtype, eps=eps)
+    _check_io(p, q, gate)
+    _check_io(pk, k, v)
+    for t in (k, v, gate):
+        if t is not None and t.dtype != q.dtype:
+            raise TypeError("q, k, v and gate must share one dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    _check_io(p, out)
+    if workspace is None:
+        with torch.cuda.device(q.device):
+            workspace = Workspace(C.lin_attn_cross_workspace_size(p, M), q.device)
+    with torch.cuda.device(q.device):
+        C.check(C.lin_attn_cross_forward(p, M, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(out),
+                                         workspace.ptr, workspace.nbytes, _stream(stream)),
+                "lin_attn_cross_forward")
+    return out
+
+
 class BlockState:
     """The constant-memory cache (S, z) of block-causal generation."""
 

@@ -42,6 +42,8 @@ struct Plan {
   Rope rope;
   Sched sc;
   long long heads;
+  long long nq;        // query tokens per head (N; the query length of a cross-attention)
+  int lq;              // query rows per segment (sc.L, or nq for a cross-attention)
   int apply_tps;       // SIMT apply: tiles per segment
   int sms;             // SM count of the device
   size_t off_flag, off_tab, off_part, off_apply, total;
@@ -178,6 +180,8 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
       if (c > sc.maxc) sc.maxc = c;
     }
   }
+  pl->nq = N;
+  pl->lq = sc.L;
   pl->apply_tps = (sc.L + kSimtTileApply - 1) / kSimtTileApply;
 
   const size_t dd1 = (size_t)p->D * (p->D + 1);
@@ -282,8 +286,8 @@ la_status run_simt(const Launch& L) {
   if (st != LA_OK) return st;
   dim3 g3(pl.apply_tps, pl.sc.nseg < 65535 ? pl.sc.nseg : 65535);
   apply_simt<D, T><<<g3, kSimtThreads, smem3, L.stream>>>(
-      static_cast<const T*>(L.q), static_cast<const T*>(L.g), static_cast<T*>(L.out), N,
-      pl.rope, pl.sc.L, pl.sc.nblk, pl.apply_tps, pl.sc.nseg, apply, gtab, L.p->eps);
+      static_cast<const T*>(L.q), static_cast<const T*>(L.g), static_cast<T*>(L.out), pl.nq,
+      pl.rope, pl.lq, pl.sc.nblk, pl.apply_tps, pl.sc.nseg, apply, gtab, L.p->eps);
   if ((st = last_error()) != LA_OK) return st;
   return mark(L, 3);
 }
@@ -303,6 +307,7 @@ la_status run(const Launch& L) {
     TcArgs a;
     a.D = L.p->D;
     a.N = L.p->N;
+    a.Lq = L.pl->lq;
     a.rope = L.pl->rope;
     a.sc = L.pl->sc;
     a.heads = L.pl->heads;
@@ -383,6 +388,21 @@ la_status block_common(const la_params* p, la_state* st, int t_offset, const voi
   return run(L);
 }
 
+// Plan of a linear cross-attention: the state is built from the n_kv keys and
+// values of each head (one segment per head), and applied to the p->N queries.
+la_status cross_plan(const la_params* p, int n_kv, Plan* pl) {
+  la_status s = check_params(p, false);
+  if (s != LA_OK) return s;
+  if (p->rope || p->mode != LA_BIDIRECTIONAL || n_kv < 1) return LA_ERR_INVALID_ARG;
+  la_params pk = *p;
+  pk.N = n_kv;
+  if ((s = make_plan(&pk, false, 0, pl)) != LA_OK) return s;
+  pl->nq = p->N;
+  pl->lq = p->N;
+  pl->apply_tps = (p->N + kSimtTileApply - 1) / kSimtTileApply;
+  return LA_OK;
+}
+
 // ---- fixed scratch for lin_attn_forward_noalloc ----------------------------
 //
 // The one device array behind lin_attn_forward_noalloc. In host code its name
@@ -452,6 +472,43 @@ la_status lin_attn_forward_timed(const la_params* p, const void* q, const void* 
   if ((s = check_workspace(pl, workspace, workspace_bytes)) != LA_OK) return s;
   Launch L{p, &pl, q, k, v, gate, out, static_cast<unsigned char*>(workspace), nullptr, nullptr,
            0, 0, 1, static_cast<cudaStream_t>(stream), events};
+  return run(L);
+}
+
+la_status lin_attn_cross_workspace_size(const la_params* p, int n_kv, size_t* bytes) {
+  if (!bytes) return LA_ERR_INVALID_ARG;
+  Plan pl;
+  la_status s = cross_plan(p, n_kv, &pl);
+  if (s != LA_OK) return s;
+  *bytes = pl.total;
+  return LA_OK;
+}
+
+la_status lin_attn_cross_forward(const la_params* p, int n_kv, const void* q, const void* k,
+                                 const void* v, const void* gate, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  la_status s = check_params(p, false);
+  if (s != LA_OK) return s;
+  if (p->rope || p->mode != LA_BIDIRECTIONAL || n_kv < 1) return LA_ERR_INVALID_ARG;
+  if ((long long)p->B * p->H * p->N == 0) return LA_OK;
+  if ((s = check_tensor(q, true)) != LA_OK) return s;
+  if ((s = check_tensor(k, true)) != LA_OK) return s;
+  if ((s = check_tensor(v, true)) != LA_OK) return s;
+  if ((s = check_tensor(out, true)) != LA_OK) return s;
+  if (gate && !aligned16(gate)) return LA_ERR_INVALID_ARG;
+  const size_t heads = (size_t)p->B * p->H;
+  const size_t qb = heads * p->N * p->D * elt_size(p);
+  const size_t kb = heads * (size_t)n_kv * p->D * elt_size(p);
+  if (overlaps(out, qb, q, qb) || overlaps(out, qb, k, kb) || overlaps(out, qb, v, kb) ||
+      overlaps(out, qb, gate, qb))
+    return LA_ERR_INVALID_ARG;
+  Plan pl;
+  if ((s = cross_plan(p, n_kv, &pl)) != LA_OK) return s;
+  if ((s = check_workspace(pl, workspace, workspace_bytes)) != LA_OK) return s;
+  la_params pk = *p;
+  pk.N = n_kv;
+  Launch L{&pk, &pl, q, k, v, gate, out, static_cast<unsigned char*>(workspace), nullptr,
+           nullptr, 0, 0, 1, static_cast<cudaStream_t>(stream), nullptr};
   return run(L);
 }
 

@@ -43,6 +43,7 @@ enum : int { kFlagStateTimeout = 1, kFlagApplyTimeout = 2 };
 struct TcArgs {
   int D;
   long long N;
+  int Lq;          // query rows per segment: sc.L, or the query length of a cross-attention
   Rope rope;
   Sched sc;
   long long heads;
@@ -1464,20 +1465,20 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   if (!a.do_apply) return LA_OK;
 
   const bool gate = a.g != nullptr;
-  if (!make_map(&mq, a.q, D, sc.L, sc.nseg, kApplyTile) ||
-      !make_map(&mo, a.out, D, sc.L, sc.nseg, kApplyTile) ||
-      !make_map(&mg, gate ? a.g : a.q, D, sc.L, sc.nseg, kApplyTile))
+  if (!make_map(&mq, a.q, D, a.Lq, sc.nseg, kApplyTile) ||
+      !make_map(&mo, a.out, D, a.Lq, sc.nseg, kApplyTile) ||
+      !make_map(&mg, gate ? a.g : a.q, D, a.Lq, sc.nseg, kApplyTile))
     return LA_ERR_CUDA;
   int s3 = 0, sb3 = 1, gs3 = 0;
   pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3, &gs3);
   const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3, sb3, gs3);
-  const long long U3 = (long long)sc.nseg * ((sc.L + kApplyTile - 1) / kApplyTile);
+  const long long U3 = (long long)sc.nseg * ((a.Lq + kApplyTile - 1) / kApplyTile);
   const int G3 = (int)(U3 < sms ? U3 : sms);
   auto k3 = a.rope.on ? (gate ? apply_tc<D, true, true> : apply_tc<D, true, false>)
                       : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
   if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
   st = launch_pdl(k3, dim3(G3), dim3(kTcThreadsApply), p3.total, a.stream, mq, mg, mo,
-                  static_cast<__nv_bfloat16*>(a.out), a.rope, sc.L, sc.nblk, U3, s3, sb3, gs3,
+                  static_cast<__nv_bfloat16*>(a.out), a.rope, a.Lq, sc.nblk, U3, s3, sb3, gs3,
                   reinterpret_cast<const uint8_t*>(a.apply), (const float2*)a.gtab, a.eps,
                   a.flag);
   if (st != LA_OK) return st;

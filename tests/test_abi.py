@@ -155,3 +155,36 @@ def test_control_block_size_matches_the_header():
     text = open(HEADER).read()
     m = re.search(r"#define\s+LA_WORKSPACE_CONTROL_BYTES\s+(\d+)u?", text)
     assert m and int(m.group(1)) == C.LA_WORKSPACE_CONTROL_BYTES
+
+
+def _cross(**kw):
+    return _params(rope=0, **kw)
+
+
+def test_cross_forward_rejects_what_it_does_not_define():
+    ok = _cross()
+    for p, n_kv in ((_params(), 40), (_cross(mode=C.LA_BLOCK_CAUSAL, block_tokens=20), 40),
+                    (_cross(mode=C.LA_TOKEN_CAUSAL), 40), (ok, 0), (ok, -3), (_cross(D=48), 40)):
+        assert C.lin_attn_cross_forward(p, n_kv, Q, K, V, None, O, WS, 1 << 20, None) == \
+            C.LA_ERR_INVALID_ARG
+        with pytest.raises(C.LinAttnError):
+            C.lin_attn_cross_workspace_size(p, n_kv)
+
+
+def test_cross_forward_pointer_checks_use_each_sequence_length():
+    p = _cross()                       # q, out: 2 heads x 60 x 32 bf16 = 7680 bytes
+    assert C.lin_attn_cross_forward(p, 40, None, K, V, None, O, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_cross_forward(p, 40, Q, K, None, None, O, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_cross_forward(p, 40, Q, K, V, O + 2, O, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    # out 32 KB past k: clear of k when k holds 40 tokens, inside it at 500
+    out = K + 0x8000
+    assert C.lin_attn_cross_forward(p, 500, Q, K, V, None, out, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_cross_forward(p, 40, Q, K, V, None, out, WS, 1 << 20, None) != \
+        C.LA_ERR_INVALID_ARG
+    # no queries: no work, whatever the pointers
+    assert C.lin_attn_cross_forward(_cross(N=0), 7, None, None, None, None, None, None, 0,
+                                    None) == C.LA_OK
