@@ -355,6 +355,46 @@ def measure_block_steps(w, steps, warmup, device, peak, peak_kind, seed):
             "hbm_frac": bytes_blk / (ms * 1e-3) / 1e9 / peak}
 
 
+def measure_cross(w, n_kv, steps, warmup, device, peak, seed):
+    """Linear cross-attention: the workload's video tokens as queries reading
+    n_kv text tokens per head as keys and values (no RoPE), one C-ABI call per
+    forward, CUDA events around `steps` calls."""
+    import torch
+    import linear_attention_video_relu_b200 as la
+    C = la._native
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    bf = torch.bfloat16
+    q = torch.randn((w.B, w.H, w.N, w.D), generator=g, device=device).to(bf)
+    k = torch.randn((w.B, w.H, n_kv, w.D), generator=g, device=device).to(bf)
+    v = torch.randn((w.B, w.H, n_kv, w.D), generator=g, device=device).to(bf)
+    out = torch.empty_like(q)
+    p = la.make_params(w.B, w.H, w.N, w.D, bf, eps=w.eps)
+    ws = la.Workspace(C.lin_attn_cross_workspace_size(p, n_kv), device)
+    stream = torch.cuda.current_stream(device)
+    args = (p, n_kv, q.data_ptr(), k.data_ptr(), v.data_ptr(), None, out.data_ptr(), ws.ptr,
+            ws.nbytes, stream.cuda_stream)
+    for _ in range(warmup):
+        C.check(C.lin_attn_cross_forward(*args), "lin_attn_cross_forward")
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        C.check(C.lin_attn_cross_forward(*args), "lin_attn_cross_forward")
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    st = C.lin_attn_device_status(ws.ptr, stream.cuda_stream)
+    if st != C.LA_OK:
+        raise RuntimeError("device status after timing: %s" % C.status_string(st))
+    ms = a.elapsed_time(b) / steps
+    nbytes = 2 * 2 * w.B * w.H * (w.N + n_kv) * w.D     # read q, k, v; write out (bf16)
+    del q, k, v, out
+    return {"workload": "%s_x_text%d" % (w.name, n_kv), "mode": "cross", "n_kv": n_kv,
+            "us_per_forward": ms * 1e3, "tokens_per_s": w.B * w.N / (ms * 1e-3),
+            "algorithmic_bytes": nbytes, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peak}
+
+
 def measure_e2e(w, steps, device, seed):
     """The same forward end to end: host (pinned) inputs copied in, the C-ABI
     call, the output copied back, every step, all inside the timed region."""
@@ -561,6 +601,8 @@ def main():
             ww = workloads.WORKLOADS[name]
             extra.append(measure_workload(ww, mode, K, 3, None, device, peak, peak_kind,
                                           ww.seed))
+        extra.append(measure_cross(workloads.WORKLOADS["480p_bidir"], 300, K, 5, device, peak,
+                                   2002))
         extra.append(measure_block_steps(workloads.WORKLOADS["720p_long"], 120, 60, device, peak,
                                          peak_kind, 1004))
         line["also"] = extra
