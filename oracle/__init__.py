@@ -4,7 +4,8 @@ TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
 baseline of ``bench.py`` use it; the CUDA library and its binding never do.
 The arithmetic lives in ``oracle.c`` (plain C, fp64, index-order sums); this
 file compiles it with gcc and marshals numpy arrays, and holds the plain fp64
-numpy form of linear cross-attention at its end.
+numpy form of linear cross-attention at its end. ``oracle.tconv`` holds the
+fp64 Mix-FFN temporal convolution with its last-frame cache.
 
 Every function here is pinned by ``tests/test_oracle.py`` against the brute
 force O(N^2) form, closed forms, invariants of the SANA-Video equations and
