@@ -110,8 +110,9 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-# CUDA-core kernels: not part of the profiled tensor-core kernels' sources
-_NOT_TC_SOURCES = ("simt.cuh",)
+# CUDA-core attention kernels and the temporal convolution: not part of the
+# profiled tensor-core kernels' sources
+_NOT_TC_SOURCES = ("simt.cuh", "tconv.cu")
 
 
 def kernel_source_hash() -> str:
@@ -395,6 +396,45 @@ def measure_cross(w, n_kv, steps, warmup, device, peak, seed):
             "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peak}
 
 
+def measure_tconv(steps, warmup, device, peak, seed):
+    """The Mix-FFN temporal convolution on 480p hidden states (B=1, 21 frames x
+    1560 positions x 2240 channels, bf16) with bias, reading and writing the
+    last-frame cache: CUDA events around `steps` calls."""
+    import torch
+    import linear_attention_video_relu_b200 as la
+    C = la._native
+    sh = workloads.TCONV_480P
+    B, T, S, nc = sh["B"], sh["T"], sh["S"], sh["C"]
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    bf = torch.bfloat16
+    x = torch.randn((B, T, S, nc), generator=g, device=device).to(bf)
+    w = 0.5 * torch.randn((3, nc), generator=g, device=device)
+    b = 0.1 * torch.randn((nc,), generator=g, device=device)
+    cache_in = torch.randn((B, S, nc), generator=g, device=device).to(bf)
+    cache_out = torch.empty_like(cache_in)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(device)
+    args = (B, T, S, nc, C.LA_BF16, x.data_ptr(), w.data_ptr(), b.data_ptr(),
+            cache_in.data_ptr(), y.data_ptr(), cache_out.data_ptr(), stream.cuda_stream)
+    for _ in range(warmup):
+        C.check(C.lin_attn_temporal_conv(*args), "lin_attn_temporal_conv")
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        C.check(C.lin_attn_temporal_conv(*args), "lin_attn_temporal_conv")
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    nbytes = (2 * T + 2) * B * S * nc * 2     # x in, y out, cache frame in and out (bf16)
+    del x, y, cache_in, cache_out
+    return {"workload": "480p_hidden_tconv", "mode": "temporal_conv_cached",
+            "shape": [B, T, S, nc], "us_per_call": ms * 1e3,
+            "tokens_per_s": B * T * S / (ms * 1e-3), "algorithmic_bytes": nbytes,
+            "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peak}
+
+
 def measure_e2e(w, steps, device, seed):
     """The same forward end to end: host (pinned) inputs copied in, the C-ABI
     call, the output copied back, every step, all inside the timed region."""
@@ -603,6 +643,7 @@ def main():
                                           ww.seed))
         extra.append(measure_cross(workloads.WORKLOADS["480p_bidir"], 300, K, 5, device, peak,
                                    2002))
+        extra.append(measure_tconv(K, 5, device, peak, 2003))
         extra.append(measure_block_steps(workloads.WORKLOADS["720p_long"], 120, 60, device, peak,
                                          peak_kind, 1004))
         line["also"] = extra

@@ -240,6 +240,37 @@ LA_API const char* lin_attn_status_string(la_status s);
  * tensor-core path). */
 LA_API int lin_attn_uses_tensor_cores(const la_params* p);
 
+/* ---- Mix-FFN temporal convolution with the last-frame cache -------------
+ * The temporal convolution of the spatial-temporal Mix-FFN (SANA-Video
+ * paper-graph page, "Spatial-Temporal Mix-FFN": kernel size 3 along time, a
+ * 3x1x1 kernel on the [T, H, W, C] hidden states, added through a shortcut)
+ * and its block-causal form ("Block Causal Mix-FFN": a zero frame after the
+ * block, the previous block's last frame cached and put before it; the conv
+ * cache of Algorithm 1). Per channel c (depthwise), frame t, position s:
+ *     y[b,t,s,c] = x[b,t,s,c] + w[0][c] x[b,t-1,s,c] + w[1][c] x[b,t,s,c]
+ *                  + w[2][c] x[b,t+1,s,c]  (+ bias[c]),
+ * with frame T (after the block) zero and frame -1 = cache_in, or zero when
+ * cache_in is NULL (the first block, or a whole-sequence call).
+ *   x, y:      [B, T, S, C] in dtype, C innermost (the [B, N, C] hidden states
+ *              of a DiT block, N = T * S, S = grid_h * grid_w).
+ *   weight:    fp32 [3][C], tap 0 on frame t-1, tap 1 on t, tap 2 on t+1.
+ *   bias:      fp32 [C], or NULL (none).
+ *   cache_in:  [B, S, C] in dtype, or NULL.
+ *   cache_out: [B, S, C] in dtype, or NULL; receives x[:, T-1], the block's
+ *              last input frame, after cache_in has been read, so cache_out ==
+ *              cache_in updates the cache in place.
+ * Arithmetic in fp32, one rounding to dtype per output; no workspace.
+ * Errors (LA_ERR_INVALID_ARG, nothing launched): a negative size; dtype not
+ * LA_F32 / LA_BF16; C not a multiple of 16 bytes' worth of dtype (8 bf16,
+ * 4 fp32); x, y or weight NULL when there is work; any pointer not 16-byte
+ * aligned; y overlapping another buffer; cache_out overlapping x, weight or
+ * bias, or overlapping cache_in without being equal to it. B*T*S*C = 0: no
+ * work, cache_out untouched. */
+LA_API la_status lin_attn_temporal_conv(int B, int T, int S, int C, la_dtype dtype,
+                                        const void* x, const float* weight, const float* bias,
+                                        const void* cache_in, void* y, void* cache_out,
+                                        void* stream);
+
 #ifdef __cplusplus
 }
 #endif

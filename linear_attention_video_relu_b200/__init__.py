@@ -11,8 +11,8 @@ The computation is the C-ABI CUDA library ``liblinattn.so`` (include/linattn.h);
 ``_native`` binds it with the same names and ``api`` wraps it for torch tensors.
 """
 from . import _native
-from .api import (BlockState, Workspace, cross_forward, forward, make_params, uses_tensor_cores,
-                  workspace_for)
+from .api import (BlockState, Workspace, cross_forward, forward, make_params, temporal_conv,
+                  uses_tensor_cores, workspace_for)
 
-__all__ = ["BlockState", "Workspace", "cross_forward", "forward", "make_params", "uses_tensor_cores",
-           "workspace_for", "_native"]
+__all__ = ["BlockState", "Workspace", "cross_forward", "forward", "make_params", "temporal_conv",
+           "uses_tensor_cores", "workspace_for", "_native"]

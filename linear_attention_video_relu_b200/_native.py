@@ -68,6 +68,9 @@ SIGNATURES = {
     "lin_attn_device_status": (ctypes.c_int, [_V, _V]),
     "lin_attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "lin_attn_uses_tensor_cores": (ctypes.c_int, [_P]),
+    "lin_attn_temporal_conv": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, _V, _V, _V, _V, _V,
+                                              _V, _V]),
 }
 
 _lib = None
@@ -173,3 +176,9 @@ def lin_attn_device_status(workspace, stream) -> int:
 
 def lin_attn_uses_tensor_cores(p: la_params) -> int:
     return load().lin_attn_uses_tensor_cores(ctypes.byref(p))
+
+
+def lin_attn_temporal_conv(B, T, S, C, dtype, x, weight, bias, cache_in, y, cache_out,
+                           stream) -> int:
+    return load().lin_attn_temporal_conv(B, T, S, C, dtype, x, weight, bias, cache_in, y,
+                                         cache_out, stream)

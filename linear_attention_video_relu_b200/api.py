@@ -190,3 +190,47 @@ class BlockState:
 
 def uses_tensor_cores(B, H, N, D, dtype, **kw) -> bool:
     return bool(C.lin_attn_uses_tensor_cores(make_params(B, H, N, D, dtype, **kw)))
+
+
+def temporal_conv(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                  cache_in: Optional[torch.Tensor] = None, *,
+                  cache_out: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """Mix-FFN temporal convolution with the last-frame cache:
+    y[t] = x[t] + w0 * x[t-1] + w1 * x[t] + w2 * x[t+1] (+ bias), per channel,
+    with a zero frame after the block and cache_in (or zero) before it.
+
+    x, out: [B, T, S, C] or [B, T, Hg, Wg, C] (bf16 or fp32); weight fp32
+    [3, C]; bias fp32 [C]; cache_in, cache_out: one frame, [B, S, C] or
+    [B, Hg, Wg, C], in x's dtype. cache_out receives x's last frame (it may be
+    cache_in itself)."""
+    if x.dim() not in (4, 5):
+        raise ValueError("x must be [B, T, S, C] or [B, T, Hg, Wg, C]")
+    if x.dtype not in _DTYPES:
+        raise TypeError("x must be bf16 or fp32")
+    B, T, nc = int(x.shape[0]), int(x.shape[1]), int(x.shape[-1])
+    S = 1
+    for d in x.shape[2:-1]:
+        S *= int(d)
+    frame_shape = (B,) + tuple(x.shape[2:])
+    if out is None:
+        out = torch.empty_like(x)
+    for t, shape, dt, what in ((x, tuple(x.shape), x.dtype, "x"),
+                               (out, tuple(x.shape), x.dtype, "out"),
+                               (weight, (3, nc), torch.float32, "weight"),
+                               (bias, (nc,), torch.float32, "bias"),
+                               (cache_in, frame_shape, x.dtype, "cache_in"),
+                               (cache_out, frame_shape, x.dtype, "cache_out")):
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous CUDA tensor" % what)
+        if tuple(t.shape) != shape or t.dtype != dt:
+            raise ValueError("%s must be %s %s, got %s %s" % (what, shape, dt, tuple(t.shape),
+                                                            t.dtype))
+    with torch.cuda.device(x.device):
+        C.check(C.lin_attn_temporal_conv(B, T, S, nc, _DTYPES[x.dtype], _ptr(x), _ptr(weight),
+                                         _ptr(bias), _ptr(cache_in), _ptr(out), _ptr(cache_out),
+                                         _stream(stream)),
+                "lin_attn_temporal_conv")
+    return out

@@ -1,8 +1,9 @@
 """Build liblinattn.so in-tree with nvcc for sm_100a.
 
-The library is one translation unit (csrc/linattn.cu and the headers it
-includes) with the CUDA runtime linked statically, so the shared object only
-needs the driver at run time.
+The library is two translation units (csrc/linattn.cu with the headers it
+includes: the attention kernels; csrc/tconv.cu: the Mix-FFN temporal
+convolution) with the CUDA runtime linked statically, so the shared object
+only needs the driver at run time.
 """
 from __future__ import annotations
 
@@ -43,7 +44,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + ".tmp.%d" % os.getpid()
     cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           os.path.join(CSRC, "linattn.cu"), "-o", tmp]
+           os.path.join(CSRC, "linattn.cu"), os.path.join(CSRC, "tconv.cu"), "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)

@@ -188,3 +188,31 @@ def test_cross_forward_pointer_checks_use_each_sequence_length():
     # no queries: no work, whatever the pointers
     assert C.lin_attn_cross_forward(_cross(N=0), 7, None, None, None, None, None, None, 0,
                                     None) == C.LA_OK
+
+
+def _tconv(B=1, T=3, S=5, nc=16, dtype=C.LA_BF16, x=0x100000, w=0x200000, b=None,
+           cin=None, y=0x300000, cout=None):
+    return C.lin_attn_temporal_conv(B, T, S, nc, dtype, x, w, b, cin, y, cout, None)
+
+
+def test_temporal_conv_rejects_bad_arguments_on_the_host():
+    bad = C.LA_ERR_INVALID_ARG
+    assert _tconv(T=-1) == bad and _tconv(S=-2) == bad and _tconv(nc=-8) == bad
+    assert _tconv(dtype=9) == bad
+    assert _tconv(nc=12) == bad                          # bf16: 8 channels per 16 bytes
+    assert _tconv(nc=12, dtype=C.LA_F32) != bad          # fp32: 4 channels per 16 bytes
+    assert _tconv(x=None) == bad and _tconv(y=None) == bad and _tconv(w=None) == bad
+    assert _tconv(x=0x100008) == bad and _tconv(b=0x400004) == bad
+    assert _tconv(cin=0x500002) == bad and _tconv(cout=0x600001) == bad
+    # x: 1 x 3 x 5 x 16 bf16 = 480 bytes; one cache frame: 160 bytes
+    assert _tconv(y=0x100000 + 256) == bad               # y overlapping x
+    assert _tconv(cin=0x300000 + 64) == bad              # y overlapping cache_in
+    assert _tconv(cout=0x100000 + 320) == bad            # cache_out overlapping x
+    assert _tconv(cin=0x500000, cout=0x500000 + 16) == bad   # partial overlap of the caches
+    assert _tconv(cin=0x500000, cout=0x500000) != bad    # the in-place cache update
+    assert _tconv(b=0x400000, cin=0x500000, cout=0x600000) != bad
+
+
+def test_temporal_conv_without_work_is_a_no_op():
+    for kw in (dict(B=0), dict(T=0), dict(S=0), dict(nc=0)):
+        assert _tconv(x=None, w=None, y=None, **kw) == C.LA_OK

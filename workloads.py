@@ -145,3 +145,35 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray
         else:
             out[name] = x
     return out
+
+
+# Hidden states of a DiT block at 480p (21 x 30 x 52 latent grid, width 2240):
+# the temporal convolution's measured shape.
+TCONV_480P = dict(B=1, T=21, S=30 * 52, C=2240)
+
+
+def make_tconv_inputs(B: int, T: int, S: int, C: int, dtype: str, seed: int,
+                      cache: bool = True, bias: bool = True) -> Dict[str, np.ndarray]:
+    """Draw x [B, T, S, C], weight [3, C], bias [C] and a cache frame [B, S, C]
+    for the Mix-FFN temporal convolution, in that order: x and the cache
+    ~ N(0, 1) in I/O precision (plus ``*_bits`` for bf16), weight ~ 0.5 N(0, 1)
+    and bias ~ 0.1 N(0, 1) in fp32 (the op's weight precision)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out: Dict[str, np.ndarray] = {}
+
+    def io(name, shape):
+        x = _draw(rng, "normal", shape)
+        if dtype == "bf16":
+            bits = round_to_bf16_bits(x)
+            out[name + "_bits"] = bits
+            out[name] = bf16_bits_to_f32(bits)
+        else:
+            out[name] = x
+
+    io("x", (B, T, S, C))
+    out["weight"] = (0.5 * _draw(rng, "normal", (3, C))).astype(np.float32)
+    if bias:
+        out["bias"] = (0.1 * _draw(rng, "normal", (C,))).astype(np.float32)
+    if cache:
+        io("cache", (B, S, C))
+    return out
