@@ -102,7 +102,8 @@ def test_the_harness_passes_the_real_oracles(monkeypatch):
     # control: the same calls against the unmutated functions all pass
     pins = _load("test_oracle_tconv.py")
     monkeypatch.setattr(tconv, "temporal_conv",
-                        _mutant_function(tconv.temporal_conv, "y = x + w[0]", "y = x + w[0]"))
+                        _mutant_function(tconv.temporal_conv, "y = x + w[0] * framed",
+                                         "y = x + w[0] * framed"))
     assert not _any_fails([pins.test_hand_worked_case, pins.test_matches_scipy_correlation,
                            pins.test_blocks_versus_whole_sequence,
                            lambda: pins.test_matches_loops(5, True, True)])
