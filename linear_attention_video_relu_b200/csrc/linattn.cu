@@ -71,7 +71,7 @@ la_status device_sms(int* sms) {
 la_status check_params(const la_params* p, bool one_block) {
   if (!p) return LA_ERR_INVALID_ARG;
   if (p->B < 0 || p->H < 0 || p->N < 0) return LA_ERR_INVALID_ARG;
-  if (p->D != 32 && p->D != 64 && p->D != 128) return LA_ERR_INVALID_ARG;
+  if (p->D != 32 && p->D != 64 && p->D != 112 && p->D != 128) return LA_ERR_INVALID_ARG;
   if (p->dtype != LA_F32 && p->dtype != LA_BF16) return LA_ERR_INVALID_ARG;
   if (!one_block) {
     if (p->mode != LA_BIDIRECTIONAL && p->mode != LA_BLOCK_CAUSAL && p->mode != LA_TOKEN_CAUSAL)
@@ -297,6 +297,7 @@ la_status dispatch_simt(const Launch& L) {
   switch (L.p->D) {
     case 32: return run_simt<32, T>(L);
     case 64: return run_simt<64, T>(L);
+    case 112: return run_simt<112, T>(L);
     case 128: return run_simt<128, T>(L);
   }
   return LA_ERR_UNSUPPORTED;

@@ -179,6 +179,7 @@ CASES = [
     (1, 2, 256, 32, None, None, False),            # the tiny fp32 workload's shape
     (2, 2, 60, 32, (3, 4, 5), (8, 12, 12), False),  # RoPE on a 3x4x5 grid
     (1, 3, 64, 16, (4, 4, 4), (4, 6, 6), True),     # gate + odd head count
+    (1, 2, 48, 112, (3, 4, 4), (16, 48, 48), True),  # the 2B model's head dim, 56 pairs
 ]
 
 
