@@ -135,6 +135,9 @@ LA_API la_status lin_attn_block_step_workspace_size(const la_params* p, size_t* 
  * the block zero, and lin_attn_device_status re-zeroes it after a call that
  * gave up a bounded wait. The rest of the workspace may hold anything on entry
  * and is clobbered.
+ * Limits (else LA_ERR_UNSUPPORTED, nothing launched): B * H <= 2^24, and
+ * B * H times the segments of a head (1 bidirectional, N / block_tokens
+ * block-causal, ceil(N / 32) token-causal) <= INT_MAX.
  * Returns LA_OK once the work is enqueued on `stream`. */
 LA_API la_status lin_attn_forward(const la_params* p, const void* q, const void* k,
                            const void* v, const void* gate, void* out,

@@ -15,6 +15,7 @@
 // as segments and a chunked apply step.
 #include "linattn.h"
 
+#include <limits.h>
 #include <math.h>
 #include <string.h>
 
@@ -95,6 +96,11 @@ la_status check_params(const la_params* p, bool one_block) {
   }
   long long heads = (long long)p->B * p->H;
   if (heads > (1LL << 24)) return LA_ERR_UNSUPPORTED;
+  // segments (head x block, or head x token chunk) are indexed with int
+  long long nblk = 1;
+  if (!one_block && p->mode == LA_BLOCK_CAUSAL && p->N > 0) nblk = p->N / p->block_tokens;
+  if (!one_block && p->mode == LA_TOKEN_CAUSAL) nblk = (p->N + kCausalChunk - 1) / kCausalChunk;
+  if (heads * nblk > (long long)INT_MAX) return LA_ERR_UNSUPPORTED;
   return LA_OK;
 }
 

@@ -227,3 +227,18 @@ def test_head_dim_112_is_accepted_on_the_cuda_core_path():
     assert C.lin_attn_uses_tensor_cores(p) == 0
     assert C.lin_attn_forward(_params(D=96, rope_dt=32, rope_dh=32, rope_dw=32), Q, K, V, None,
                               O, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+
+
+def test_segment_count_limit():
+    # B * H times the segments of a head must fit an int: 2^24 heads of
+    # 256-token blocks of one token each would need 2^32 segments
+    p = _params(B=1 << 12, H=1 << 12, N=256, rope=0, mode=C.LA_BLOCK_CAUSAL, block_tokens=1)
+    assert C.lin_attn_forward(p, Q, K, V, None, O, WS, 1 << 20, None) == C.LA_ERR_UNSUPPORTED
+    p = _params(B=1 << 12, H=1 << 12, N=256 * 32, rope=0, mode=C.LA_TOKEN_CAUSAL)
+    assert C.lin_attn_forward(p, Q, K, V, None, O, WS, 1 << 20, None) == C.LA_ERR_UNSUPPORTED
+    # 2^24 heads with 64 segments each fit (2^30): past the host checks
+    # (fake pointers 2^40 bytes apart, clear of one another at this size)
+    p = _params(B=1 << 12, H=1 << 12, N=64, rope=0, mode=C.LA_BLOCK_CAUSAL, block_tokens=1)
+    far = [i << 40 for i in range(1, 6)]
+    assert C.lin_attn_forward(p, far[0], far[1], far[2], None, far[3], far[4], 1 << 20,
+                              None) not in (C.LA_ERR_UNSUPPORTED, C.LA_ERR_INVALID_ARG)
