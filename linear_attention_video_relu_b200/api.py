@@ -47,14 +47,27 @@ def _stream(stream: Optional[torch.cuda.Stream]):
     return s.cuda_stream
 
 
-def _check_io(p: C.la_params, *ts):
+_DTYPE_OF = {v: k for k, v in _DTYPES.items()}
+
+
+def _same_device(ref: torch.Tensor, *ts):
+    for t in ts:
+        if t is not None and t.device != ref.device:
+            raise ValueError("all tensors must be on %s, got one on %s" % (ref.device, t.device))
+
+
+def _check_io(p: C.la_params, *ts, require_cuda: bool = True):
+    """Contiguous CUDA tensors of shape [B, H, N, D] in the params' dtype
+    (require_cuda=False checks the rest on host tensors)."""
     for t in ts:
         if t is None:
             continue
-        if not t.is_cuda or not t.is_contiguous():
+        if (require_cuda and not t.is_cuda) or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
         if tuple(t.shape) != (p.B, p.H, p.N, p.D):
             raise ValueError("expected shape %s, got %s" % ((p.B, p.H, p.N, p.D), tuple(t.shape)))
+        if t.dtype != _DTYPE_OF[p.dtype]:
+            raise TypeError("expected dtype %s, got %s" % (_DTYPE_OF[p.dtype], t.dtype))
 
 
 class Workspace:
@@ -97,6 +110,7 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[to
     if out is None:
         out = torch.empty_like(q)
     _check_io(p, out)
+    _same_device(q, k, v, gate, out, None if workspace is None else workspace.buf)
     if workspace is None:
         workspace = workspace_for(p, q.device)
     with torch.cuda.device(q.device):
@@ -120,12 +134,10 @@ def cross_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     pk = make_params(B, H, M, D, q.dtype, eps=eps)
     _check_io(p, q, gate)
     _check_io(pk, k, v)
-    for t in (k, v, gate):
-        if t is not None and t.dtype != q.dtype:
-            raise TypeError("q, k, v and gate must share one dtype")
     if out is None:
         out = torch.empty_like(q)
     _check_io(p, out)
+    _same_device(q, k, v, gate, out, None if workspace is None else workspace.buf)
     if workspace is None:
         with torch.cuda.device(q.device):
             workspace = Workspace(C.lin_attn_cross_workspace_size(p, M), q.device)
@@ -153,7 +165,8 @@ class BlockState:
             C.check(C.lin_attn_state_reset(self._st, _stream(stream)), "lin_attn_state_reset")
 
     def _workspace(self, p):
-        key = (p.N, p.D, p.dtype, p.rope, p.grid_t, p.grid_h, p.grid_w)
+        key = (p.N, p.D, p.dtype, p.rope, p.grid_t, p.grid_h, p.grid_w, p.rope_dt, p.rope_dh,
+               p.rope_dw)
         ws = self._ws.get(key)
         if ws is None:
             ws = workspace_for(p, self.S.device, block_step=True)
@@ -169,6 +182,8 @@ class BlockState:
         _check_io(p, q, k, v, gate)
         if out is None:
             out = torch.empty_like(q)
+        _check_io(p, out)
+        _same_device(self.S, q, k, v, gate, out)
         ws = self._workspace(p)
         with torch.cuda.device(q.device):
             C.check(C.lin_attn_block_step(p, self._st, t_offset, _ptr(q), _ptr(k), _ptr(v),
@@ -182,6 +197,7 @@ class BlockState:
         B, H, N, D = k.shape
         p = make_params(B, H, N, D, k.dtype, "bidirectional", 0, grid, rope_split, theta, 1e-6)
         _check_io(p, k, v)
+        _same_device(self.S, k, v)
         ws = self._workspace(p)
         with torch.cuda.device(k.device):
             C.check(C.lin_attn_state_update(p, self._st, t_offset, _ptr(k), _ptr(v), ws.ptr,
@@ -228,6 +244,7 @@ def temporal_conv(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Te
         if tuple(t.shape) != shape or t.dtype != dt:
             raise ValueError("%s must be %s %s, got %s %s" % (what, shape, dt, tuple(t.shape),
                                                             t.dtype))
+    _same_device(x, out, weight, bias, cache_in, cache_out)
     with torch.cuda.device(x.device):
         C.check(C.lin_attn_temporal_conv(B, T, S, nc, _DTYPES[x.dtype], _ptr(x), _ptr(weight),
                                          _ptr(bias), _ptr(cache_in), _ptr(out), _ptr(cache_out),
