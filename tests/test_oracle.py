@@ -399,3 +399,16 @@ def test_cross_closed_forms():
     np.testing.assert_allclose(out[rows], np.broadcast_to(v[0, 0, 0], out[rows].shape), rtol=1e-12)
     # queries with no positive entry give exactly zero
     assert np.array_equal(oracle.cross_forward(-np.abs(q), k, v), np.zeros_like(q))
+
+
+def test_cross_golden_worked_example():
+    # tests/golden/cross_attention_worked.txt: 2 queries, 3 keys, D = 2
+    g = _read_golden("cross_attention_worked.txt")
+    arr = lambda key, *shape: np.array([float(x) for x in g[key]]).reshape(shape)
+    q, k, v = arr("q", 1, 1, 2, 2), arr("k", 1, 1, 3, 2), arr("v", 1, 1, 3, 2)
+    num, den = arr("num", 2, 2), arr("den", 2)
+    out = oracle.cross_forward(q, k, v, eps=1e-6)
+    np.testing.assert_allclose(out[0, 0], num / (den[:, None] + 1e-6), rtol=1e-15, atol=0)
+    # a zero gate halves it exactly
+    half = oracle.cross_forward(q, k, v, g=np.zeros_like(q), eps=1e-6)
+    assert np.array_equal(half, out / 2)

@@ -65,7 +65,8 @@ def test_tconv_pins_reject_mutant(name, monkeypatch):
     monkeypatch.setattr(tconv, "temporal_conv", mutant)
     calls = [pins.test_hand_worked_case, pins.test_matches_scipy_correlation,
              pins.test_zero_initialised_conv_is_the_identity, pins.test_blocks_versus_whole_sequence,
-             pins.test_causality_across_blocks, pins.test_channels_and_positions_are_independent]
+             pins.test_causality_across_blocks, pins.test_channels_and_positions_are_independent,
+             pins.test_golden_two_block_chain]
     calls += [lambda T=T, c=c, b=b: pins.test_matches_loops(T, c, b)
               for T in (1, 2, 5) for c, b in ((False, False), (True, False), (True, True))]
     assert _any_fails(calls), name + " passed every pin"
@@ -94,7 +95,7 @@ def test_cross_pins_reject_mutant(name, monkeypatch):
     monkeypatch.setattr(oracle, "cross_forward", mutant)
     calls = [pins.test_cross_matches_bruteforce_with_gate,
              pins.test_cross_with_equal_lengths_is_the_self_attention_oracle,
-             pins.test_cross_closed_forms]
+             pins.test_cross_closed_forms, pins.test_cross_golden_worked_example]
     assert _any_fails(calls), name + " passed every pin"
 
 

@@ -109,3 +109,22 @@ def test_channels_and_positions_are_independent():
     assert np.array_equal(ys, y[..., sel])
     ys, _ = tconv.temporal_conv(x[:, :, 2:4], w, bias, cache[:, 2:4])
     assert np.array_equal(ys, y[:, :, 2:4])
+
+
+def test_golden_two_block_chain():
+    # tests/golden/temporal_conv_worked.txt: a hand-worked chain of two blocks
+    import os
+    rows = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", "temporal_conv_worked.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, *vals = line.split()
+                rows[key] = np.array([float(x) for x in vals])
+    w = np.stack([rows["w0"], rows["w1"], rows["w2"]])
+    cache = rows["cache"].reshape(1, 1, 2)
+    for blk in ("block1", "block2"):
+        x = rows[blk + ".x"].reshape(1, -1, 1, 2)
+        y, cache = tconv.temporal_conv(x, w, rows["bias"], cache)
+        assert y.ravel().tolist() == rows[blk + ".y"].tolist()
+        assert cache.ravel().tolist() == rows[blk + ".cache"].tolist()
