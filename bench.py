@@ -553,6 +553,41 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+# the SANA-Video 2B model's attention shape: 20 heads of 112 at 480p
+W_2B_480P = workloads.Workload("480p_2b_d112", B=1, H=20, N=21 * 30 * 52, D=112, dtype="bf16",
+                               seed=2004, grid=(21, 30, 52), rope_split=(16, 48, 48))
+
+
+def secondary_lines(K, device, peak, peak_kind):
+    """The other workloads and rows, each timed on its own; a line that fails
+    records its error instead of ending the run."""
+    jobs = []
+    for name, mode in (("480p_block_causal", "block_causal"), ("720p_long", "bidirectional"),
+                       ("720p_long", "block_causal"), ("gated_d128", "bidirectional"),
+                       ("480p_bidir", "token_causal")):
+        ww = workloads.WORKLOADS[name]
+        jobs.append((name + "/" + mode,
+                     lambda ww=ww, mode=mode: measure_workload(ww, mode, K, 3, None, device, peak,
+                                                               peak_kind, ww.seed)))
+    jobs.append(("480p_2b_d112/bidirectional",
+                 lambda: measure_workload(W_2B_480P, "bidirectional", K, 3, None, device, peak,
+                                          peak_kind, W_2B_480P.seed)))
+    jobs.append(("480p_bidir_x_text300/cross",
+                 lambda: measure_cross(workloads.WORKLOADS["480p_bidir"], 300, K, 5, device,
+                                       peak, 2002)))
+    jobs.append(("480p_hidden_tconv", lambda: measure_tconv(K, 5, device, peak, 2003)))
+    jobs.append(("720p_long_block_step",
+                 lambda: measure_block_steps(workloads.WORKLOADS["720p_long"], 120, 60, device,
+                                             peak, peak_kind, 1004)))
+    out = []
+    for name, job in jobs:
+        try:
+            out.append(job())
+        except Exception as e:   # reported in the line, not swallowed
+            out.append({"workload": name, "error": "%s: %s" % (type(e).__name__, e)})
+    return out
+
+
 def config_of(w, mode, world):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "mode": mode,
             "grid": list(w.grid) if w.grid else None,
@@ -633,20 +668,7 @@ def main():
     if rank == 0 and args.e2e_steps > 0:
         line["e2e"] = measure_e2e(w, args.e2e_steps, device, w.seed)
     if not args.no_extra and rank == 0:
-        extra = []
-        K = max(20, args.steps // 5)
-        for name, mode in (("480p_block_causal", "block_causal"), ("720p_long", "bidirectional"),
-                           ("720p_long", "block_causal"), ("gated_d128", "bidirectional"),
-                           ("480p_bidir", "token_causal")):
-            ww = workloads.WORKLOADS[name]
-            extra.append(measure_workload(ww, mode, K, 3, None, device, peak, peak_kind,
-                                          ww.seed))
-        extra.append(measure_cross(workloads.WORKLOADS["480p_bidir"], 300, K, 5, device, peak,
-                                   2002))
-        extra.append(measure_tconv(K, 5, device, peak, 2003))
-        extra.append(measure_block_steps(workloads.WORKLOADS["720p_long"], 120, 60, device, peak,
-                                         peak_kind, 1004))
-        line["also"] = extra
+        line["also"] = secondary_lines(max(20, args.steps // 5), device, peak, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

@@ -119,3 +119,25 @@ def test_committed_profiles_name_their_command():
         text = open(os.path.join(pdir, n)).read()
         assert "ncu " in text and "bench.py" in text, n
         assert len(text) < 8192, n
+
+
+def test_secondary_lines_record_errors(monkeypatch):
+    # a failing secondary line is reported with its error; the others still run
+    calls = []
+
+    def ok(*a, **k):
+        calls.append(a[0] if a else None)
+        return {"workload": "ok"}
+
+    def boom(*a, **k):
+        raise RuntimeError("device status after timing: bounded wait gave up")
+
+    monkeypatch.setattr(bench, "measure_workload", ok)
+    monkeypatch.setattr(bench, "measure_cross", boom)
+    monkeypatch.setattr(bench, "measure_tconv", ok)
+    monkeypatch.setattr(bench, "measure_block_steps", ok)
+    lines = bench.secondary_lines(20, None, 6535.7, "measured")
+    errs = [l for l in lines if "error" in l]
+    assert len(errs) == 1 and errs[0]["workload"] == "480p_bidir_x_text300/cross"
+    assert "bounded wait" in errs[0]["error"]
+    assert len(lines) == 9 and sum(1 for l in lines if l == {"workload": "ok"}) == 8
