@@ -91,12 +91,12 @@ __host__ __device__ inline int cta_of_unit(const Sched& s, long long u) {
 }
 
 // cta_of_unit with one multiply-shift when U * G < 2^31.
-__device__ __forceinline__ int cta_of_unit_fast(const Sched& s, long long u) {
+__host__ __device__ __forceinline__ int cta_of_unit_fast(const Sched& s, long long u) {
   return s.fastU ? fdiv(s.divU, (int)((u + 1) * s.G - 1)) : cta_of_unit(s, u);
 }
 
 // Number of CTAs (= partial slots) that hold tiles of segment seg.
-__device__ __forceinline__ int parts_of(const Sched& s, int seg) {
+__host__ __device__ __forceinline__ int parts_of(const Sched& s, int seg) {
   const long long ub = (long long)seg * s.tps;
   return cta_of_unit_fast(s, ub + s.tps - 1) - cta_of_unit_fast(s, ub) + 1;
 }
