@@ -82,8 +82,10 @@ typedef enum { LA_BIDIRECTIONAL = 0, LA_BLOCK_CAUSAL = 1, LA_TOKEN_CAUSAL = 2 } 
 typedef struct {
   int B, H, N, D;        /* batch, heads, tokens per head, head dim.
                             D in {32, 64, 112, 128} (112: the SANA-Video 2B
-                            head dim, on the CUDA-core kernels); N >= 0
-                            (N = 0: no work). */
+                            head dim; bf16 forwards run it on the 128-wide
+                            tensor-core kernels with zero padding, block steps
+                            on the CUDA-core kernels); N >= 0 (N = 0: no
+                            work). */
   la_dtype dtype;        /* dtype of q, k, v, gate and out */
   la_mode mode;          /* bidirectional, block-causal or token-causal */
   int block_tokens;      /* block-causal: tokens per block, N % block_tokens == 0.

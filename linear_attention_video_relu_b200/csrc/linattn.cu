@@ -106,6 +106,9 @@ la_status check_params(const la_params* p, bool one_block) {
 
 bool want_tc(const la_params* p, bool one_block) {
   if (!one_block && p->mode == LA_TOKEN_CAUSAL) return false;   // CUDA-core kernels only
+  // 112-wide heads run padded on the 128 kernels, whose carried-state I/O is
+  // 128 wide: block steps at D = 112 stay on the CUDA-core kernels
+  if (one_block && p->D == 112) return false;
   const int entries = p->rope ? p->grid_t * rope_stride(p->rope_dt / 2) +
                                     p->grid_h * rope_stride(p->rope_dh / 2) +
                                     p->grid_w * rope_stride(p->rope_dw / 2)
@@ -169,7 +172,8 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   sc.nblk = (N + sc.L - 1) / sc.L;
   if (sc.nblk < 1) sc.nblk = 1;
   sc.nseg = (int)(pl->heads * sc.nblk);
-  sc.TT = pl->tc ? tc_state_tile(p->D) : kSimtTileState;
+  const int Dk = pl->tc ? tc_kernel_dim(p->D) : p->D;   // head dim the kernels run at
+  sc.TT = pl->tc ? tc_state_tile(Dk) : kSimtTileState;
   sc.tps = (sc.L + sc.TT - 1) / sc.TT;
   sc.U = (long long)sc.nseg * sc.tps;
   long long G = pl->tc ? (long long)sms * tc_state_ctas_per_sm(p->D) : 2LL * sms;
@@ -190,7 +194,7 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   pl->lq = sc.L;
   pl->apply_tps = (sc.L + kSimtTileApply - 1) / kSimtTileApply;
 
-  const size_t dd1 = (size_t)p->D * (p->D + 1);
+  const size_t dd1 = (size_t)Dk * (Dk + 1);
   size_t off = 0;
   pl->off_flag = off;                     // control block: flag word, then counters
   off += LA_WORKSPACE_CONTROL_BYTES;
@@ -199,7 +203,7 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   pl->off_part = off;
   off += round_up((size_t)sc.nseg * sc.maxc * dd1 * sizeof(float), kAlign);
   pl->off_apply = off;   // fp32 apply states (SIMT) or B-operand images (tensor cores)
-  const size_t per_seg = pl->tc ? (size_t)image_bytes(p->D) : dd1 * sizeof(float);
+  const size_t per_seg = pl->tc ? (size_t)image_bytes(Dk) : dd1 * sizeof(float);
   off += round_up((size_t)sc.nseg * per_seg, kAlign);
   pl->total = off;
   return LA_OK;

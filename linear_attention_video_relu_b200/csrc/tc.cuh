@@ -41,7 +41,7 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 enum : int { kFlagStateTimeout = 1, kFlagApplyTimeout = 2 };
 
 struct TcArgs {
-  int D;
+  int D;           // I/O head dim (64, 112 or 128; 112 runs on the 128 kernels)
   long long N;
   int Lq;          // query rows per segment: sc.L, or the query length of a cross-attention
   Rope rope;
@@ -177,11 +177,17 @@ inline int pick_apply_stages(int D, int entries, int gate) {
 // Which calls take the tensor-core kernels: bf16 I/O, D in {64, 128}, and RoPE
 // widths that are multiples of 8 (a 16-byte chunk never spans two axes), with
 // both kernels' shared memory within budget (gated or not).
+// Head dim the tensor-core kernels run at for an I/O head dim: 112-wide rows
+// run on the 128 kernels, the tensor maps reading columns 112..127 as zero
+// fill and the apply kernel storing only the first 112 columns.
+inline int tc_kernel_dim(int D) { return D == 112 ? 128 : D; }
+
 inline bool tc_supported(bool bf16, int D, int rope, int dt, int dh, int dw, int entries) {
-  if (!bf16 || (D != 64 && D != 128)) return false;
+  if (!bf16 || (D != 64 && D != 112 && D != 128)) return false;
   if (rope && ((dt % 8) || (dh % 8) || (dw % 8))) return false;
   int e = rope ? entries : 0;
-  return pick_state_stages(D, e) > 0 && pick_apply_stages(D, e, 1) > 0;
+  const int Dk = tc_kernel_dim(D);
+  return pick_state_stages(Dk, e) > 0 && pick_apply_stages(Dk, e, 1) > 0;
 }
 
 // ---- device helpers ------------------------------------------------------------
@@ -298,6 +304,13 @@ __device__ __forceinline__ ChunkCol chunk_col(const Rope& r, int chunk) {
   const int p0 = 4 * chunk;
   c.ax = p0 < r.pair_base[1] ? 0 : (p0 < r.pair_base[2] ? 1 : 2);
   c.pair_off = p0 - (c.ax == 0 ? 0 : (c.ax == 1 ? r.pair_base[1] : r.pair_base[2]));
+  // padding columns past the last rotary pair (a 112-wide head on the 128
+  // kernels) hold zeros: any finite cos/sin leaves them zero, so they read
+  // the first entries of the t axis
+  if (p0 >= r.pair_base[2] + r.half[2]) {
+    c.ax = 0;
+    c.pair_off = 0;
+  }
   return c;
 }
 
@@ -977,7 +990,7 @@ __host__ __device__ constexpr uint32_t tmem_cols_pow2(uint32_t n) {
 template <int D, bool ROPE, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
-         const __grid_constant__ CUtensorMap tm_o, __nv_bfloat16* __restrict__ out,
+         const __grid_constant__ CUtensorMap tm_o, __nv_bfloat16* __restrict__ out, int ocols,
          const __grid_constant__ Rope rope, int L, int nblk,
          long long U, int stages, int sbuf, int gst, const uint8_t* __restrict__ images,
          const float2* __restrict__ gtab, float eps, int* flag) {
@@ -1245,7 +1258,8 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       if (ready && gready && (!DIRECT || r < L)) {
         const float inv = 1.f / (eps + (__uint_as_float(dz[0]) + __uint_as_float(dz[1])));
         const uint64_t inv2 = ptx::f2(inv, inv);
-        uint4* dst = reinterpret_cast<uint4*>(out + ((long long)seg * L + r) * D + col0);
+        // rows of ocols values: D, or 112 for a 112-wide head on the 128 kernels
+        uint4* dst = reinterpret_cast<uint4*>(out + ((long long)seg * L + r) * ocols + col0);
         const uint32_t gt = gbase + (DIRECT ? gs : s) * TILE_BYTES;
         const int h = col0 / 64;
 #pragma unroll
@@ -1270,8 +1284,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           }
           const uint4 ov = make_uint4(ptx::pack_bf16x2(o[0], o[1]), ptx::pack_bf16x2(o[2], o[3]),
                                       ptx::pack_bf16x2(o[4], o[5]), ptx::pack_bf16x2(o[6], o[7]));
-          if (DIRECT) dst[k4] = ov;
-          else ptx::st_shared_v4(base + s * TILE_BYTES + off, ov);
+          if (DIRECT) {
+            if (col0 + 8 * k4 < ocols) dst[k4] = ov;
+          } else {
+            ptx::st_shared_v4(base + s * TILE_BYTES + off, ov);
+          }
         }
       }
       ptx::tc_fence_before();
@@ -1438,8 +1455,9 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   const int entries = a.rope.on ? a.rope.entries : 0;
   const Sched& sc = a.sc;
   CUtensorMap mk, mv, mq, mg, mo;
-  if (!make_map(&mk, a.k, D, sc.L, sc.nseg, tc_state_tile_c(D)) ||
-      !make_map(&mv, a.v, D, sc.L, sc.nseg, tc_state_tile_c(D)))
+  // tensor maps over the I/O rows (a.D wide); columns past a.D read as zeros
+  if (!make_map(&mk, a.k, a.D, sc.L, sc.nseg, tc_state_tile_c(D)) ||
+      !make_map(&mv, a.v, a.D, sc.L, sc.nseg, tc_state_tile_c(D)))
     return LA_ERR_CUDA;
   la_status st;
   const int s1 = pick_state_stages(D, entries);
@@ -1465,9 +1483,9 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   if (!a.do_apply) return LA_OK;
 
   const bool gate = a.g != nullptr;
-  if (!make_map(&mq, a.q, D, a.Lq, sc.nseg, kApplyTile) ||
-      !make_map(&mo, a.out, D, a.Lq, sc.nseg, kApplyTile) ||
-      !make_map(&mg, gate ? a.g : a.q, D, a.Lq, sc.nseg, kApplyTile))
+  if (!make_map(&mq, a.q, a.D, a.Lq, sc.nseg, kApplyTile) ||
+      !make_map(&mo, a.out, a.D, a.Lq, sc.nseg, kApplyTile) ||
+      !make_map(&mg, gate ? a.g : a.q, a.D, a.Lq, sc.nseg, kApplyTile))
     return LA_ERR_CUDA;
   int s3 = 0, sb3 = 1, gs3 = 0;
   pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3, &gs3);
@@ -1478,7 +1496,8 @@ la_status tc_run_d(const TcArgs& a, int sms) {
                       : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
   if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
   st = launch_pdl(k3, dim3(G3), dim3(kTcThreadsApply), p3.total, a.stream, mq, mg, mo,
-                  static_cast<__nv_bfloat16*>(a.out), a.rope, a.Lq, sc.nblk, U3, s3, sb3, gs3,
+                  static_cast<__nv_bfloat16*>(a.out), a.D, a.rope, a.Lq, sc.nblk, U3, s3, sb3,
+                  gs3,
                   reinterpret_cast<const uint8_t*>(a.apply), (const float2*)a.gtab, a.eps,
                   a.flag);
   if (st != LA_OK) return st;
@@ -1487,7 +1506,7 @@ la_status tc_run_d(const TcArgs& a, int sms) {
 
 inline la_status tc_run(const TcArgs& a, int sms) {
   if (a.D == 64) return tc_run_d<64>(a, sms);
-  if (a.D == 128) return tc_run_d<128>(a, sms);
+  if (a.D == 112 || a.D == 128) return tc_run_d<128>(a, sms);
   return LA_ERR_UNSUPPORTED;
 }
 
