@@ -47,6 +47,7 @@ struct Plan {
   int lq;              // query rows per segment (sc.L, or nq for a cross-attention)
   int apply_tps;       // SIMT apply: tiles per segment
   int sms;             // SM count of the device
+  Layout lay;          // memory order of q, k, v, gate, out
   size_t off_flag, off_tab, off_part, off_apply, total;
 };
 
@@ -74,6 +75,7 @@ la_status check_params(const la_params* p, bool one_block) {
   if (p->B < 0 || p->H < 0 || p->N < 0) return LA_ERR_INVALID_ARG;
   if (p->D != 32 && p->D != 64 && p->D != 112 && p->D != 128) return LA_ERR_INVALID_ARG;
   if (p->dtype != LA_F32 && p->dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+  if (p->layout != LA_LAYOUT_BHND && p->layout != LA_LAYOUT_BNHD) return LA_ERR_INVALID_ARG;
   if (!one_block) {
     if (p->mode != LA_BIDIRECTIONAL && p->mode != LA_BLOCK_CAUSAL && p->mode != LA_TOKEN_CAUSAL)
       return LA_ERR_INVALID_ARG;
@@ -129,6 +131,9 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   pl->tc = want_tc(p, one_block);
   pl->sms = sms;
   pl->heads = (long long)p->B * p->H;
+  pl->lay.bnhd = p->layout == LA_LAYOUT_BNHD ? 1 : 0;
+  pl->lay.H = p->H > 0 ? p->H : 1;
+  pl->lay.div_h = make_fastdiv(pl->lay.H);
 
   Rope& r = pl->rope;
   r.on = p->rope ? 1 : 0;
@@ -268,7 +273,8 @@ la_status run_simt(const Launch& L) {
   if (st != LA_OK) return st;
   if ((st = mark(L, 0)) != LA_OK) return st;
   state_partial_simt<D, T><<<pl.sc.G, kSimtThreads, smem1, L.stream>>>(
-      static_cast<const T*>(L.k), static_cast<const T*>(L.v), N, pl.rope, pl.sc, part, gtab);
+      static_cast<const T*>(L.k), static_cast<const T*>(L.v), N, pl.lay, pl.rope, pl.sc, part,
+      gtab);
   if ((st = last_error()) != LA_OK) return st;
   if ((st = mark(L, 1)) != LA_OK) return st;
   dim3 g2((D * (D + 1) + 255) / 256, (unsigned)(pl.heads < 65535 ? pl.heads : 65535));
@@ -285,7 +291,7 @@ la_status run_simt(const Launch& L) {
     const int gc = pl.sc.nseg < (1 << 20) ? pl.sc.nseg : (1 << 20);
     apply_causal_simt<D, T><<<gc, kSimtThreads, smemc, L.stream>>>(
         static_cast<const T*>(L.q), static_cast<const T*>(L.k), static_cast<const T*>(L.v),
-        static_cast<const T*>(L.g), static_cast<T*>(L.out), N, pl.rope, pl.sc.nblk,
+        static_cast<const T*>(L.g), static_cast<T*>(L.out), N, pl.lay, pl.rope, pl.sc.nblk,
         pl.sc.nseg, apply, gtab, L.p->eps);
     if ((st = last_error()) != LA_OK) return st;
     return mark(L, 3);
@@ -297,7 +303,7 @@ la_status run_simt(const Launch& L) {
   dim3 g3(pl.apply_tps, pl.sc.nseg < 65535 ? pl.sc.nseg : 65535);
   apply_simt<D, T><<<g3, kSimtThreads, smem3, L.stream>>>(
       static_cast<const T*>(L.q), static_cast<const T*>(L.g), static_cast<T*>(L.out), pl.nq,
-      pl.rope, pl.lq, pl.sc.nblk, pl.apply_tps, pl.sc.nseg, apply, gtab, L.p->eps);
+      pl.lay, pl.rope, pl.lq, pl.sc.nblk, pl.apply_tps, pl.sc.nseg, apply, gtab, L.p->eps);
   if ((st = last_error()) != LA_OK) return st;
   return mark(L, 3);
 }
@@ -329,6 +335,8 @@ la_status run(const Launch& L) {
     a.out = L.out;
     a.flag = reinterpret_cast<int*>(L.ws + L.pl->off_flag);
     a.counters = reinterpret_cast<int*>(L.ws + L.pl->off_flag + kCounterOffset);
+    a.bnhd = L.pl->lay.bnhd;
+    a.H = L.pl->lay.H;
     a.fused = L.pl->sc.nblk == 1 && L.pl->sc.nseg <= kMaxCounters;
     a.gtab = reinterpret_cast<float2*>(L.ws + L.pl->off_tab);
     a.part = reinterpret_cast<float*>(L.ws + L.pl->off_part);

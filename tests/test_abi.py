@@ -245,3 +245,13 @@ def test_segment_count_limit():
     far = [i << 40 for i in range(1, 6)]
     assert C.lin_attn_forward(p, far[0], far[1], far[2], None, far[3], far[4], 1 << 20,
                               None) not in (C.LA_ERR_UNSUPPORTED, C.LA_ERR_INVALID_ARG)
+
+
+def test_layout_field():
+    # [B,N,H,D] passes the host checks; anything else but the two orders is refused
+    p = _params(layout=C.LA_LAYOUT_BNHD)
+    assert C.lin_attn_forward(p, Q, K, V, None, O, WS, 1 << 20, None) != C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_forward(_params(layout=2), Q, K, V, None, O, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=16, rope_dh=24, rope_dw=24,
+                                                layout=C.LA_LAYOUT_BNHD)) == 1
