@@ -32,8 +32,8 @@
  *   - Memory. The caller owns all device memory (inputs, output, state,
  *     workspace); the library allocates and frees nothing and keeps no global
  *     mutable state, so calls are re-entrant.
- *   - Layout. q, k, v, gate, out are contiguous [B, H, N, D] with D innermost,
- *     in the I/O dtype. The state is fp32: S [B, H, D, D] with
+ *   - Layout. q, k, v, gate, out are contiguous [B, H, N, D] (or [B, N, H, D]
+ *     with p->layout = LA_LAYOUT_BNHD) with D innermost, in the I/O dtype. The state is fp32: S [B, H, D, D] with
  *     S[a][c] = sum_j RoPE(phi(k_j))_a v_j,c, and z [B, H, D].
  *   - Asynchrony. A call checks its arguments on the host, enqueues kernels on
  *     `stream` (a cudaStream_t passed as void*, NULL = legacy default stream)
@@ -79,11 +79,18 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;   /* I/O dtype; state is fp32
 
 typedef enum { LA_BIDIRECTIONAL = 0, LA_BLOCK_CAUSAL = 1, LA_TOKEN_CAUSAL = 2 } la_mode;
 
+/* Memory order of q, k, v, gate and out (D innermost either way). BNHD is
+ * the order a fused QKV projection of [B, N, C] hidden states writes its
+ * heads in, so the op reads it without a transpose. */
+typedef enum { LA_LAYOUT_BHND = 0, LA_LAYOUT_BNHD = 1 } la_layout;
+
 typedef struct {
   int B, H, N, D;        /* batch, heads, tokens per head, head dim.
                             D in {32, 64, 112, 128} (112: the SANA-Video 2B
-                            head dim, on the CUDA-core kernels); N >= 0
-                            (N = 0: no work). */
+                            head dim; bf16 forwards run it on the 128-wide
+                            tensor-core kernels with zero padding, block steps
+                            on the CUDA-core kernels); N >= 0 (N = 0: no
+                            work). */
   la_dtype dtype;        /* dtype of q, k, v, gate and out */
   la_mode mode;          /* bidirectional, block-causal or token-causal */
   int block_tokens;      /* block-causal: tokens per block, N % block_tokens == 0.
@@ -94,6 +101,10 @@ typedef struct {
   int rope_dt, rope_dh, rope_dw;  /* even widths with sum D (t, h, w order) */
   double rope_theta;     /* RoPE base, > 0 (10000 in the workloads here) */
   float eps;             /* added to the denominator, >= 0 (1e-6 here) */
+  la_layout layout;      /* LA_LAYOUT_BHND ([B,H,N,D], zero) or LA_LAYOUT_BNHD
+                            ([B,N,H,D]); every tensor of the call uses it, and
+                            a block step's q, k, v, gate, out are [B,N,H,D]
+                            with N the block's tokens */
 } la_params;
 
 /* A carried block-causal state: caller-owned device memory, fp32,

@@ -23,6 +23,8 @@ LA_WORKSPACE_CONTROL_BYTES = 65536   # control block at the start of a workspace
 
 LA_F32 = 0
 LA_BF16 = 1
+LA_LAYOUT_BHND = 0
+LA_LAYOUT_BNHD = 1
 LA_BIDIRECTIONAL = 0
 LA_BLOCK_CAUSAL = 1
 LA_TOKEN_CAUSAL = 2
@@ -35,7 +37,7 @@ class la_params(ctypes.Structure):
         ("rope", ctypes.c_int),
         ("grid_t", ctypes.c_int), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
         ("rope_dt", ctypes.c_int), ("rope_dh", ctypes.c_int), ("rope_dw", ctypes.c_int),
-        ("rope_theta", ctypes.c_double), ("eps", ctypes.c_float),
+        ("rope_theta", ctypes.c_double), ("eps", ctypes.c_float), ("layout", ctypes.c_int),
     ]
 
 

@@ -2,8 +2,8 @@
 
 PyTorch provides device memory and streams only; the computation is the
 CUDA library's. Shapes follow include/linattn.h: q, k, v, gate, out are
-contiguous [B, H, N, D] in bf16 or fp32; the carried state is fp32
-S [B, H, D, D] and z [B, H, D].
+contiguous [B, H, N, D] (layout="bhnd") or [B, N, H, D] (layout="bnhd") in
+bf16 or fp32; the carried state is fp32 S [B, H, D, D] and z [B, H, D].
 """
 from __future__ import annotations
 
@@ -16,12 +16,23 @@ from . import _native as C
 _DTYPES = {torch.bfloat16: C.LA_BF16, torch.float32: C.LA_F32}
 _MODES = {"bidirectional": C.LA_BIDIRECTIONAL, "block_causal": C.LA_BLOCK_CAUSAL,
           "token_causal": C.LA_TOKEN_CAUSAL}
+_LAYOUTS = {"bhnd": C.LA_LAYOUT_BHND, "bnhd": C.LA_LAYOUT_BNHD}
+
+
+def _dims(t: torch.Tensor, layout: str):
+    """(B, H, N, D) of a [B, H, N, D] or [B, N, H, D] tensor."""
+    if layout not in _LAYOUTS:
+        raise ValueError("layout must be 'bhnd' or 'bnhd'")
+    if t.dim() != 4:
+        raise ValueError("expected a 4D tensor, got shape %s" % (tuple(t.shape),))
+    a, b, c, d = (int(x) for x in t.shape)
+    return (a, b, c, d) if layout == "bhnd" else (a, c, b, d)
 
 
 def make_params(B: int, H: int, N: int, D: int, dtype: torch.dtype, mode: str = "bidirectional",
                 block_tokens: int = 0, grid: Optional[Sequence[int]] = None,
                 rope_split: Optional[Sequence[int]] = None, theta: float = 10000.0,
-                eps: float = 1e-6) -> C.la_params:
+                eps: float = 1e-6, layout: str = "bhnd") -> C.la_params:
     p = C.la_params()
     p.B, p.H, p.N, p.D = B, H, N, D
     if dtype not in _DTYPES:
@@ -35,6 +46,9 @@ def make_params(B: int, H: int, N: int, D: int, dtype: torch.dtype, mode: str = 
         p.rope_dt, p.rope_dh, p.rope_dw = (int(x) for x in rope_split)
     p.rope_theta = float(theta)
     p.eps = float(eps)
+    if layout not in _LAYOUTS:
+        raise ValueError("layout must be 'bhnd' or 'bnhd'")
+    p.layout = _LAYOUTS[layout]
     return p
 
 
@@ -57,15 +71,16 @@ def _same_device(ref: torch.Tensor, *ts):
 
 
 def _check_io(p: C.la_params, *ts, require_cuda: bool = True):
-    """Contiguous CUDA tensors of shape [B, H, N, D] in the params' dtype
-    (require_cuda=False checks the rest on host tensors)."""
+    """Contiguous CUDA tensors of shape [B, H, N, D] (or [B, N, H, D]) in the
+    params' dtype (require_cuda=False checks the rest on host tensors)."""
+    shape = ((p.B, p.H, p.N, p.D) if p.layout == C.LA_LAYOUT_BHND else (p.B, p.N, p.H, p.D))
     for t in ts:
         if t is None:
             continue
         if (require_cuda and not t.is_cuda) or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
-        if tuple(t.shape) != (p.B, p.H, p.N, p.D):
-            raise ValueError("expected shape %s, got %s" % ((p.B, p.H, p.N, p.D), tuple(t.shape)))
+        if tuple(t.shape) != shape:
+            raise ValueError("expected shape %s, got %s" % (shape, tuple(t.shape)))
         if t.dtype != _DTYPE_OF[p.dtype]:
             raise TypeError("expected dtype %s, got %s" % (_DTYPE_OF[p.dtype], t.dtype))
 
@@ -102,10 +117,13 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[to
             *, mode: str = "bidirectional", block_tokens: int = 0,
             grid: Optional[Sequence[int]] = None, rope_split: Optional[Sequence[int]] = None,
             theta: float = 10000.0, eps: float = 1e-6, out: Optional[torch.Tensor] = None,
-            workspace: Optional[Workspace] = None, stream=None) -> torch.Tensor:
-    """out = RoPE(phi q) S / (phi q . z + eps) [* sigmoid(gate)] over [B, H, N, D]."""
-    B, H, N, D = q.shape
-    p = make_params(B, H, N, D, q.dtype, mode, block_tokens, grid, rope_split, theta, eps)
+            workspace: Optional[Workspace] = None, stream=None,
+            layout: str = "bhnd") -> torch.Tensor:
+    """out = RoPE(phi q) S / (phi q . z + eps) [* sigmoid(gate)] over [B, H, N, D]
+    tensors (or [B, N, H, D] ones with layout="bnhd")."""
+    B, H, N, D = _dims(q, layout)
+    p = make_params(B, H, N, D, q.dtype, mode, block_tokens, grid, rope_split, theta, eps,
+                    layout)
     _check_io(p, q, k, v, gate)
     if out is None:
         out = torch.empty_like(q)
@@ -123,15 +141,16 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[to
 def cross_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                   gate: Optional[torch.Tensor] = None, *, eps: float = 1e-6,
                   out: Optional[torch.Tensor] = None, workspace: Optional[Workspace] = None,
-                  stream=None) -> torch.Tensor:
+                  stream=None, layout: str = "bhnd") -> torch.Tensor:
     """Linear cross-attention: q, gate, out [B, H, N, D] read the state of
-    k, v [B, H, M, D] (no RoPE; every query sees every key)."""
-    B, H, N, D = q.shape
-    if k.dim() != 4 or tuple(k.shape[:2]) != (B, H) or k.shape[3] != D:
-        raise ValueError("k must be [B, H, M, D] with q's B, H, D; got %s" % (tuple(k.shape),))
-    M = int(k.shape[2])
-    p = make_params(B, H, N, D, q.dtype, eps=eps)
-    pk = make_params(B, H, M, D, q.dtype, eps=eps)
+    k, v [B, H, M, D] (no RoPE; every query sees every key); [B, N, H, D] and
+    [B, M, H, D] with layout="bnhd"."""
+    B, H, N, D = _dims(q, layout)
+    kB, kH, M, kD = _dims(k, layout)
+    if (kB, kH, kD) != (B, H, D):
+        raise ValueError("k must have q's B, H and D; got shape %s" % (tuple(k.shape),))
+    p = make_params(B, H, N, D, q.dtype, eps=eps, layout=layout)
+    pk = make_params(B, H, M, D, q.dtype, eps=eps, layout=layout)
     _check_io(p, q, gate)
     _check_io(pk, k, v)
     if out is None:
@@ -166,7 +185,7 @@ class BlockState:
 
     def _workspace(self, p):
         key = (p.N, p.D, p.dtype, p.rope, p.grid_t, p.grid_h, p.grid_w, p.rope_dt, p.rope_dh,
-               p.rope_dw)
+               p.rope_dw, p.layout)
         ws = self._ws.get(key)
         if ws is None:
             ws = workspace_for(p, self.S.device, block_step=True)
@@ -175,10 +194,11 @@ class BlockState:
 
     def step(self, q, k, v, gate=None, *, t_offset: int = 0, commit: bool = True,
              grid=None, rope_split=None, theta: float = 10000.0, eps: float = 1e-6,
-             out=None, stream=None) -> torch.Tensor:
+             out=None, stream=None, layout: str = "bhnd") -> torch.Tensor:
         """One block of block-causal attention against the carried state."""
-        B, H, N, D = q.shape
-        p = make_params(B, H, N, D, q.dtype, "bidirectional", 0, grid, rope_split, theta, eps)
+        B, H, N, D = _dims(q, layout)
+        p = make_params(B, H, N, D, q.dtype, "bidirectional", 0, grid, rope_split, theta, eps,
+                        layout)
         _check_io(p, q, k, v, gate)
         if out is None:
             out = torch.empty_like(q)
@@ -192,10 +212,11 @@ class BlockState:
         return out
 
     def update(self, k, v, *, t_offset: int = 0, grid=None, rope_split=None,
-               theta: float = 10000.0, stream=None) -> None:
+               theta: float = 10000.0, stream=None, layout: str = "bhnd") -> None:
         """Fold a block's k, v into the state without producing output."""
-        B, H, N, D = k.shape
-        p = make_params(B, H, N, D, k.dtype, "bidirectional", 0, grid, rope_split, theta, 1e-6)
+        B, H, N, D = _dims(k, layout)
+        p = make_params(B, H, N, D, k.dtype, "bidirectional", 0, grid, rope_split, theta, 1e-6,
+                        layout)
         _check_io(p, k, v)
         _same_device(self.S, k, v)
         ws = self._workspace(p)

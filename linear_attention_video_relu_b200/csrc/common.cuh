@@ -60,6 +60,27 @@ struct Rope {
   float inv_pi_lo[64];
 };
 
+// Memory order of q, k, v, gate and out: [B, H, N, D] (bnhd = 0) or
+// [B, N, H, D] (bnhd = 1, the order a fused QKV projection writes its heads
+// in), D innermost either way; head = b * H + h.
+struct Layout {
+  int bnhd;
+  int H;
+  FastDiv div_h;   // by H
+  // element offset of (head, token n, dim 0) in a tensor of N tokens per head
+  // and rows of D values
+  __host__ __device__ __forceinline__ long long row(int head, long long n, long long N,
+                                                    int D) const {
+    if (!bnhd) return ((long long)head * N + n) * D;
+    const int b = fdiv(div_h, head), h = head - b * H;
+    return (((long long)b * N + n) * H + h) * D;
+  }
+  // elements between consecutive tokens of one head
+  __host__ __device__ __forceinline__ long long tok_stride(int D) const {
+    return bnhd ? (long long)H * D : (long long)D;
+  }
+};
+
 // Work schedule of the state build. The tokens of every head are cut into
 // segments of L tokens (the whole head in bidirectional mode, one block in
 // block-causal mode); a segment is cut into tps tiles of TT tokens (the last

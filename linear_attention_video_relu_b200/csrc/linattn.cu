@@ -47,6 +47,7 @@ struct Plan {
   int lq;              // query rows per segment (sc.L, or nq for a cross-attention)
   int apply_tps;       // SIMT apply: tiles per segment
   int sms;             // SM count of the device
+  Layout lay;          // memory order of q, k, v, gate, out
   size_t off_flag, off_tab, off_part, off_apply, total;
 };
 
@@ -74,6 +75,7 @@ la_status check_params(const la_params* p, bool one_block) {
   if (p->B < 0 || p->H < 0 || p->N < 0) return LA_ERR_INVALID_ARG;
   if (p->D != 32 && p->D != 64 && p->D != 112 && p->D != 128) return LA_ERR_INVALID_ARG;
   if (p->dtype != LA_F32 && p->dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+  if (p->layout != LA_LAYOUT_BHND && p->layout != LA_LAYOUT_BNHD) return LA_ERR_INVALID_ARG;
   if (!one_block) {
     if (p->mode != LA_BIDIRECTIONAL && p->mode != LA_BLOCK_CAUSAL && p->mode != LA_TOKEN_CAUSAL)
       return LA_ERR_INVALID_ARG;
@@ -106,6 +108,9 @@ la_status check_params(const la_params* p, bool one_block) {
 
 bool want_tc(const la_params* p, bool one_block) {
   if (!one_block && p->mode == LA_TOKEN_CAUSAL) return false;   // CUDA-core kernels only
+  // 112-wide heads run padded on the 128 kernels, whose carried-state I/O is
+  // 128 wide: block steps at D = 112 stay on the CUDA-core kernels
+  if (one_block && p->D == 112) return false;
   const int entries = p->rope ? p->grid_t * rope_stride(p->rope_dt / 2) +
                                     p->grid_h * rope_stride(p->rope_dh / 2) +
                                     p->grid_w * rope_stride(p->rope_dw / 2)
@@ -126,6 +131,9 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   pl->tc = want_tc(p, one_block);
   pl->sms = sms;
   pl->heads = (long long)p->B * p->H;
+  pl->lay.bnhd = p->layout == LA_LAYOUT_BNHD ? 1 : 0;
+  pl->lay.H = p->H > 0 ? p->H : 1;
+  pl->lay.div_h = make_fastdiv(pl->lay.H);
 
   Rope& r = pl->rope;
   r.on = p->rope ? 1 : 0;
@@ -169,7 +177,8 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   sc.nblk = (N + sc.L - 1) / sc.L;
   if (sc.nblk < 1) sc.nblk = 1;
   sc.nseg = (int)(pl->heads * sc.nblk);
-  sc.TT = pl->tc ? tc_state_tile(p->D) : kSimtTileState;
+  const int Dk = pl->tc ? tc_kernel_dim(p->D) : p->D;   // head dim the kernels run at
+  sc.TT = pl->tc ? tc_state_tile(Dk) : kSimtTileState;
   sc.tps = (sc.L + sc.TT - 1) / sc.TT;
   sc.U = (long long)sc.nseg * sc.tps;
   long long G = pl->tc ? (long long)sms * tc_state_ctas_per_sm(p->D) : 2LL * sms;
@@ -190,7 +199,7 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   pl->lq = sc.L;
   pl->apply_tps = (sc.L + kSimtTileApply - 1) / kSimtTileApply;
 
-  const size_t dd1 = (size_t)p->D * (p->D + 1);
+  const size_t dd1 = (size_t)Dk * (Dk + 1);
   size_t off = 0;
   pl->off_flag = off;                     // control block: flag word, then counters
   off += LA_WORKSPACE_CONTROL_BYTES;
@@ -199,7 +208,7 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
   pl->off_part = off;
   off += round_up((size_t)sc.nseg * sc.maxc * dd1 * sizeof(float), kAlign);
   pl->off_apply = off;   // fp32 apply states (SIMT) or B-operand images (tensor cores)
-  const size_t per_seg = pl->tc ? (size_t)image_bytes(p->D) : dd1 * sizeof(float);
+  const size_t per_seg = pl->tc ? (size_t)image_bytes(Dk) : dd1 * sizeof(float);
   off += round_up((size_t)sc.nseg * per_seg, kAlign);
   pl->total = off;
   return LA_OK;
@@ -264,7 +273,8 @@ la_status run_simt(const Launch& L) {
   if (st != LA_OK) return st;
   if ((st = mark(L, 0)) != LA_OK) return st;
   state_partial_simt<D, T><<<pl.sc.G, kSimtThreads, smem1, L.stream>>>(
-      static_cast<const T*>(L.k), static_cast<const T*>(L.v), N, pl.rope, pl.sc, part, gtab);
+      static_cast<const T*>(L.k), static_cast<const T*>(L.v), N, pl.lay, pl.rope, pl.sc, part,
+      gtab);
   if ((st = last_error()) != LA_OK) return st;
   if ((st = mark(L, 1)) != LA_OK) return st;
   dim3 g2((D * (D + 1) + 255) / 256, (unsigned)(pl.heads < 65535 ? pl.heads : 65535));
@@ -281,7 +291,7 @@ la_status run_simt(const Launch& L) {
     const int gc = pl.sc.nseg < (1 << 20) ? pl.sc.nseg : (1 << 20);
     apply_causal_simt<D, T><<<gc, kSimtThreads, smemc, L.stream>>>(
         static_cast<const T*>(L.q), static_cast<const T*>(L.k), static_cast<const T*>(L.v),
-        static_cast<const T*>(L.g), static_cast<T*>(L.out), N, pl.rope, pl.sc.nblk,
+        static_cast<const T*>(L.g), static_cast<T*>(L.out), N, pl.lay, pl.rope, pl.sc.nblk,
         pl.sc.nseg, apply, gtab, L.p->eps);
     if ((st = last_error()) != LA_OK) return st;
     return mark(L, 3);
@@ -293,7 +303,7 @@ la_status run_simt(const Launch& L) {
   dim3 g3(pl.apply_tps, pl.sc.nseg < 65535 ? pl.sc.nseg : 65535);
   apply_simt<D, T><<<g3, kSimtThreads, smem3, L.stream>>>(
       static_cast<const T*>(L.q), static_cast<const T*>(L.g), static_cast<T*>(L.out), pl.nq,
-      pl.rope, pl.lq, pl.sc.nblk, pl.apply_tps, pl.sc.nseg, apply, gtab, L.p->eps);
+      pl.lay, pl.rope, pl.lq, pl.sc.nblk, pl.apply_tps, pl.sc.nseg, apply, gtab, L.p->eps);
   if ((st = last_error()) != LA_OK) return st;
   return mark(L, 3);
 }
@@ -325,6 +335,8 @@ la_status run(const Launch& L) {
     a.out = L.out;
     a.flag = reinterpret_cast<int*>(L.ws + L.pl->off_flag);
     a.counters = reinterpret_cast<int*>(L.ws + L.pl->off_flag + kCounterOffset);
+    a.bnhd = L.pl->lay.bnhd;
+    a.H = L.pl->lay.H;
     a.fused = L.pl->sc.nblk == 1 && L.pl->sc.nseg <= kMaxCounters;
     a.gtab = reinterpret_cast<float2*>(L.ws + L.pl->off_tab);
     a.part = reinterpret_cast<float*>(L.ws + L.pl->off_part);

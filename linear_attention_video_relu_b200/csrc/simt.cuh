@@ -38,7 +38,7 @@ __device__ inline void token_pos(const Rope& r, long long n, int& tl, int& h, in
 template <int D, typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N,
-                   Rope rope, Sched sc, float* __restrict__ partials,
+                   Layout lay, Rope rope, Sched sc, float* __restrict__ partials,
                    float2* __restrict__ gtab) {
   constexpr int TT = kSimtTileState;
   constexpr int R = D / 16;
@@ -101,16 +101,17 @@ state_partial_simt(const T* __restrict__ k, const T* __restrict__ v, long long N
     const int seglen = (int)min((long long)sc.L, N - (long long)blk * sc.L);
     const int rows = min(TT, seglen - r0);
     const long long nbase = (long long)blk * sc.L + r0;
-    const T* kh = k + ((long long)head * N + nbase) * D;
-    const T* vh = v + ((long long)head * N + nbase) * D;
+    const T* kh = k + lay.row(head, nbase, N, D);
+    const T* vh = v + lay.row(head, nbase, N, D);
+    const long long ts = lay.tok_stride(D);
     for (int idx = tid; idx < TT * (D / 2); idx += kSimtThreads) {
       const int r = idx / (D / 2), pr = idx - r * (D / 2);
       float x0 = 0.f, x1 = 0.f, v0 = 0.f, v1 = 0.f;
       if (r < rows) {
-        x0 = relu(to_f32(kh[r * D + 2 * pr]));
-        x1 = relu(to_f32(kh[r * D + 2 * pr + 1]));
-        v0 = to_f32(vh[r * D + 2 * pr]);
-        v1 = to_f32(vh[r * D + 2 * pr + 1]);
+        x0 = relu(to_f32(kh[r * ts + 2 * pr]));
+        x1 = relu(to_f32(kh[r * ts + 2 * pr + 1]));
+        v0 = to_f32(vh[r * ts + 2 * pr]);
+        v1 = to_f32(vh[r * ts + 2 * pr + 1]);
       }
       float y0 = x0, y1 = x1;
       if (rope.on && r < rows) {
@@ -190,7 +191,7 @@ reduce_states(const float* __restrict__ partials, Sched sc, float* __restrict__ 
 template <int D, typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out,
-           long long N, Rope rope, int L, int nblk, int tps, int nseg,
+           long long N, Layout lay, Rope rope, int L, int nblk, int tps, int nseg,
            const float* __restrict__ apply,
            const float2* __restrict__ gtab, float eps) {
   constexpr int TT = kSimtTileApply;
@@ -209,7 +210,8 @@ apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out
   const int r0 = tile * TT;
   const int rows = min(TT, L - r0);
   const long long nbase = (long long)blk * L + r0;
-  const long long ebase = ((long long)head * N + nbase) * D;
+  const long long ebase = lay.row(head, nbase, N, D);
+  const long long ts = lay.tok_stride(D);
 
   const float4* src = reinterpret_cast<const float4*>(apply + (long long)seg * DD1);
   for (int i = tid; i < DD1 / 4; i += kSimtThreads) reinterpret_cast<float4*>(s_S)[i] = src[i];
@@ -217,8 +219,8 @@ apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out
     const int r = idx / (D / 2), pr = idx - r * (D / 2);
     float x0 = 0.f, x1 = 0.f;
     if (r < rows) {
-      x0 = relu(to_f32(q[ebase + r * D + 2 * pr]));
-      x1 = relu(to_f32(q[ebase + r * D + 2 * pr + 1]));
+      x0 = relu(to_f32(q[ebase + r * ts + 2 * pr]));
+      x1 = relu(to_f32(q[ebase + r * ts + 2 * pr + 1]));
     }
     float y0 = x0, y1 = x1;
     if (rope.on && r < rows) {
@@ -250,8 +252,9 @@ apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out
 #pragma unroll 8
     for (int a = 0; a < D; ++a) num = fmaf(s_qr[r * D + a], s_S[a * D + c], num);
     float o = num / s_den[r];
-    if (g) o *= sigmoid(to_f32(g[ebase + idx]));
-    out[ebase + idx] = from_f32<T>(o);
+    const long long e = ebase + r * ts + c;
+    if (g) o *= sigmoid(to_f32(g[e]));
+    out[e] = from_f32<T>(o);
   }
   __syncthreads();
   }
@@ -267,7 +270,8 @@ apply_simt(const T* __restrict__ q, const T* __restrict__ g, T* __restrict__ out
 template <int D, typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 apply_causal_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                  const T* __restrict__ g, T* __restrict__ out, long long N, Rope rope, int nblk,
+                  const T* __restrict__ g, T* __restrict__ out, long long N, Layout lay,
+                  Rope rope, int nblk,
                   int nseg, const float* __restrict__ apply, const float2* __restrict__ gtab,
                   float eps) {
   constexpr int C = kCausalChunk;
@@ -290,7 +294,8 @@ apply_causal_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const int head = seg / nblk, blk = seg - head * nblk;
     const long long nbase = (long long)blk * C;
     const int rows = (int)min((long long)C, N - nbase);
-    const long long ebase = ((long long)head * N + nbase) * D;
+    const long long ebase = lay.row(head, nbase, N, D);
+    const long long ts = lay.tok_stride(D);
     // the state of the chunks before this one (zero for the first)
     if (blk > 0) {
       const float4* src = reinterpret_cast<const float4*>(apply + (long long)(seg - 1) * DD1);
@@ -302,7 +307,7 @@ apply_causal_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
       const int r = idx / (D / 2), pr = idx - r * (D / 2);
       float qx = 0.f, qy = 0.f, kx = 0.f, ky = 0.f, v0 = 0.f, v1 = 0.f;
       if (r < rows) {
-        const long long e = ebase + r * D + 2 * pr;
+        const long long e = ebase + r * ts + 2 * pr;
         qx = relu(to_f32(q[e]));
         qy = relu(to_f32(q[e + 1]));
         kx = relu(to_f32(k[e]));
@@ -365,8 +370,9 @@ apply_causal_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
       for (int a = 0; a < D; ++a) num = fmaf(s_qr[r * D + a], s_S[a * D + c], num);
       for (int j = 0; j <= r; ++j) num = fmaf(s_P[r * C + j], s_v[j * D + c], num);
       float o = num / s_den[r];
-      if (g) o *= sigmoid(to_f32(g[ebase + idx]));
-      out[ebase + idx] = from_f32<T>(o);
+      const long long e = ebase + r * ts + c;
+      if (g) o *= sigmoid(to_f32(g[e]));
+      out[e] = from_f32<T>(o);
     }
     __syncthreads();
   }

@@ -41,7 +41,7 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 enum : int { kFlagStateTimeout = 1, kFlagApplyTimeout = 2 };
 
 struct TcArgs {
-  int D;
+  int D;           // I/O head dim (64, 112 or 128; 112 runs on the 128 kernels)
   long long N;
   int Lq;          // query rows per segment: sc.L, or the query length of a cross-attention
   Rope rope;
@@ -56,6 +56,7 @@ struct TcArgs {
   float* stS;
   float* stz;
   int* counters;   // per-segment arrival counters (zero between calls)
+  int bnhd, H;     // [B,N,H,D] tensors (else [B,H,N,D]); heads per batch entry
   int fused;       // one segment per head: the state build writes the images
   int use_state, commit, do_apply;
   float eps;
@@ -177,11 +178,17 @@ inline int pick_apply_stages(int D, int entries, int gate) {
 // Which calls take the tensor-core kernels: bf16 I/O, D in {64, 128}, and RoPE
 // widths that are multiples of 8 (a 16-byte chunk never spans two axes), with
 // both kernels' shared memory within budget (gated or not).
+// Head dim the tensor-core kernels run at for an I/O head dim: 112-wide rows
+// run on the 128 kernels, the tensor maps reading columns 112..127 as zero
+// fill and the apply kernel storing only the first 112 columns.
+inline int tc_kernel_dim(int D) { return D == 112 ? 128 : D; }
+
 inline bool tc_supported(bool bf16, int D, int rope, int dt, int dh, int dw, int entries) {
-  if (!bf16 || (D != 64 && D != 128)) return false;
+  if (!bf16 || (D != 64 && D != 112 && D != 128)) return false;
   if (rope && ((dt % 8) || (dh % 8) || (dw % 8))) return false;
   int e = rope ? entries : 0;
-  return pick_state_stages(D, e) > 0 && pick_apply_stages(D, e, 1) > 0;
+  const int Dk = tc_kernel_dim(D);
+  return pick_state_stages(Dk, e) > 0 && pick_apply_stages(Dk, e, 1) > 0;
 }
 
 // ---- device helpers ------------------------------------------------------------
@@ -284,6 +291,31 @@ struct TileIter {
   }
 };
 
+// Coordinates of (segment, row) in the 4D tensor maps of q, k, v, gate and
+// out. [B,H,N,D] tensors are mapped as {D, L, nseg, 1}: coordinates
+// (x, row, seg, 0). [B,N,H,D] tensors as {D, H, L, B * nblk} (strides D, H*D,
+// L*H*D elements): coordinates (x, h, row, b * nblk + blk). A box of 64
+// columns x rows x one head lands in shared memory in the same order either
+// way, and rows past a segment's L read as zero fill in both.
+struct SegCoords {
+  int bnhd, H, nblk;
+  FastDiv div_nblk, div_h;
+  __device__ __forceinline__ int3 of(int seg, int row) const {
+    if (!bnhd) return make_int3(row, seg, 0);
+    const int head = fdiv(div_nblk, seg), blk = seg - head * nblk;
+    const int b = fdiv(div_h, head), h = head - b * H;
+    return make_int3(h, row, b * nblk + blk);
+  }
+  // element offset of row r of segment seg (L rows per segment) in an output
+  // tensor with rows of ocols values
+  __device__ __forceinline__ long long out_row(int seg, int L, int r, int ocols) const {
+    if (!bnhd) return ((long long)seg * L + r) * ocols;
+    const int head = fdiv(div_nblk, seg), blk = seg - head * nblk;
+    const int b = fdiv(div_h, head), h = head - b * H;
+    return ((((long long)b * nblk + blk) * L + r) * H + h) * (long long)ocols;
+  }
+};
+
 // A math warp owns one 16-byte chunk column (8 dims = 4 rotation pairs, all on
 // one axis) and its lanes walk consecutive token rows. The TMA warp writes,
 // for every row of a tile, the table offset of the row's position on each
@@ -298,6 +330,13 @@ __device__ __forceinline__ ChunkCol chunk_col(const Rope& r, int chunk) {
   const int p0 = 4 * chunk;
   c.ax = p0 < r.pair_base[1] ? 0 : (p0 < r.pair_base[2] ? 1 : 2);
   c.pair_off = p0 - (c.ax == 0 ? 0 : (c.ax == 1 ? r.pair_base[1] : r.pair_base[2]));
+  // padding columns past the last rotary pair (a 112-wide head on the 128
+  // kernels) hold zeros: any finite cos/sin leaves them zero, so they read
+  // the first entries of the t axis
+  if (p0 >= r.pair_base[2] + r.half[2]) {
+    c.ax = 0;
+    c.pair_off = 0;
+  }
   return c;
 }
 
@@ -528,8 +567,8 @@ constexpr int kTailSegs = 32;   // segments a CTA can leave to its tail
 template <int D, bool ROPE>
 __global__ void __launch_bounds__(kTcThreadsState, 1)
 state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const __grid_constant__ Rope rope, const __grid_constant__ Sched sc, int stages,
-               float* __restrict__ partials, float2* __restrict__ gtab, int* flag,
+               const __grid_constant__ Rope rope, const __grid_constant__ Sched sc,
+               const __grid_constant__ SegCoords scd, int stages, float* __restrict__ partials, float2* __restrict__ gtab, int* flag,
                int* __restrict__ counters, uint8_t* __restrict__ images, float* stS,
                float* stz, int use_state, int commit) {
   constexpr int TT = tc_state_tile_c(D);      // tokens per tile
@@ -622,12 +661,11 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       if (lane == 0) {
         const uint32_t kt = base + it.stage * STAGE_BYTES, vt = kt + TILE_BYTES;
         ptx::mbar_expect_tx(full_bar(it.stage), STAGE_BYTES);
+        const int3 c = scd.of(it.seg, it.tile * TT);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h) {
-          ptx::tma_load_3d(kt + h * HALF_BYTES, &tm_k, 64 * h, it.tile * TT, it.seg,
-                           full_bar(it.stage));
-          ptx::tma_load_3d(vt + h * HALF_BYTES, &tm_v, 64 * h, it.tile * TT, it.seg,
-                           full_bar(it.stage));
+          ptx::tma_load_4d(kt + h * HALF_BYTES, &tm_k, 64 * h, c.x, c.y, c.z, full_bar(it.stage));
+          ptx::tma_load_4d(vt + h * HALF_BYTES, &tm_v, 64 * h, c.x, c.y, c.z, full_bar(it.stage));
         }
       }
       ++issued;
@@ -977,9 +1015,9 @@ __host__ __device__ constexpr uint32_t tmem_cols_pow2(uint32_t n) {
 template <int D, bool ROPE, bool GATE>
 __global__ void __launch_bounds__(kTcThreadsApply, 1)
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
-         const __grid_constant__ CUtensorMap tm_o, __nv_bfloat16* __restrict__ out,
+         const __grid_constant__ CUtensorMap tm_o, __nv_bfloat16* __restrict__ out, int ocols,
          const __grid_constant__ Rope rope, int L, int nblk,
-         long long U, int stages, int sbuf, int gst, const uint8_t* __restrict__ images,
+         const __grid_constant__ SegCoords scd, long long U, int stages, int sbuf, int gst, const uint8_t* __restrict__ images,
          const float2* __restrict__ gtab, float eps, int* flag) {
   constexpr int TM = kApplyTile;
   constexpr int HALVES = D / 64;
@@ -1095,13 +1133,14 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       }
       if (lane == 0) {
         ptx::mbar_expect_tx(full_bar(it.stage), TX);
+        const int3 c = scd.of(it.seg, it.tile * TM);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h) {
-          ptx::tma_load_3d(base + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_q, 64 * h,
-                           it.tile * TM, it.seg, full_bar(it.stage));
+          ptx::tma_load_4d(base + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_q, 64 * h, c.x,
+                           c.y, c.z, full_bar(it.stage));
           if (!DIRECT && GATE)
-            ptx::tma_load_3d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h,
-                             it.tile * TM, it.seg, full_bar(it.stage));
+            ptx::tma_load_4d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h, c.x,
+                             c.y, c.z, full_bar(it.stage));
         }
       }
       ++issued;
@@ -1180,10 +1219,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       for (long long u = u0; u < u1; ++u, it.next()) {
         if (!wait_bounded(oready_bar(it.stage), it.phase, flag, kFlagApplyTimeout, &s_abort))
           break;
+        const int3 c = scd.of(it.seg, it.tile * TM);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
-          ptx::tma_store_3d(&tm_o, base + it.stage * TILE_BYTES + h * HALF_BYTES, 64 * h,
-                            it.tile * TM, it.seg);
+          ptx::tma_store_4d(&tm_o, base + it.stage * TILE_BYTES + h * HALF_BYTES, 64 * h, c.x,
+                            c.y, c.z);
         ptx::bulk_commit();
         ptx::bulk_wait_read<0>();
         ptx::mbar_arrive(empty_bar(it.stage));
@@ -1200,10 +1240,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                           &s_abort))
           break;
         ptx::mbar_expect_tx(gfull_bar(it.stage), TILE_BYTES);
+        const int3 c = scd.of(it.seg, it.tile * TM);
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
-          ptx::tma_load_3d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h,
-                           it.tile * TM, it.seg, gfull_bar(it.stage));
+          ptx::tma_load_4d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h, c.x,
+                           c.y, c.z, gfull_bar(it.stage));
         ++issued;
       }
       for (long long i = issued - gst < 0 ? 0 : issued - gst; i < issued; ++i)
@@ -1245,7 +1286,8 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       if (ready && gready && (!DIRECT || r < L)) {
         const float inv = 1.f / (eps + (__uint_as_float(dz[0]) + __uint_as_float(dz[1])));
         const uint64_t inv2 = ptx::f2(inv, inv);
-        uint4* dst = reinterpret_cast<uint4*>(out + ((long long)seg * L + r) * D + col0);
+        // rows of ocols values: D, or 112 for a 112-wide head on the 128 kernels
+        uint4* dst = reinterpret_cast<uint4*>(out + scd.out_row(seg, L, r, ocols) + col0);
         const uint32_t gt = gbase + (DIRECT ? gs : s) * TILE_BYTES;
         const int h = col0 / 64;
 #pragma unroll
@@ -1270,8 +1312,11 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           }
           const uint4 ov = make_uint4(ptx::pack_bf16x2(o[0], o[1]), ptx::pack_bf16x2(o[2], o[3]),
                                       ptx::pack_bf16x2(o[4], o[5]), ptx::pack_bf16x2(o[6], o[7]));
-          if (DIRECT) dst[k4] = ov;
-          else ptx::st_shared_v4(base + s * TILE_BYTES + off, ov);
+          if (DIRECT) {
+            if (col0 + 8 * k4 < ocols) dst[k4] = ov;
+          } else {
+            ptx::st_shared_v4(base + s * TILE_BYTES + off, ov);
+          }
         }
       }
       ptx::tc_fence_before();
@@ -1373,14 +1418,33 @@ inline EncodeTiledFn encode_fn() {
 }
 
 // [nseg][L][D] bf16 view of a [B,H,N,D] tensor; box = 64 columns x rows x 1.
-inline bool make_map(CUtensorMap* m, const void* ptr, int D, int L, int nseg, int rows) {
+// 4D map of a bf16 tensor of rows D values wide, cut into segments of L rows
+// (see SegCoords): {D, L, nseg, 1} for [B,H,N,D], {D, H, L, B * nblk} for
+// [B,N,H,D]; box 64 columns x `rows` rows of one segment.
+inline bool make_map(CUtensorMap* m, const void* ptr, int D, int L, int nseg, int rows,
+                     const SegCoords& sc) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)nseg};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)L * D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+  const cuuint64_t row = (cuuint64_t)D * 2;   // bytes of one row
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4] = {64, 1, 1, 1};
+  if (!sc.bnhd) {
+    dims[0] = (cuuint64_t)D; dims[1] = (cuuint64_t)L; dims[2] = (cuuint64_t)nseg; dims[3] = 1;
+    strides[0] = row;
+    strides[1] = row * (cuuint64_t)L;
+    strides[2] = row * (cuuint64_t)L * (cuuint64_t)nseg;
+    box[1] = (cuuint32_t)rows;
+  } else {
+    const cuuint64_t H = (cuuint64_t)sc.H;
+    dims[0] = (cuuint64_t)D; dims[1] = H; dims[2] = (cuuint64_t)L;
+    dims[3] = (cuuint64_t)nseg / H;            // B * nblk
+    strides[0] = row;
+    strides[1] = row * H;
+    strides[2] = row * H * (cuuint64_t)L;
+    box[2] = (cuuint32_t)rows;
+  }
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
@@ -1438,8 +1502,15 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   const int entries = a.rope.on ? a.rope.entries : 0;
   const Sched& sc = a.sc;
   CUtensorMap mk, mv, mq, mg, mo;
-  if (!make_map(&mk, a.k, D, sc.L, sc.nseg, tc_state_tile_c(D)) ||
-      !make_map(&mv, a.v, D, sc.L, sc.nseg, tc_state_tile_c(D)))
+  SegCoords scd;
+  scd.bnhd = a.bnhd;
+  scd.H = a.H > 0 ? a.H : 1;
+  scd.nblk = sc.nblk;
+  scd.div_nblk = make_fastdiv(sc.nblk);
+  scd.div_h = make_fastdiv(scd.H);
+  // tensor maps over the I/O rows (a.D wide); columns past a.D read as zeros
+  if (!make_map(&mk, a.k, a.D, sc.L, sc.nseg, tc_state_tile_c(D), scd) ||
+      !make_map(&mv, a.v, a.D, sc.L, sc.nseg, tc_state_tile_c(D), scd))
     return LA_ERR_CUDA;
   la_status st;
   const int s1 = pick_state_stages(D, entries);
@@ -1449,7 +1520,7 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   if ((st = tc_mark(a, 0)) != LA_OK) return st;
   uint8_t* images = reinterpret_cast<uint8_t*>(a.apply);
   st = launch_pdl(k1, dim3(sc.G), dim3(kTcThreadsState), p1.total, a.stream, mk, mv, a.rope,
-                  sc, s1, a.part, a.gtab, a.flag, a.fused ? a.counters : nullptr, images,
+                  sc, scd, s1, a.part, a.gtab, a.flag, a.fused ? a.counters : nullptr, images,
                   a.stS, a.stz, a.use_state, a.commit);
   if (st != LA_OK) return st;
   if ((st = tc_mark(a, 1)) != LA_OK) return st;
@@ -1465,9 +1536,9 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   if (!a.do_apply) return LA_OK;
 
   const bool gate = a.g != nullptr;
-  if (!make_map(&mq, a.q, D, a.Lq, sc.nseg, kApplyTile) ||
-      !make_map(&mo, a.out, D, a.Lq, sc.nseg, kApplyTile) ||
-      !make_map(&mg, gate ? a.g : a.q, D, a.Lq, sc.nseg, kApplyTile))
+  if (!make_map(&mq, a.q, a.D, a.Lq, sc.nseg, kApplyTile, scd) ||
+      !make_map(&mo, a.out, a.D, a.Lq, sc.nseg, kApplyTile, scd) ||
+      !make_map(&mg, gate ? a.g : a.q, a.D, a.Lq, sc.nseg, kApplyTile, scd))
     return LA_ERR_CUDA;
   int s3 = 0, sb3 = 1, gs3 = 0;
   pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3, &gs3);
@@ -1478,7 +1549,8 @@ la_status tc_run_d(const TcArgs& a, int sms) {
                       : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
   if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
   st = launch_pdl(k3, dim3(G3), dim3(kTcThreadsApply), p3.total, a.stream, mq, mg, mo,
-                  static_cast<__nv_bfloat16*>(a.out), a.rope, a.Lq, sc.nblk, U3, s3, sb3, gs3,
+                  static_cast<__nv_bfloat16*>(a.out), a.D, a.rope, a.Lq, sc.nblk, scd, U3, s3,
+                  sb3, gs3,
                   reinterpret_cast<const uint8_t*>(a.apply), (const float2*)a.gtab, a.eps,
                   a.flag);
   if (st != LA_OK) return st;
@@ -1487,7 +1559,7 @@ la_status tc_run_d(const TcArgs& a, int sms) {
 
 inline la_status tc_run(const TcArgs& a, int sms) {
   if (a.D == 64) return tc_run_d<64>(a, sms);
-  if (a.D == 128) return tc_run_d<128>(a, sms);
+  if (a.D == 112 || a.D == 128) return tc_run_d<128>(a, sms);
   return LA_ERR_UNSUPPORTED;
 }
 

@@ -218,13 +218,16 @@ def test_temporal_conv_without_work_is_a_no_op():
         assert _tconv(x=None, w=None, y=None, **kw) == C.LA_OK
 
 
-def test_head_dim_112_is_accepted_on_the_cuda_core_path():
+def test_head_dim_112_is_accepted():
     # 56 rotary pairs split over (t, h, w); passes the host checks (the fake
-    # pointers then fail only at the device query) and never takes the
-    # tensor-core kernels
+    # pointers then fail only at the device query); bf16 with widths that are
+    # multiples of 8 takes the (padded) tensor-core kernels, fp32 does not
     p = _params(D=112, rope_dt=16, rope_dh=48, rope_dw=48)
     assert C.lin_attn_forward(p, Q, K, V, None, O, WS, 1 << 20, None) != C.LA_ERR_INVALID_ARG
-    assert C.lin_attn_uses_tensor_cores(p) == 0
+    assert C.lin_attn_uses_tensor_cores(p) == 1
+    assert C.lin_attn_uses_tensor_cores(_params(D=112, rope_dt=16, rope_dh=48, rope_dw=48,
+                                                dtype=C.LA_F32)) == 0
+    assert C.lin_attn_uses_tensor_cores(_params(D=112, rope_dt=20, rope_dh=46, rope_dw=46)) == 0
     assert C.lin_attn_forward(_params(D=96, rope_dt=32, rope_dh=32, rope_dw=32), Q, K, V, None,
                               O, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
 
@@ -242,3 +245,13 @@ def test_segment_count_limit():
     far = [i << 40 for i in range(1, 6)]
     assert C.lin_attn_forward(p, far[0], far[1], far[2], None, far[3], far[4], 1 << 20,
                               None) not in (C.LA_ERR_UNSUPPORTED, C.LA_ERR_INVALID_ARG)
+
+
+def test_layout_field():
+    # [B,N,H,D] passes the host checks; anything else but the two orders is refused
+    p = _params(layout=C.LA_LAYOUT_BNHD)
+    assert C.lin_attn_forward(p, Q, K, V, None, O, WS, 1 << 20, None) != C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_forward(_params(layout=2), Q, K, V, None, O, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=16, rope_dh=24, rope_dw=24,
+                                                layout=C.LA_LAYOUT_BNHD)) == 1

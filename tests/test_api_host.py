@@ -36,3 +36,14 @@ def test_fp32_params_want_fp32_tensors():
     api._check_io(_p(torch.float32), x, require_cuda=False)
     with pytest.raises(TypeError):
         api._check_io(_p(torch.float32), x.to(torch.bfloat16), require_cuda=False)
+
+
+def test_bnhd_shapes():
+    p = api.make_params(1, 2, 6, 32, torch.bfloat16, layout="bnhd")
+    api._check_io(p, torch.zeros((1, 6, 2, 32), dtype=torch.bfloat16), require_cuda=False)
+    with pytest.raises(ValueError):
+        api._check_io(p, torch.zeros((1, 2, 6, 32), dtype=torch.bfloat16), require_cuda=False)
+    assert api._dims(torch.zeros((1, 6, 2, 32)), "bnhd") == (1, 2, 6, 32)
+    assert api._dims(torch.zeros((1, 2, 6, 32)), "bhnd") == (1, 2, 6, 32)
+    with pytest.raises(ValueError):
+        api.make_params(1, 2, 6, 32, torch.bfloat16, layout="nbhd")
