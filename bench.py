@@ -582,10 +582,35 @@ def secondary_lines(K, device, peak, peak_kind):
     out = []
     for name, job in jobs:
         try:
-            out.append(job())
+            out.append(compact(job()))
         except Exception as e:   # reported in the line, not swallowed
-            out.append({"workload": name, "error": "%s: %s" % (type(e).__name__, e)})
+            out.append({"w": name, "error": ("%s: %s" % (type(e).__name__, e))[:160]})
     return out
+
+
+def compact(r: dict) -> dict:
+    """A secondary result in a few short keys, so that every one of them fits
+    in the tail of the output: w workload, mode, ms (or us) per call, frac =
+    algorithmic HBM bytes / time as a fraction of the peak, and per kernel its
+    average us and roofline fraction (sb state build, ap apply, red the
+    separate reduction)."""
+    c = {"w": r["workload"], "mode": r.get("mode")}
+    if "ms_per_step" in r:
+        c["ms"] = round(r["ms_per_step"], 4)
+    for key, short in (("us_per_forward", "us"), ("us_per_call", "us"),
+                       ("us_per_block", "us_blk")):
+        if key in r:
+            c[short] = round(r[key], 2)
+    if "tokens_per_s" in r:
+        c["tok_s"] = float("%.4g" % r["tokens_per_s"])
+    if "hbm_frac" in r:
+        c["frac"] = round(r["hbm_frac"], 4)
+    k = r.get("kernels")
+    if k:
+        c["sb"] = [k["state_build"]["avg_us"], k["state_build"]["frac"]]
+        c["ap"] = [k["apply"]["avg_us"], k["apply"]["frac"]]
+        c["red_us"] = k["reduce_us"]
+    return c
 
 
 def config_of(w, mode, world):
@@ -667,10 +692,11 @@ def main():
         line["metric"] = "linear-attn fwd tokens/s (profiling run: %s, %s)" % (w.name, mode)
     if rank == 0 and args.e2e_steps > 0:
         line["e2e"] = measure_e2e(w, args.e2e_steps, device, w.seed)
-    if not args.no_extra and rank == 0:
-        line["also"] = secondary_lines(max(20, args.steps // 5), device, peak, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
+    if not args.no_extra and rank == 0:
+        # last in the line, in short keys (see compact), so it survives in a tail
+        line["also"] = secondary_lines(max(20, args.steps // 5), device, peak, peak_kind)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:

@@ -30,10 +30,13 @@
  *
  * Conventions for every entry point:
  *   - Memory. The caller owns all device memory (inputs, output, state,
- *     workspace); the library allocates and frees nothing and keeps no global
- *     mutable state, so calls are re-entrant.
+ *     workspace); the library allocates and frees nothing. Every entry point
+ *     but lin_attn_forward_noalloc keeps no global mutable state, so those
+ *     calls are re-entrant; lin_attn_forward_noalloc works in one device
+ *     array shared by all its calls (see its comment).
  *   - Layout. q, k, v, gate, out are contiguous [B, H, N, D] (or [B, N, H, D]
- *     with p->layout = LA_LAYOUT_BNHD) with D innermost, in the I/O dtype. The state is fp32: S [B, H, D, D] with
+ *     with p->layout = LA_LAYOUT_BNHD) with D innermost, in the I/O dtype.
+ *     The state is fp32: S [B, H, D, D] with
  *     S[a][c] = sum_j RoPE(phi(k_j))_a v_j,c, and z [B, H, D].
  *   - Asynchrony. A call checks its arguments on the host, enqueues kernels on
  *     `stream` (a cudaStream_t passed as void*, NULL = legacy default stream)
@@ -209,6 +212,11 @@ LA_API la_status lin_attn_cross_workspace_size(const la_params* p, int n_kv, siz
  *     that overlap on the GPU -- on different streams, or from different host
  *     threads without ordering -- race on it and give wrong results; order them
  *     on one stream.
+ *   - No status query: the array's control block (with the flag a kernel sets
+ *     when it gives up a bounded wait) is cleared at the start of every call,
+ *     and no entry point reads it back, so a call whose kernel gave up such a
+ *     wait cannot be detected on this path. Callers that need that check use
+ *     lin_attn_forward with lin_attn_device_status.
  * Arguments and results are those of lin_attn_forward without the workspace. */
 LA_API la_status lin_attn_forward_noalloc(const la_params* p, const void* q, const void* k,
                                           const void* v, const void* gate, void* out,
@@ -228,7 +236,9 @@ LA_API la_status lin_attn_state_reset(const la_state* st, void* stream);
  * with (S, z) the carried state and (S_blk, z_blk) the sums over this block.
  * commit != 0 then sets S += S_blk, z += z_blk in place (the cache update at
  * the last denoising step); commit == 0 leaves the state byte-identical.
- * gate may be NULL. The state must match p (B, H, D). */
+ * gate may be NULL. The state must match p (B, H, D). q, k, v, gate and out
+ * may not share bytes with S or z, nor S with z (else LA_ERR_INVALID_ARG,
+ * nothing launched): the state is updated in place while they are read. */
 LA_API la_status lin_attn_block_step(const la_params* p, la_state* st, int t_offset,
                               const void* q, const void* k, const void* v,
                               const void* gate, void* out, int commit,

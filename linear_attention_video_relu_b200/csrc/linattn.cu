@@ -396,9 +396,17 @@ la_status block_common(const la_params* p, la_state* st, int t_offset, const voi
   if (t_offset < 0) return LA_ERR_INVALID_ARG;
   if ((long long)p->B * p->H * p->N == 0) return LA_OK;
   if ((s = check_io(p, q, k, v, gate, out, do_apply)) != LA_OK) return s;
-  size_t sbytes = (size_t)p->B * p->H * p->D * p->D * sizeof(float);
-  if (do_apply && (overlaps(out, (size_t)p->B * p->H * p->N * p->D * elt_size(p), st->S, sbytes)))
-    return LA_ERR_INVALID_ARG;
+  // The state is read and (commit) updated in place while q, k, v and gate
+  // are still being read and out written: none of them may share its bytes,
+  // and S and z may not share bytes with each other.
+  const size_t sbytes = (size_t)p->B * p->H * p->D * p->D * sizeof(float);
+  const size_t zbytes = (size_t)p->B * p->H * p->D * sizeof(float);
+  const size_t tbytes = (size_t)p->B * p->H * p->N * p->D * elt_size(p);
+  if (overlaps(st->S, sbytes, st->z, zbytes)) return LA_ERR_INVALID_ARG;
+  const void* io[5] = {q, k, v, gate, out};
+  for (const void* t : io)
+    if (overlaps(t, tbytes, st->S, sbytes) || overlaps(t, tbytes, st->z, zbytes))
+      return LA_ERR_INVALID_ARG;
   Plan pl;
   if ((s = make_plan(p, true, t_offset, &pl)) != LA_OK) return s;
   if ((s = check_workspace(pl, workspace, workspace_bytes)) != LA_OK) return s;
@@ -430,10 +438,13 @@ la_status cross_plan(const la_params* p, int n_kv, Plan* pl) {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_noalloc_once[kMaxDevices];
-void* g_noalloc_ptr[kMaxDevices];
-cudaError_t g_noalloc_err[kMaxDevices];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices];   // set once a lookup on that device succeeded
 
+// Device address of the scratch array on the current device. Only a
+// successful lookup is kept: a failed one (say, a call made before the
+// context could be created) returns LA_ERR_CUDA and is tried again by the
+// next call.
 la_status noalloc_scratch(void** ptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -441,11 +452,15 @@ la_status noalloc_scratch(void** ptr) {
     return LA_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
-  std::call_once(g_noalloc_once[dev], [dev] {
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
-    if (g_noalloc_err[dev] != cudaSuccess) cudaGetLastError();
-  });
-  if (g_noalloc_err[dev] != cudaSuccess || !g_noalloc_ptr[dev]) return LA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return LA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
   *ptr = g_noalloc_ptr[dev];
   return LA_OK;
 }
@@ -557,7 +572,8 @@ la_status lin_attn_forward_noalloc(const la_params* p, const void* q, const void
 }
 
 la_status lin_attn_state_init(la_state* st, int B, int H, int D, float* S, float* z) {
-  if (!st || B < 0 || H < 0 || (D != 32 && D != 64 && D != 128)) return LA_ERR_INVALID_ARG;
+  if (!st || B < 0 || H < 0 || (D != 32 && D != 64 && D != 112 && D != 128))
+    return LA_ERR_INVALID_ARG;
   if (!S || !z || !aligned16(S) || !aligned16(z)) return LA_ERR_INVALID_ARG;
   st->S = S;
   st->z = z;

@@ -255,3 +255,43 @@ def test_layout_field():
         C.LA_ERR_INVALID_ARG
     assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=16, rope_dh=24, rope_dw=24,
                                                 layout=C.LA_LAYOUT_BNHD)) == 1
+
+
+def test_block_step_rejects_tensors_sharing_bytes_with_the_state():
+    # A block step reads the state and (commit) updates it in place while q,
+    # k, v and gate are still being read and out written, so none of them may
+    # overlap S or z, and S and z may not overlap each other.
+    p = _params()                       # B=1, H=2, N=60, D=32, bf16: 7680-byte tensors
+    S, Z = 0x100000, 0x110000           # S: 8192 bytes, z: 256 bytes
+    st = C.la_state()
+    assert C.lin_attn_state_init(st, 1, 2, 32, S, Z) == C.LA_OK
+    # clear of the state: past the host checks (fails only at the device query)
+    assert C.lin_attn_block_step(p, st, 0, Q, K, V, None, O, 1, WS, 1 << 20, None) != \
+        C.LA_ERR_INVALID_ARG
+    bad = [
+        (Q, K, V, None, S + 64),        # out inside S
+        (Q, K, V, None, Z - 128),       # out running into z
+        (S + 4096, K, V, None, O),      # q inside S
+        (Q, Z, V, None, O),             # k on z
+        (Q, K, S, None, O),             # v on S
+        (Q, K, V, Z - 16, O),           # gate running into z
+    ]
+    for q, k, v, g, o in bad:
+        assert C.lin_attn_block_step(p, st, 0, q, k, v, g, o, 1, WS, 1 << 20, None) == \
+            C.LA_ERR_INVALID_ARG, (q, k, v, g, o)
+    assert C.lin_attn_state_update(p, st, 0, Z, V, WS, 1 << 20, None) == C.LA_ERR_INVALID_ARG
+    assert C.lin_attn_state_update(p, st, 0, K, S + 8176, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+    # S and z sharing bytes
+    st2 = C.la_state()
+    assert C.lin_attn_state_init(st2, 1, 2, 32, S, S + 4096) == C.LA_OK
+    assert C.lin_attn_block_step(p, st2, 0, Q, K, V, None, O, 1, WS, 1 << 20, None) == \
+        C.LA_ERR_INVALID_ARG
+
+
+def test_state_init_accepts_every_head_dim_of_the_forward():
+    st = C.la_state()
+    for d in (32, 64, 112, 128):
+        assert C.lin_attn_state_init(st, 1, 2, d, 0x100000, 0x200000) == C.LA_OK
+        assert st.D == d
+    assert C.lin_attn_state_init(st, 1, 2, 96, 0x100000, 0x200000) == C.LA_ERR_INVALID_ARG

@@ -138,6 +138,30 @@ def test_secondary_lines_record_errors(monkeypatch):
     monkeypatch.setattr(bench, "measure_block_steps", ok)
     lines = bench.secondary_lines(20, None, 6535.7, "measured")
     errs = [l for l in lines if "error" in l]
-    assert len(errs) == 1 and errs[0]["workload"] == "480p_bidir_x_text300/cross"
+    assert len(errs) == 1 and errs[0]["w"] == "480p_bidir_x_text300/cross"
     assert "bounded wait" in errs[0]["error"]
-    assert len(lines) == 9 and sum(1 for l in lines if l == {"workload": "ok"}) == 8
+    assert len(lines) == 9 and sum(1 for l in lines if l.get("w") == "ok") == 8
+
+
+def test_secondary_lines_are_short():
+    # every secondary result is reduced to a few short keys, so that ten of
+    # them fit in the last ~3 KB of the bench output
+    kern = lambda us, f: {"avg_us": us, "frac": f, "kernel": "x", "bound": "hbm",
+                          "achieved": 1.0, "peak": 6535.7, "unit": "GB/s", "traffic": None,
+                          "algorithmic_bytes": 1, "peak_source": "measured"}
+    full = {"workload": "720p_long", "mode": "block_causal", "ms_per_step": 0.69123456,
+            "tokens_per_s": 319876543.21, "hbm_gbs": 5234.5678, "hbm_frac": 0.80098765,
+            "kernels": {"state_build": kern(350.123, 0.7712), "reduce_us": 14.2,
+                        "apply": kern(320.5, 0.8123)}}
+    c = bench.compact(full)
+    assert c["w"] == "720p_long" and c["mode"] == "block_causal"
+    assert c["ms"] == 0.6912 and c["frac"] == 0.801 and c["sb"] == [350.123, 0.7712]
+    assert c["ap"] == [320.5, 0.8123] and c["red_us"] == 14.2
+    cross = {"workload": "480p_bidir_x_text300", "mode": "cross", "n_kv": 300,
+             "us_per_forward": 61.66, "tokens_per_s": 5.3e8, "algorithmic_bytes": 1,
+             "hbm_gbs": 4392.1, "hbm_frac": 0.672}
+    blk = {"workload": "720p_long_block_step", "block_tokens": 3680, "us_per_block": 30.9,
+           "tokens_per_s": 1.19e8, "hbm_frac": 0.2986}
+    lines = [bench.compact(r) for r in (full, cross, blk)]
+    assert lines[1]["us"] == 61.66 and lines[2]["us_blk"] == 30.9
+    assert all(len(json.dumps(l)) < 200 for l in lines)
