@@ -1302,12 +1302,17 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           const int chunk = (col0 % 64) / 8 + k4;
           const uint32_t off = h * HALF_BYTES + row * 128 + ((chunk ^ (row & 7)) << 4);
           if (GATE) {
+            // sigmoid(g) = 1 / (1 + 2^(-g log2 e)) with the approximate
+            // exp2 and reciprocal of the special-function unit (a few ulp
+            // relative for every g; the output is then rounded to bf16)
             const uint4 gr = ptx::ld_shared_v4(gt + off);
             const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+            constexpr float kNegLog2e = -1.4426950408889634f;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              o[2 * e] *= __frcp_rn(1.f + __expf(-ptx::bf16_lo(gw[e])));
-              o[2 * e + 1] *= __frcp_rn(1.f + __expf(-ptx::bf16_hi(gw[e])));
+              o[2 * e] *= ptx::rcp_approx(1.f + ptx::ex2_approx(kNegLog2e * ptx::bf16_lo(gw[e])));
+              o[2 * e + 1] *=
+                  ptx::rcp_approx(1.f + ptx::ex2_approx(kNegLog2e * ptx::bf16_hi(gw[e])));
             }
           }
           const uint4 ov = make_uint4(ptx::pack_bf16x2(o[0], o[1]), ptx::pack_bf16x2(o[2], o[3]),
