@@ -59,7 +59,9 @@ def launches_per_forward(w, mode) -> int:
     """Kernels one forward launches: state build (+ reduction when a head has
     more than one segment) + apply."""
     if mode == "token_causal":
-        return 3   # CUDA-core kernels: state partials, scan, chunked apply
+        # tensor cores (bf16, D = 64): state partials + causal apply; CUDA
+        # cores: state partials, scan, chunked apply
+        return 2 if (w.dtype == "bf16" and w.D == 64) else 3
     one_segment = mode == "bidirectional" or w.block_tokens in (0, w.N)
     return 2 if one_segment else 3
 
@@ -300,11 +302,16 @@ def measure_workload(w, mode, steps, warmup, pg, device, peak, peak_kind, seed):
     tensor_bytes = w.B * w.H * w.N * w.D * elt
     state_bytes = 2 * tensor_bytes
     apply_bytes = (3 if w.gate else 2) * tensor_bytes
+    total_bytes = w.algorithmic_bytes()
+    if mode == "token_causal":
+        # the two-pass causal form reads k and v twice: 12 D bytes per
+        # token-head (bf16), the apply kernel reading q, k, v and writing out
+        apply_bytes += 2 * tensor_bytes
+        total_bytes += 2 * tensor_bytes
     step_ms = ms / steps
     k_state = roofline_entry("state_build", state_bytes, kern[0], peak, peak_kind, w.name)
     k_reduce_us = round(sum(kern[1]) / len(kern[1]) * 1e3, 2)
     k_apply = roofline_entry("apply", apply_bytes, kern[2], peak, peak_kind, w.name)
-    total_bytes = w.algorithmic_bytes()
     res = {
         "workload": w.name, "mode": mode, "ms_per_step": step_ms,
         "tokens_per_s": w.B * w.N / (step_ms * 1e-3),

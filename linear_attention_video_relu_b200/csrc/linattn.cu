@@ -11,8 +11,10 @@
 //                    the tensor-core path folded into the state build when
 //                    every head is one segment
 //   3. apply        (out = RoPE(phi q) S / (phi q . z + eps), gate)
-// The token-causal mode runs on the CUDA-core kernels with 32-token chunks
-// as segments and a chunked apply step.
+// The token-causal mode runs on the tensor cores at bf16 and D = 64 (the state
+// build's partials, then causal_tc carrying the running state through each
+// CTA's range), else on the CUDA-core kernels with 32-token chunks as
+// segments and a chunked apply step.
 #include "linattn.h"
 
 #include <limits.h>
@@ -21,6 +23,7 @@
 
 #include <mutex>
 
+#include "causal.cuh"
 #include "common.cuh"
 #include "simt.cuh"
 #include "tc.cuh"
@@ -107,7 +110,6 @@ la_status check_params(const la_params* p, bool one_block) {
 }
 
 bool want_tc(const la_params* p, bool one_block) {
-  if (!one_block && p->mode == LA_TOKEN_CAUSAL) return false;   // CUDA-core kernels only
   // 112-wide heads run padded on the 128 kernels, whose carried-state I/O is
   // 128 wide: block steps at D = 112 stay on the CUDA-core kernels
   if (one_block && p->D == 112) return false;
@@ -115,6 +117,9 @@ bool want_tc(const la_params* p, bool one_block) {
                                     p->grid_h * rope_stride(p->rope_dh / 2) +
                                     p->grid_w * rope_stride(p->rope_dw / 2)
                               : 0;
+  if (!one_block && p->mode == LA_TOKEN_CAUSAL)   // tensor cores at D = 64 only
+    return causal_tc_supported(p->dtype == LA_BF16, p->D, p->rope, p->rope_dt, p->rope_dh,
+                               p->rope_dw, entries);
   return tc_supported(p->dtype == LA_BF16, p->D, p->rope, p->rope_dt, p->rope_dh, p->rope_dw,
                       entries);
 }
@@ -169,10 +174,13 @@ la_status make_plan(const la_params* p, bool one_block, int t_offset, Plan* pl) 
 
   Sched& sc = pl->sc;
   const int N = p->N;
-  // token-causal: chunks of kCausalChunk tokens (the last one ragged)
+  // token-causal: on the CUDA-core kernels, segments of kCausalChunk tokens
+  // (the last one ragged); on the tensor cores, one segment per head (the
+  // apply kernel carries the running state through each CTA's range)
   pl->causal = !one_block && p->mode == LA_TOKEN_CAUSAL;
-  sc.L = pl->causal ? kCausalChunk
-                    : ((!one_block && p->mode == LA_BLOCK_CAUSAL) ? p->block_tokens : N);
+  sc.L = (pl->causal && !pl->tc)
+             ? kCausalChunk
+             : ((!one_block && p->mode == LA_BLOCK_CAUSAL) ? p->block_tokens : N);
   if (sc.L < 1) sc.L = 1;
   sc.nblk = (N + sc.L - 1) / sc.L;
   if (sc.nblk < 1) sc.nblk = 1;
@@ -349,6 +357,7 @@ la_status run(const Launch& L) {
     a.eps = L.p->eps;
     a.stream = L.stream;
     a.events = L.events;
+    if (L.pl->causal) return causal_run(a);
     return tc_run(a, L.pl->sms);
   }
   if (L.p->dtype == LA_BF16) return dispatch_simt<__nv_bfloat16>(L);

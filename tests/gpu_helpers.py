@@ -138,4 +138,8 @@ def sample_rows(w: workloads.Workload, count: int, seed: int, mode: str) -> np.n
         if mode == "block_causal":
             for b in range(1, w.N // w.block_tokens, max(1, (w.N // w.block_tokens) // 4)):
                 rows.update((base + b * w.block_tokens - 1, base + b * w.block_tokens))
+        if mode == "token_causal":
+            # both sides of 128-token chunk edges
+            for c in range(1, (w.N + 127) // 128, max(1, (w.N // 128) // 6)):
+                rows.update((base + 128 * c - 1, base + 128 * c))
     return np.array(sorted(rows), dtype=np.int64)

@@ -137,8 +137,14 @@ def test_tensor_core_path_selection_is_host_logic():
     assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=20, rope_dh=22, rope_dw=22)) == 0
     assert C.lin_attn_uses_tensor_cores(_params(D=128, rope_dt=32, rope_dh=48, rope_dw=48)) == 1
     assert C.lin_attn_uses_tensor_cores(_params(D=64, rope=0)) == 1
-    # token-causal runs on the CUDA-core kernels
+    # token-causal runs on the tensor cores at bf16 and D = 64 only
     assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=16, rope_dh=24, rope_dw=24,
+                                                mode=C.LA_TOKEN_CAUSAL)) == 1
+    assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=16, rope_dh=24, rope_dw=24,
+                                                mode=C.LA_TOKEN_CAUSAL, dtype=C.LA_F32)) == 0
+    assert C.lin_attn_uses_tensor_cores(_params(D=128, rope_dt=32, rope_dh=48, rope_dw=48,
+                                                mode=C.LA_TOKEN_CAUSAL)) == 0
+    assert C.lin_attn_uses_tensor_cores(_params(D=64, rope_dt=20, rope_dh=22, rope_dw=22,
                                                 mode=C.LA_TOKEN_CAUSAL)) == 0
 
 

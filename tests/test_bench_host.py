@@ -85,6 +85,9 @@ def test_launches_per_forward():
     assert bench.launches_per_forward(W["480p_bidir"], "bidirectional") == 2
     assert bench.launches_per_forward(W["480p_block_causal"], "block_causal") == 3
     assert bench.launches_per_forward(W["720p_long"], "block_causal") == 3
+    # token-causal: two kernels on the tensor cores (bf16, D = 64), three on CUDA cores
+    assert bench.launches_per_forward(W["480p_bidir"], "token_causal") == 2
+    assert bench.launches_per_forward(W["tiny_f32"], "token_causal") == 3
 
 
 def test_profile_traffic_lookup_is_tied_to_the_sources(tmp_path, monkeypatch):

@@ -93,6 +93,16 @@ def token_causal_cases():
            rope_split=(32, 48, 48), gate=True, modes=("token_causal",)),
         dataclasses.replace(W["480p_bidir"].scaled(1), name="tc_480p_1frame",
                             modes=("token_causal",)),
+        # tensor-core path: one 128-token tile per CTA (each CTA starts from
+        # the sum of up to 39 earlier partials of its head)
+        mk("tc_multi_cta", B=1, H=3, N=5 * 32 * 32, D=64, dtype="bf16", seed=35,
+           grid=(5, 32, 32), rope_split=(16, 24, 24), modes=("token_causal",)),
+        # ranges of one or two tiles that cross head boundaries, with the gate
+        mk("tc_span_heads_gate", B=1, H=5, N=4 * 37 * 32, D=64, dtype="bf16", seed=36,
+           grid=(4, 37, 32), rope_split=(16, 24, 24), gate=True, modes=("token_causal",)),
+        # no RoPE, a ragged last tile
+        mk("tc_no_rope", B=2, H=2, N=300, D=64, dtype="bf16", seed=37,
+           modes=("token_causal",)),
     ]
 
 
@@ -121,7 +131,7 @@ def test_token_causal_matches_oracle(w):
 
 FULL = [("480p_bidir", "bidirectional"), ("480p_block_causal", "block_causal"),
         ("720p_long", "bidirectional"), ("720p_long", "block_causal"),
-        ("gated_d128", "bidirectional")]
+        ("gated_d128", "bidirectional"), ("480p_bidir", "token_causal")]
 
 
 @pytest.mark.parametrize("name,mode", FULL)
@@ -150,6 +160,7 @@ def test_deterministic_bitwise():
     wc = W["480p_block_causal"].scaled(6)
     tc = upload(wc, workloads.make_inputs(wc))
     assert torch.equal(run_forward(wc, tc, "block_causal"), run_forward(wc, tc, "block_causal"))
+    assert torch.equal(run_forward(w, t, "token_causal"), run_forward(w, t, "token_causal"))
 
 
 def test_one_block_equals_bidirectional():
@@ -308,6 +319,9 @@ def test_tensor_core_path_is_selected_for_the_bf16_workloads():
         w = W[name]
         assert la.uses_tensor_cores(w.B, w.H, w.N, w.D, torch.bfloat16, grid=w.grid,
                                     rope_split=w.rope_split)
+    w = W["480p_bidir"]
+    assert la.uses_tensor_cores(w.B, w.H, w.N, w.D, torch.bfloat16, mode="token_causal",
+                                grid=w.grid, rope_split=w.rope_split)
     # fp32 I/O, D = 32 and RoPE widths that are not multiples of 8 use CUDA cores
     assert not la.uses_tensor_cores(1, 2, 256, 32, torch.float32)
     assert not la.uses_tensor_cores(1, 4, 60, 32, torch.bfloat16, grid=(3, 4, 5),
