@@ -12,7 +12,8 @@
 // starts a head) and walks its tiles in order, carrying the state. Per
 // 128-token chunk c, with A = RoPE(phi Q_c), Kr = RoPE(phi K_c):
 //   P      = A Kr^T                     tensor cores, fp32 in tensor memory
-//   P_m    = P with P_ij = 0 for j > i  math warps, bf16 into shared memory
+//   P_m    = P with P_ij = 0 for j > i  math warps, bf16 back into tensor
+//                                        memory (the A operand of P_m V)
 //   num    = A S_<c + P_m V_c           tensor cores (S_<c as bf16 hi + lo)
 //   S_<c+1 = S_<c + Kr^T V_c            tensor cores, fp32 in tensor memory
 //   den_i  = phi q_i . (z_<c + sum_{j <= i in c} phi k_j) + eps
@@ -35,8 +36,7 @@ constexpr uint32_t kCTile = 128 * 64 * 2;   // one 128 x 64 bf16 tile (16 KB)
 
 struct CausalPlan {
   int stages;
-  uint32_t off_pm, off_simg, off_tab, off_pos, off_den, off_wtot, off_zs, off_bar, off_tmem,
-      total;
+  uint32_t off_simg, off_tab, off_pos, off_den, off_wtot, off_zs, off_bar, off_tmem, total;
 };
 
 // barriers: full, kready, empty per stage; pfull, pm, sfull, simg, numfull[2],
@@ -47,8 +47,6 @@ __host__ __device__ inline CausalPlan causal_plan(int entries, int stages) {
   CausalPlan p;
   p.stages = stages;
   uint32_t off = stages * 3u * kCTile;         // q, k, v tiles per stage
-  p.off_pm = off;
-  off += 2u * kCTile;                          // P_m: 128 x 128 bf16, two K halves
   p.off_simg = off;
   off += 2u * 2u * 64u * 128u;                 // two S images (hi rows, lo rows)
   p.off_tab = off;
@@ -85,10 +83,26 @@ __device__ __forceinline__ void tmem_st_32x32_x16(uint32_t taddr, const uint32_t
       : "memory");
 }
 
-// S image (B operand of A S: 64 rows d, K = 64 values a, 128-byte swizzle;
-// hi rows, then lo rows 8 KB further): byte offset of (d, a).
-__device__ __forceinline__ uint32_t simg_off(int d, int a) {
-  return (uint32_t)(d * 128 + ((((a >> 3) ^ (d & 7)) & 7) << 4) + ((a & 7) << 1));
+// S image: the B operand of A S in MN-major form (64 rows a = K, 64 values d
+// = N per 128-byte row, 128-byte swizzle), hi rows then lo rows 8 KB further
+// -- the layout of the tensor-memory rows of S, so a thread owning row a
+// writes its values with 16-byte stores. Byte offset of the 16-byte chunk
+// holding d = 8 cd .. 8 cd + 7 of row a:
+__device__ __forceinline__ uint32_t simg_chunk(int a, int cd) {
+  return (uint32_t)(a * 128 + (((cd ^ (a & 7)) & 7) << 4));
+}
+
+// The 8 fp32 values v[0..7] as bf16 hi + lo (v - hi) 16-byte chunks.
+__device__ __forceinline__ void split_hilo8(const uint32_t* v, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float x = __uint_as_float(v[2 * e]), y = __uint_as_float(v[2 * e + 1]);
+    h[e] = ptx::pack_bf16x2(x, y);
+    l[e] = ptx::pack_bf16x2(x - ptx::bf16_lo(h[e]), y - ptx::bf16_hi(h[e]));
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // Warp-wide inclusive prefix sum over the lanes of 8 values.
@@ -117,12 +131,13 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   constexpr uint32_t HALF = TM * 128;           // one 64-column half of a 128-row tile
   constexpr uint32_t IDESC_P = ptx::idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(64, 64, 1, 1);
-  constexpr uint32_t IDESC_N2 = ptx::idesc_bf16_f32(128, 64, 0, 0);
+  constexpr uint32_t IDESC_N2 = ptx::idesc_bf16_f32(128, 64, 0, 1);
   constexpr uint32_t IDESC_N3 = ptx::idesc_bf16_f32(128, 64, 0, 1);
   // tensor memory columns
   constexpr uint32_t TP = 0;                    // P: 128 lanes x 128 columns
   constexpr uint32_t TNUM = 128;                // two 64-column numerator buffers
   constexpr uint32_t TS = 256;                  // S: M = 64 (lanes 0-15 of each quadrant)
+  constexpr uint32_t TPM = 320;                 // P_m: bf16 pairs, 64 columns
   constexpr uint32_t TMEM_COLS = 512;
 
   extern __shared__ uint8_t smem_raw[];
@@ -135,7 +150,6 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   float* s_den = reinterpret_cast<float*>(sm + P.off_den);
   float* s_wtot = reinterpret_cast<float*>(sm + P.off_wtot);
   float* s_zs = reinterpret_cast<float*>(sm + P.off_zs);
-  const uint32_t pm_base = base + P.off_pm;
   const uint32_t simg_base = base + P.off_simg;
   const uint32_t bar0 = base + P.off_bar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -249,17 +263,17 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t adesc = ptx::smem_desc_sw128(qt + kk * 32, 16, 1024);
-          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(simg + kk * 32, 16, 1024), IDESC_N2,
+          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(simg + kk * 2048, 8192, 1024), IDESC_N2,
                         kk ? 1u : 0u);
-          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(simg + 8192 + kk * 32, 16, 1024),
+          ptx::mma_bf16(acc, adesc, ptx::smem_desc_sw128(simg + 8192 + kk * 2048, 8192, 1024),
                         IDESC_N2, 1u);
         }
         if (!wait_bounded(pm_bar, cph, flag, kFlagApplyTimeout, &s_abort)) break;
         ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          ptx::mma_bf16(acc, ptx::smem_desc_sw128(pm_base + (kk / 4) * HALF + (kk % 4) * 32, 16, 1024),
-                        ptx::smem_desc_sw128(vt + kk * 2048, HALF, 1024), IDESC_N3, 1u);
+          ptx::mma_bf16_ta(acc, tmem + TPM + 8u * kk,
+                           ptx::smem_desc_sw128(vt + kk * 2048, HALF, 1024), IDESC_N3, 1u);
         ptx::mma_commit(numfull_bar(b));
         ptx::mma_commit(empty_bar(it.stage));
       }
@@ -292,27 +306,43 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       const float* pbase = partials + (long long)seg0 * sc.maxc * DD1;
       // S rows a = 16 q4 + lane (lanes 0-15), columns d = 16 jw .. 16 jw + 15
       const int a = 16 * q4 + (lane & 15);
+      // S[a][d] = column d of S, row a (at d * D + a of a partial): the 16
+      // loads of a partial in flight together, the partials added in order
+      float acc[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+      float zacc = 0.f;
+      for (int k = 0; k < np; ++k) {
+        const float* pk = pbase + (long long)k * DD1 + a;
+        float t[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) t[e] = __ldcg(pk + (16 * jw + e) * D);
+        const float tz = jw == 0 ? __ldcg(pk + D * D) : 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] += t[e];
+        zacc += tz;
+      }
       uint32_t sv[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int d = 16 * jw + e;
-        float s = 0.f;
-        for (int k = 0; k < np; ++k) s += __ldcg(pbase + (long long)k * DD1 + d * D + a);
-        sv[e] = __float_as_uint(s);
-        if (lane < 16) {
-          const uint32_t h = ptx::pack_bf16x2(s, 0.f) & 0xFFFFu;
-          const float lo = s - ptx::bf16_lo(h);
-          const uint32_t l = ptx::pack_bf16x2(lo, 0.f) & 0xFFFFu;
-          uint8_t* img = sm + P.off_simg + 16384u;   // image of the start state: buffer 1
-          *reinterpret_cast<uint16_t*>(img + simg_off(d, a)) = (uint16_t)h;
-          *reinterpret_cast<uint16_t*>(img + 8192 + simg_off(d, a)) = (uint16_t)l;
+      for (int e = 0; e < 16; ++e) sv[e] = __float_as_uint(acc[e]);
+      if (lane < 16) {
+        uint8_t* img = sm + P.off_simg + 16384u;   // image of the start state: buffer 1
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint4 hi, lo;
+          split_hilo8(sv + 8 * h, hi, lo);
+          *reinterpret_cast<uint4*>(img + simg_chunk(a, 2 * jw + h)) = hi;
+          *reinterpret_cast<uint4*>(img + 8192 + simg_chunk(a, 2 * jw + h)) = lo;
         }
+        if (jw == 0) s_zs[a] = zacc;
       }
       tmem_st_32x32_x16(tmem + lane_bits + TS + 16u * jw, sv);
-      if (tt < D) {
-        float z = 0.f;
-        for (int k = 0; k < np; ++k) z += __ldcg(pbase + (long long)k * DD1 + D * D + tt);
-        s_zs[tt] = z;
+      // the blocks of P_m above the diagonal block row stay zero
+      if (jw > q4) {
+        uint32_t zero[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) zero[e] = 0u;
+        tmem_st_32x32_x16(tmem + lane_bits + TPM + 16u * jw, zero);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -445,11 +475,8 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       {
         const bool rdy = wait_bounded(pfull_bar, cph, flag, kFlagApplyTimeout, &s_abort);
         ptx::tc_fence_after();
-        const int row = 32 * q4 + lane;
-        const uint32_t h = (uint32_t)(jw >> 1);
-        uint32_t pk2[16];
         if (jw <= q4) {
-          uint32_t pv[32];
+          uint32_t pv[32], pk2[16];
           tmem_ld_cols<32>(tmem + lane_bits + TP + 32u * jw, pv);
           ptx::tmem_wait_ld();
 #pragma unroll
@@ -461,20 +488,11 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             }
             pk2[e] = ptx::pack_bf16x2(p0, p1);
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk2[e] = 0u;
+          tmem_st_32x32_x16(tmem + lane_bits + TPM + 16u * jw, pk2);
+          ptx::tmem_wait_st();
         }
         (void)rdy;
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int chunk = (jw & 1) * 4 + k4;
-          const uint32_t off = h * HALF + row * 128 + ((chunk ^ (row & 7)) << 4);
-          ptx::st_shared_v4(pm_base + off, make_uint4(pk2[4 * k4], pk2[4 * k4 + 1],
-                                                      pk2[4 * k4 + 2], pk2[4 * k4 + 3]));
-        }
         ptx::tc_fence_before();
-        ptx::fence_proxy_async();
         ptx::mbar_arrive(pm_bar);
       }
       // ---- D: image of the state after this chunk (or the zero state when the
@@ -497,13 +515,11 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           const int a = 16 * q4 + lane;
           uint8_t* img = sm + P.off_simg + (uint32_t)b * 16384u;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int d = 16 * jw + e;
-            const float s = __uint_as_float(sv[e]);
-            const uint32_t hw = ptx::pack_bf16x2(s, 0.f) & 0xFFFFu;
-            const uint32_t lw = ptx::pack_bf16x2(s - ptx::bf16_lo(hw), 0.f) & 0xFFFFu;
-            *reinterpret_cast<uint16_t*>(img + simg_off(d, a)) = (uint16_t)hw;
-            *reinterpret_cast<uint16_t*>(img + 8192 + simg_off(d, a)) = (uint16_t)lw;
+          for (int h = 0; h < 2; ++h) {
+            uint4 hi, lo;
+            split_hilo8(sv + 8 * h, hi, lo);
+            *reinterpret_cast<uint4*>(img + simg_chunk(a, 2 * jw + h)) = hi;
+            *reinterpret_cast<uint4*>(img + 8192 + simg_chunk(a, 2 * jw + h)) = lo;
           }
         }
         if (restart) {
