@@ -54,7 +54,7 @@ __host__ __device__ inline CausalPlan causal_plan(int entries, int stages) {
   p.off_pos = off;
   off = align_up(off + (entries ? stages * 3u * 128u * 2u : 0u), 16);
   p.off_den = off;
-  off += 2u * 128u * 8u * 4u;                  // denominator parts [buf][row][chunk col]
+  off += 3u * 128u * 8u * 4u;                  // denominator parts [chunk % 3][row][col]
   p.off_wtot = off;
   off += 2u * 2u * 8u * 8u * 4u;               // key-sum totals [buf][row half][col][8]
   p.off_zs = off;
@@ -369,8 +369,9 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       const int row = 32 * q4 + lane;
       const int r = ptile * TM + row;
       if (rdy && r < L) {
-        const float4 d0 = *reinterpret_cast<const float4*>(s_den + (eb * TM + row) * 8);
-        const float4 d1 = *reinterpret_cast<const float4*>(s_den + (eb * TM + row) * 8 + 4);
+        const int dbuf = pc % 3;
+        const float4 d0 = *reinterpret_cast<const float4*>(s_den + (dbuf * TM + row) * 8);
+        const float4 d1 = *reinterpret_cast<const float4*>(s_den + (dbuf * TM + row) * 8 + 4);
         const float den = eps + (((d0.x + d0.y) + (d0.z + d0.w)) + ((d1.x + d1.y) + (d1.z + d1.w)));
         const float inv = 1.f / den;
         const uint64_t inv2 = ptx::f2(inv, inv);
@@ -409,14 +410,18 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         gv[1] = __ldg(src + 1);
       }
     };
-    long long c = 0;
-    for (long long u = u0; u < u1; ++u, ++c) {
-      const int b = (int)(c & 1);
-      const uint32_t cph = (uint32_t)(c & 1);
-      const int seg = it.seg, tile = it.tile, stage = it.stage;
+    // ---- A(ca): RoPE(phi q), RoPE(phi k) in place for chunk ca (the TMA
+    // stage of itA); running key sums and the chunk's denominators ----
+    TileIter itA = it;
+    auto transform = [&](long long ca) {
+      const int stage = itA.stage;
       const uint32_t qt = base + stage * 3u * kCTile, kt = qt + kCTile;
-      // ---- A: RoPE(phi q), RoPE(phi k) in place; running key sums, denominators ----
-      const bool ok = wait_bounded(full_bar(stage), it.phase, flag, kFlagApplyTimeout, &s_abort);
+      if (itA.tile == 0) {   // a head starts: no earlier keys
+#pragma unroll
+        for (int e = 0; e < 8; ++e) zr[e] = 0.f;
+      }
+      const bool ok = wait_bounded(full_bar(stage), itA.phase, flag, kFlagApplyTimeout, &s_abort);
+      (void)ok;
       float pq[2][8], pk[2][8];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -443,19 +448,19 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       }
       ptx::fence_proxy_async();
       ptx::mbar_arrive(kready_bar(stage));
-      (void)ok;
       // inclusive key sums down this warp's 64 rows, then across the two halves
+      const int wb = (int)(ca & 1);
       warp_scan8(pk[0], lane);
       warp_scan8(pk[1], lane);
-      float* wt = s_wtot + ((b * 2 + rh) * 8 + cc) * 8;
+      float* wt = s_wtot + ((wb * 2 + rh) * 8 + cc) * 8;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         pk[1][e] += __shfl_sync(0xffffffffu, pk[0][e], 31);
         if (lane == 31) wt[e] = pk[1][e];
       }
       ptx::bar_sync(2, kMath);
-      const float* w0 = s_wtot + ((b * 2 + 0) * 8 + cc) * 8;
-      const float* w1 = s_wtot + ((b * 2 + 1) * 8 + cc) * 8;
+      const float* w0 = s_wtot + ((wb * 2 + 0) * 8 + cc) * 8;
+      const float* w1 = s_wtot + ((wb * 2 + 1) * 8 + cc) * 8;
       float dq[2] = {0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -464,8 +469,20 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         dq[1] = fmaf(pq[1][e], base_e + pk[1][e], dq[1]);
         zr[e] += w0[e] + w1[e];
       }
+      const int db = (int)(ca % 3);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) s_den[(b * TM + 64 * rh + 32 * i + lane) * 8 + cc] = dq[i];
+      for (int i = 0; i < 2; ++i) s_den[(db * TM + 64 * rh + 32 * i + lane) * 8 + cc] = dq[i];
+      itA.next();
+    };
+
+    const long long nch = u1 - u0;
+    transform(0);
+    for (long long c = 0; c < nch; ++c) {
+      const int b = (int)(c & 1);
+      const uint32_t cph = (uint32_t)(c & 1);
+      const int seg = it.seg, tile = it.tile;
+      // the next chunk's transform while the tensor cores finish this one
+      if (c + 1 < nch) transform(c + 1);
       // ---- B: the previous chunk's epilogue ----
       if (pend >= 0) {
         load_gate(pend_seg, pend_tile);
@@ -521,10 +538,6 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             *reinterpret_cast<uint4*>(img + simg_chunk(a, 2 * jw + h)) = hi;
             *reinterpret_cast<uint4*>(img + 8192 + simg_chunk(a, 2 * jw + h)) = lo;
           }
-        }
-        if (restart) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) zr[e] = 0.f;
         }
         ptx::tc_fence_before();
         ptx::fence_proxy_async();
