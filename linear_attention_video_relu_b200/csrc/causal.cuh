@@ -54,7 +54,7 @@ __host__ __device__ inline CausalPlan causal_plan(int entries, int stages) {
   p.off_pos = off;
   off = align_up(off + (entries ? stages * 3u * 128u * 2u : 0u), 16);
   p.off_den = off;
-  off += 3u * 128u * 8u * 4u;                  // denominator parts [chunk % 3][row][col]
+  off += 3u * 8u * 128u * 4u;                  // denominator parts [chunk % 3][col][row]
   p.off_wtot = off;
   off += 2u * 2u * 8u * 8u * 4u;               // key-sum totals [buf][row half][col][8]
   p.off_zs = off;
@@ -369,10 +369,13 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       const int row = 32 * q4 + lane;
       const int r = ptile * TM + row;
       if (rdy && r < L) {
-        const int dbuf = pc % 3;
-        const float4 d0 = *reinterpret_cast<const float4*>(s_den + (dbuf * TM + row) * 8);
-        const float4 d1 = *reinterpret_cast<const float4*>(s_den + (dbuf * TM + row) * 8 + 4);
-        const float den = eps + (((d0.x + d0.y) + (d0.z + d0.w)) + ((d1.x + d1.y) + (d1.z + d1.w)));
+        // the 8 chunk columns' parts of this row's denominator (column-major:
+        // consecutive rows in consecutive banks)
+        const float* dp = s_den + (pc % 3) * 8 * TM + row;
+        float dv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dv[e] = dp[e * TM];
+        const float den = eps + (((dv[0] + dv[1]) + (dv[2] + dv[3])) + ((dv[4] + dv[5]) + (dv[6] + dv[7])));
         const float inv = 1.f / den;
         const uint64_t inv2 = ptx::f2(inv, inv);
         uint4* dst = reinterpret_cast<uint4*>(out + scd.out_row(pseg, L, r, D) + 16 * jw);
@@ -471,7 +474,7 @@ causal_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       }
       const int db = (int)(ca % 3);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) s_den[(db * TM + 64 * rh + 32 * i + lane) * 8 + cc] = dq[i];
+      for (int i = 0; i < 2; ++i) s_den[(db * 8 + cc) * TM + 64 * rh + 32 * i + lane] = dq[i];
       itA.next();
     };
 
