@@ -52,6 +52,10 @@ def parse_args():
                     choices=["bidirectional", "block_causal", "token_causal"])
     ap.add_argument("--settle", type=int, default=50,
                     help="untimed forwards before the timed region (clock settling)")
+    ap.add_argument("--only", default=None,
+                    help="run one secondary measurement alone (for profiling runs) and print "
+                         "its line, e.g. 480p_bidir_x_text300/cross, 480p_hidden_tconv, "
+                         "480p_2b_d112/bidirectional, 480p_bidir/token_causal")
     return ap.parse_args()
 
 
@@ -117,15 +121,23 @@ def measured_peaks():
 _NOT_TC_SOURCES = ("simt.cuh", "tconv.cu")
 
 
-def kernel_source_hash() -> str:
-    """Hash of the tensor-core kernels' sources (every CUDA source but the
-    CUDA-core kernels, host launch code included) with comments and whitespace
-    removed, so that a committed traffic figure stays tied to the code it was
-    measured on, not to its comments or to other kernels."""
+def _source_selected(name: str, kind: str) -> bool:
+    if kind == "tconv":
+        return name == "tconv.cu"
+    return name not in _NOT_TC_SOURCES
+
+
+def kernel_source_hash(kind: str = "tc") -> str:
+    """Hash of a kernel family's sources with comments and whitespace removed,
+    so that a committed traffic figure stays tied to the code it was measured
+    on, not to its comments or to other kernels. kind "tc": the attention
+    kernels (every CUDA source but the CUDA-core kernels and the temporal
+    convolution, host launch code included); "tconv": the temporal
+    convolution's translation unit."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_video_relu_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")) and name not in _NOT_TC_SOURCES:
+        if name.endswith((".cu", ".cuh")) and _source_selected(name, kind):
             with open(os.path.join(csrc, name)) as f:
                 text = f.read()
             text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -140,7 +152,7 @@ def ncu_traffic(kernel: str, workload: str):
     the current kernel sources (a line '# bench-traffic <kernel> <workload>
     <bytes> <source-hash>' in profiles/*.txt); else None."""
     pdir = os.path.join(ROOT, "profiles")
-    want = kernel_source_hash()
+    want = kernel_source_hash("tconv" if kernel == "temporal_conv" else "tc")
     if not os.path.isdir(pdir):
         return None
     for name in sorted(os.listdir(pdir)):
@@ -309,9 +321,10 @@ def measure_workload(w, mode, steps, warmup, pg, device, peak, peak_kind, seed):
         apply_bytes += 2 * tensor_bytes
         total_bytes += 2 * tensor_bytes
     step_ms = ms / steps
-    k_state = roofline_entry("state_build", state_bytes, kern[0], peak, peak_kind, w.name)
+    key = w.name if mode == "bidirectional" else "%s/%s" % (w.name, mode)
+    k_state = roofline_entry("state_build", state_bytes, kern[0], peak, peak_kind, key)
     k_reduce_us = round(sum(kern[1]) / len(kern[1]) * 1e3, 2)
-    k_apply = roofline_entry("apply", apply_bytes, kern[2], peak, peak_kind, w.name)
+    k_apply = roofline_entry("apply", apply_bytes, kern[2], peak, peak_kind, key)
     res = {
         "workload": w.name, "mode": mode, "ms_per_step": step_ms,
         "tokens_per_s": w.B * w.N / (step_ms * 1e-3),
@@ -397,10 +410,13 @@ def measure_cross(w, n_kv, steps, warmup, device, peak, seed):
     ms = a.elapsed_time(b) / steps
     nbytes = 2 * 2 * w.B * w.H * (w.N + n_kv) * w.D     # read q, k, v; write out (bf16)
     del q, k, v, out
-    return {"workload": "%s_x_text%d" % (w.name, n_kv), "mode": "cross", "n_kv": n_kv,
+    name = "%s_x_text%d" % (w.name, n_kv)
+    t_sb, t_ap = ncu_traffic("state_build", name), ncu_traffic("apply", name)
+    return {"workload": name, "mode": "cross", "n_kv": n_kv,
             "us_per_forward": ms * 1e3, "tokens_per_s": w.B * w.N / (ms * 1e-3),
             "algorithmic_bytes": nbytes, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
-            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peak}
+            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peak,
+            "traffic": (t_sb + t_ap) if (t_sb is not None and t_ap is not None) else None}
 
 
 def measure_tconv(steps, warmup, device, peak, seed):
@@ -439,7 +455,8 @@ def measure_tconv(steps, warmup, device, peak, seed):
     return {"workload": "480p_hidden_tconv", "mode": "temporal_conv_cached",
             "shape": [B, T, S, nc], "us_per_call": ms * 1e3,
             "tokens_per_s": B * T * S / (ms * 1e-3), "algorithmic_bytes": nbytes,
-            "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peak}
+            "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peak,
+            "traffic": ncu_traffic("temporal_conv", "480p_hidden_tconv")}
 
 
 def measure_e2e(w, steps, device, seed):
@@ -568,24 +585,34 @@ W_2B_480P = workloads.Workload("480p_2b_d112", B=1, H=20, N=21 * 30 * 52, D=112,
 def secondary_lines(K, device, peak, peak_kind):
     """The other workloads and rows, each timed on its own; a line that fails
     records its error instead of ending the run."""
+    return run_jobs(secondary_jobs(K, device, peak, peak_kind))
+
+
+def secondary_jobs(K, device, peak, peak_kind, warmup=3):
+    """(name, measurement) of every secondary line, K timed steps each."""
     jobs = []
     for name, mode in (("480p_block_causal", "block_causal"), ("720p_long", "bidirectional"),
                        ("720p_long", "block_causal"), ("gated_d128", "bidirectional"),
                        ("480p_bidir", "token_causal")):
         ww = workloads.WORKLOADS[name]
         jobs.append((name + "/" + mode,
-                     lambda ww=ww, mode=mode: measure_workload(ww, mode, K, 3, None, device, peak,
-                                                               peak_kind, ww.seed)))
+                     lambda ww=ww, mode=mode: measure_workload(ww, mode, K, warmup, None, device,
+                                                               peak, peak_kind, ww.seed)))
     jobs.append(("480p_2b_d112/bidirectional",
-                 lambda: measure_workload(W_2B_480P, "bidirectional", K, 3, None, device, peak,
+                 lambda: measure_workload(W_2B_480P, "bidirectional", K, warmup, None, device, peak,
                                           peak_kind, W_2B_480P.seed)))
     jobs.append(("480p_bidir_x_text300/cross",
-                 lambda: measure_cross(workloads.WORKLOADS["480p_bidir"], 300, K, 5, device,
-                                       peak, 2002)))
-    jobs.append(("480p_hidden_tconv", lambda: measure_tconv(K, 5, device, peak, 2003)))
+                 lambda: measure_cross(workloads.WORKLOADS["480p_bidir"], 300, K, max(warmup, 1),
+                                       device, peak, 2002)))
+    jobs.append(("480p_hidden_tconv",
+                 lambda: measure_tconv(K, max(warmup, 1), device, peak, 2003)))
     jobs.append(("720p_long_block_step",
-                 lambda: measure_block_steps(workloads.WORKLOADS["720p_long"], 120, 60, device,
-                                             peak, peak_kind, 1004)))
+                 lambda: measure_block_steps(workloads.WORKLOADS["720p_long"], max(K, 60),
+                                             max(warmup, 60), device, peak, peak_kind, 1004)))
+    return jobs
+
+
+def run_jobs(jobs):
     out = []
     for name, job in jobs:
         try:
@@ -612,11 +639,16 @@ def compact(r: dict) -> dict:
         c["tok_s"] = float("%.4g" % r["tokens_per_s"])
     if "hbm_frac" in r:
         c["frac"] = round(r["hbm_frac"], 4)
+    mb = lambda t: None if t is None else round(t / 1e6, 1)
     k = r.get("kernels")
     if k:
-        c["sb"] = [k["state_build"]["avg_us"], k["state_build"]["frac"]]
-        c["ap"] = [k["apply"]["avg_us"], k["apply"]["frac"]]
+        # [event-timed us, roofline fraction, ncu DRAM MB per launch or null]
+        c["sb"] = [k["state_build"]["avg_us"], k["state_build"]["frac"],
+                   mb(k["state_build"].get("traffic"))]
+        c["ap"] = [k["apply"]["avg_us"], k["apply"]["frac"], mb(k["apply"].get("traffic"))]
         c["red_us"] = k["reduce_us"]
+    if "traffic" in r:
+        c["traffic_MB"] = mb(r["traffic"])
     return c
 
 
@@ -646,6 +678,18 @@ def main():
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     peak, peak_kind = measured_peaks()
+    if args.only:
+        # one secondary line alone (profiling runs)
+        jobs = [j for j in secondary_jobs(args.steps, device, peak, peak_kind, args.warmup)
+                if j[0] == args.only]
+        if not jobs:
+            raise SystemExit("unknown --only job %r" % args.only)
+        if rank == 0:
+            print(json.dumps(run_jobs(jobs)[0]), flush=True)
+        if pg is not None:
+            barrier(pg, device)
+            pg.destroy_process_group()
+        return
     w = workloads.WORKLOADS[args.workload]
     mode = args.mode
 

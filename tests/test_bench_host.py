@@ -149,8 +149,8 @@ def test_secondary_lines_record_errors(monkeypatch):
 def test_secondary_lines_are_short():
     # every secondary result is reduced to a few short keys, so that ten of
     # them fit in the last ~3 KB of the bench output
-    kern = lambda us, f: {"avg_us": us, "frac": f, "kernel": "x", "bound": "hbm",
-                          "achieved": 1.0, "peak": 6535.7, "unit": "GB/s", "traffic": None,
+    kern = lambda us, f, t=None: {"avg_us": us, "frac": f, "kernel": "x", "bound": "hbm",
+                          "achieved": 1.0, "peak": 6535.7, "unit": "GB/s", "traffic": t,
                           "algorithmic_bytes": 1, "peak_source": "measured"}
     full = {"workload": "720p_long", "mode": "block_causal", "ms_per_step": 0.69123456,
             "tokens_per_s": 319876543.21, "hbm_gbs": 5234.5678, "hbm_frac": 0.80098765,
@@ -158,8 +158,8 @@ def test_secondary_lines_are_short():
                         "apply": kern(320.5, 0.8123)}}
     c = bench.compact(full)
     assert c["w"] == "720p_long" and c["mode"] == "block_causal"
-    assert c["ms"] == 0.6912 and c["frac"] == 0.801 and c["sb"] == [350.123, 0.7712]
-    assert c["ap"] == [320.5, 0.8123] and c["red_us"] == 14.2
+    assert c["ms"] == 0.6912 and c["frac"] == 0.801 and c["sb"] == [350.123, 0.7712, None]
+    assert c["ap"] == [320.5, 0.8123, None] and c["red_us"] == 14.2
     cross = {"workload": "480p_bidir_x_text300", "mode": "cross", "n_kv": 300,
              "us_per_forward": 61.66, "tokens_per_s": 5.3e8, "algorithmic_bytes": 1,
              "hbm_gbs": 4392.1, "hbm_frac": 0.672}
@@ -167,4 +167,33 @@ def test_secondary_lines_are_short():
            "tokens_per_s": 1.19e8, "hbm_frac": 0.2986}
     lines = [bench.compact(r) for r in (full, cross, blk)]
     assert lines[1]["us"] == 61.66 and lines[2]["us_blk"] == 30.9
+    full["kernels"]["apply"] = kern(320.5, 0.8123, 272841984)
+    assert bench.compact(full)["ap"] == [320.5, 0.8123, 272.8]
+    assert bench.compact(dict(cross, traffic=270900000))["traffic_MB"] == 270.9
     assert all(len(json.dumps(l)) < 200 for l in lines)
+
+
+def test_only_selects_one_secondary_job():
+    names = [n for n, _ in bench.secondary_jobs(5, None, 6535.7, "measured")]
+    assert len(names) == len(set(names)) == 9
+    for n in ("480p_bidir_x_text300/cross", "480p_hidden_tconv", "480p_2b_d112/bidirectional",
+              "480p_bidir/token_causal"):
+        assert n in names
+
+
+def test_traffic_of_the_temporal_conv_follows_its_own_source(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    csrc = tmp_path / "linear_attention_video_relu_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "tc.cuh").write_text("int a;\n")
+    (csrc / "tconv.cu").write_text("int b;\n")
+    ht, hc = bench.kernel_source_hash("tconv"), bench.kernel_source_hash()
+    assert ht != hc
+    (tmp_path / "profiles" / "t.txt").write_text(
+        "# bench-traffic temporal_conv 480p_hidden_tconv 300 %s\n" % ht)
+    assert bench.ncu_traffic("temporal_conv", "480p_hidden_tconv") == 300
+    (csrc / "tc.cuh").write_text("int a; int c;\n")      # other kernels change: still valid
+    assert bench.ncu_traffic("temporal_conv", "480p_hidden_tconv") == 300
+    (csrc / "tconv.cu").write_text("int b; int d;\n")    # its own source changes: stale
+    assert bench.ncu_traffic("temporal_conv", "480p_hidden_tconv") is None
