@@ -137,9 +137,12 @@ LA_API la_status lin_attn_block_step_workspace_size(const la_params* p, size_t* 
  *                  is Algorithm 1 run with an empty initial cache.
  *   token-causal:  out_i uses S, z summed over tokens 0..i of its head (the
  *                  causal form, Eq. 3 of "Block Linear Attention with
- *                  Constant-Memory KV Cache"). Runs on the CUDA-core
- *                  kernels: chunks of 32 tokens, the running sums over
- *                  earlier chunks plus the masked sums inside the chunk.
+ *                  Constant-Memory KV Cache"). bf16 at D = 64 (RoPE
+ *                  widths multiples of 8) runs on the tensor cores: each
+ *                  CTA starts from the sums over the tokens before its
+ *                  range and walks it in chunks of 128 tokens, adding the
+ *                  masked in-chunk products and carrying the state. Other
+ *                  shapes run on the CUDA-core kernels in chunks of 32.
  * q, k, v, out: [B,H,N,D] device pointers in p->dtype. gate: NULL or the same
  * shape and dtype (logits; out is multiplied by their sigmoid).
  * workspace: device memory of at least lin_attn_workspace_size bytes, 256-byte
@@ -261,9 +264,9 @@ LA_API la_status lin_attn_device_status(void* workspace, void* stream);
 LA_API const char* lin_attn_status_string(la_status s);
 
 /* Which kernel family lin_attn_forward would use for `p` on the current
- * device: 1 = tensor-core (tcgen05 + TMA, bf16 I/O, D in {64, 128}),
- * 0 = CUDA-core (fp32 I/O, token-causal mode, or shapes outside the
- * tensor-core path). */
+ * device: 1 = tensor-core (tcgen05 + TMA, bf16 I/O, D in {64, 112, 128}),
+ * 0 = CUDA-core (fp32 I/O, token-causal mode other than bf16 at D = 64,
+ * or shapes outside the tensor-core path). */
 LA_API int lin_attn_uses_tensor_cores(const la_params* p);
 
 /* ---- Mix-FFN temporal convolution with the last-frame cache -------------

@@ -519,16 +519,41 @@ __device__ void reduce_segment(const float* __restrict__ partials, const Sched& 
   }
 }
 
+// The carried-state values of reduction item `item` (4 consecutive K-values
+// a0.. of row n of the transposed state; n = D is z), or zeros.
+template <int D>
+__device__ __forceinline__ void carried4(const float* gS, const float* gz, int use_state,
+                                         int item, float (&r)[4]) {
+  constexpr int QPR = D / 4, ITEMS = (D + 1) * QPR;
+  const int n = item / QPR;
+  const int a0 = 4 * (item - n * QPR);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) r[e] = 0.f;
+  if (use_state && item < ITEMS) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) r[e] = n == D ? gz[a0 + e] : gS[(a0 + e) * D + n];
+  }
+}
+
 // reduce_segment over np partial slots already copied to shared memory
 // (slot i at sp + i * D(D + 1)): the same fp32 operations in the same order.
+// `first` holds the carried-state values of the thread's first item (loaded
+// by the caller while the partials were being copied); each next item's are
+// loaded while the thread works on the current one, so the global loads
+// overlap instead of costing a round trip per item.
 template <int D>
 __device__ void reduce_segment_smem(const float* sp, int np, int seg,
                                     uint8_t* __restrict__ images, float* __restrict__ stS,
                                     float* __restrict__ stz, int use_state, int commit, int tid,
-                                    int nthr) {
+                                    int nthr, const float (&first)[4]) {
   constexpr int DD = D * D, DD1 = D * (D + 1), QPR = D / 4, ITEMS = (D + 1) * QPR;
   uint8_t* img = images + (long long)seg * image_bytes(D);
+  float* gS = use_state ? stS + (long long)seg * DD : nullptr;
+  float* gz = use_state ? stz + (long long)seg * D : nullptr;
+  float nxt[4] = {first[0], first[1], first[2], first[3]};
   for (int item = tid; item < ITEMS; item += nthr) {
+    const float cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+    carried4<D>(gS, gz, use_state, item + nthr, nxt);
     const int n = item / QPR;
     const int a0 = 4 * (item - n * QPR);
     const bool zrow = n == D;
@@ -536,22 +561,14 @@ __device__ void reduce_segment_smem(const float* sp, int np, int seg,
     float4 acc = *reinterpret_cast<const float4*>(sp + off);
     for (int i = 1; i < np; ++i)
       acc = add4(acc, *reinterpret_cast<const float4*>(sp + (long long)i * DD1 + off));
-    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (use_state) {
-      float r[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        r[e] = zrow ? stz[(long long)seg * D + a0 + e] : stS[(long long)seg * DD + (a0 + e) * D + n];
-      run = make_float4(r[0], r[1], r[2], r[3]);
-    }
-    run = add4(run, acc);
+    const float4 run = add4(make_float4(cur[0], cur[1], cur[2], cur[3]), acc);
     store_image4<D>(img + image_offset<D>(n, a0), zrow, a0, run);
     if (use_state && commit) {
       const float r[4] = {run.x, run.y, run.z, run.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        if (zrow) stz[(long long)seg * D + a0 + e] = r[e];
-        else stS[(long long)seg * DD + (a0 + e) * D + n] = r[e];
+        if (zrow) gz[a0 + e] = r[e];
+        else gS[(a0 + e) * D + n] = r[e];
       }
     }
   }
@@ -636,15 +653,19 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     ptx::tmem_relinquish();
   }
   __syncthreads();
-  if (threadIdx.x == 0) ptx::launch_dependents();
   // Launched early (programmatic dependent launch) behind the previous
   // kernel of the stream: k and v are read, and the workspace is written,
   // only after griddepcontrol.wait (by the TMA warp before its loads, by the
   // math warps before the table goes out; everything else follows the loads).
+  // The kernel lets its own dependent (the apply kernel) launch only once it
+  // is past that wait: the apply kernel then knows that everything before
+  // this kernel in the stream has completed, and reads its q (and gate)
+  // tiles before its own wait.
 
   if (warp == 0) {
     // ---------------- TMA producer (+ row offsets of the RoPE table) ----------------
     ptx::grid_dependency_wait();
+    if (lane == 0) ptx::launch_dependents();
     TileIter it;
     it.init(u0, sc.tps, stages);
     long long issued = 0;
@@ -864,12 +885,12 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     ptx::tmem_dealloc(*s_tmem, TMEM_COLS);
   }
   if (s_npend > 0 && !s_abort) {
-    // At D = 128 (six partial rows per thread) the drained stage ring takes
-    // up to `cap` partial slots: bulk-copy a segment's partials there at once
-    // and reduce them from shared memory. At D = 64 the register path, with
-    // fewer rows per thread, is as fast.
+    // The drained stage ring (with the tables behind it) takes up to `cap`
+    // partial slots: bulk-copy a segment's partials there at once and reduce
+    // them from shared memory -- one round trip to L2 for all of them instead
+    // of one per row group of each thread.
     constexpr uint32_t SLOT = DD1 * 4;
-    const int cap = D == 128 ? (int)(P.off_bar / SLOT) : 0;
+    const int cap = (int)(P.off_bar / SLOT);
     __threadfence();
     uint32_t tph = 0;
     for (int k = 0; k < s_npend; ++k) {
@@ -887,11 +908,14 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           ptx::bulk_load(base + (uint32_t)i * SLOT,
                          partials + ((long long)seg * sc.maxc + i) * DD1, SLOT, tail_bar);
       }
+      float first[4];
+      carried4<D>(use_state ? stS + (long long)seg * D * D : nullptr,
+                  use_state ? stz + (long long)seg * D : nullptr, use_state, threadIdx.x, first);
       const bool got = wait_bounded(tail_bar, tph, flag, kFlagStateTimeout, &s_abort);
       if (!__syncthreads_and(got)) break;   // every thread leaves together
       tph ^= 1u;
       reduce_segment_smem<D>(reinterpret_cast<const float*>(sm), np, seg, images, stS, stz,
-                             use_state, commit, threadIdx.x, kTcThreadsState);
+                             use_state, commit, threadIdx.x, kTcThreadsState, first);
       __syncthreads();   // before the next segment's copies overwrite the slots
     }
   }
@@ -1018,7 +1042,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
          const __grid_constant__ CUtensorMap tm_o, __nv_bfloat16* __restrict__ out, int ocols,
          const __grid_constant__ Rope rope, int L, int nblk,
          const __grid_constant__ SegCoords scd, long long U, int stages, int sbuf, int gst, const uint8_t* __restrict__ images,
-         const float2* __restrict__ gtab, float eps, int* flag) {
+         const float2* __restrict__ gtab, float eps, int* flag, int early) {
   constexpr int TM = kApplyTile;
   constexpr int HALVES = D / 64;
   constexpr int HALF_BYTES = TM * 128;
@@ -1096,9 +1120,14 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   }
   __syncthreads();
   if (threadIdx.x == 0) ptx::launch_dependents();
-  // launched early (programmatic dependent launch): the images and the RoPE
-  // table are read only after the kernels that write them have completed
-  ptx::grid_dependency_wait();
+  // Launched early (programmatic dependent launch) behind the kernel that
+  // writes its images (the state build, or the separate reduction), which
+  // lets it launch only once past its own dependency wait: everything before
+  // that kernel in the stream -- q and the gate among it -- is complete. So
+  // q (and gate) tiles of the first `early` stages may be loaded, and (with a
+  // RoPE table built here) transformed, while that kernel still runs; the
+  // images, and otherwise the state build's RoPE table, are read only after
+  // griddepcontrol.wait.
 
   if (warp == 0) {
     // ---------------- TMA loads: S images per segment, q (and gate) tiles ----------------
@@ -1106,7 +1135,41 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     it.init(u0, tps, stages);
     long long issued = 0;
     int cur_seg = -1, ss = -1;
-    for (long long u = u0; u < u1; ++u, it.next()) {
+    // q (and gate) tiles into stage it.stage once it is free
+    auto load_q = [&](const TileIter& t) -> bool {
+      int ok = 1;
+      if (lane == 0)
+        ok = wait_bounded(empty_bar(t.stage), t.phase ^ 1u, flag, kFlagApplyTimeout, &s_abort);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+      if (ROPE) {
+        const int blk = t.seg - (t.seg / nblk) * nblk;
+        write_row_offsets(rope, s_pos + t.stage * 3 * TM, TM, blk * L + t.tile * TM, lane);
+        __syncwarp();
+      }
+      if (lane == 0) {
+        ptx::mbar_expect_tx(full_bar(t.stage), TX);
+        const int3 c = scd.of(t.seg, t.tile * TM);
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h) {
+          ptx::tma_load_4d(base + t.stage * TILE_BYTES + h * HALF_BYTES, &tm_q, 64 * h, c.x,
+                           c.y, c.z, full_bar(t.stage));
+          if (!DIRECT && GATE)
+            ptx::tma_load_4d(gbase + t.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h, c.x,
+                             c.y, c.z, full_bar(t.stage));
+        }
+      }
+      ++issued;
+      return true;
+    };
+    // `early` stages go out before the wait (the host's choice, by measure)
+    const long long pre = u1 - u0 < early ? u1 - u0 : early;
+    bool pre_ok = true;
+    {
+      TileIter ip = it;
+      for (long long k = 0; k < pre && pre_ok; ++k, ip.next()) pre_ok = load_q(ip);
+    }
+    ptx::grid_dependency_wait();
+    for (long long u = u0; u < u1 && pre_ok; ++u, it.next()) {
       int ok = 1;
       if (it.seg != cur_seg) {
         // the segment's image into the next slot, once its last user is done
@@ -1123,27 +1186,7 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
-      if (lane == 0)
-        ok = wait_bounded(empty_bar(it.stage), it.phase ^ 1u, flag, kFlagApplyTimeout, &s_abort);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      if (ROPE) {
-        const int blk = it.seg - (it.seg / nblk) * nblk;
-        write_row_offsets(rope, s_pos + it.stage * 3 * TM, TM, blk * L + it.tile * TM, lane);
-        __syncwarp();
-      }
-      if (lane == 0) {
-        ptx::mbar_expect_tx(full_bar(it.stage), TX);
-        const int3 c = scd.of(it.seg, it.tile * TM);
-#pragma unroll
-        for (int h = 0; h < HALVES; ++h) {
-          ptx::tma_load_4d(base + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_q, 64 * h, c.x,
-                           c.y, c.z, full_bar(it.stage));
-          if (!DIRECT && GATE)
-            ptx::tma_load_4d(gbase + it.stage * TILE_BYTES + h * HALF_BYTES, &tm_g, 64 * h, c.x,
-                             c.y, c.z, full_bar(it.stage));
-        }
-      }
-      ++issued;
+      if (u - u0 >= pre && !load_q(it)) break;
     }
     if (lane == 0) {
       for (long long i = issued - stages < 0 ? 0 : issued - stages; i < issued; ++i)
@@ -1261,8 +1304,16 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     const uint32_t lane_bits = (uint32_t)(32 * q4) << 16;
     const int col0 = jw * EC;                    // epilogue columns of this thread
     if (ROPE) {
-      for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = gtab[e];
-      ptx::bar_sync(1, kMath);                   // table complete before the first lookup
+      // complete before the first lookup: built here where q tiles are
+      // transformed before the dependency wait, else copied from the state
+      // build's after it
+      if (early > 0) {
+        build_rope_table(rope, s_tab, tt);
+      } else {
+        ptx::grid_dependency_wait();
+        for (int e = tt; e < rope.entries; e += kMath) s_tab[e] = gtab[e];
+        ptx::bar_sync(1, kMath);
+      }
     }
     ChunkCol col[CPW];
 #pragma unroll
@@ -1549,6 +1600,12 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3, &gs3);
   const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3, sb3, gs3);
   const long long U3 = (long long)sc.nseg * ((a.Lq + kApplyTile - 1) / kApplyTile);
+  // q (and gate) stages the apply kernel loads before its dependency wait,
+  // by measure on B200: two behind a state build that reduces its own
+  // segments, at D = 128 and without RoPE; none on the D = 64 RoPE path and
+  // behind the separate reduction kernel, where the early traffic slowed the
+  // reductions (L2-latency bound) more than it saved
+  const int early = a.fused && (D == 128 || !a.rope.on) ? 2 : 0;
   const int G3 = (int)(U3 < sms ? U3 : sms);
   auto k3 = a.rope.on ? (gate ? apply_tc<D, true, true> : apply_tc<D, true, false>)
                       : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
@@ -1557,7 +1614,7 @@ la_status tc_run_d(const TcArgs& a, int sms) {
                   static_cast<__nv_bfloat16*>(a.out), a.D, a.rope, a.Lq, sc.nblk, scd, U3, s3,
                   sb3, gs3,
                   reinterpret_cast<const uint8_t*>(a.apply), (const float2*)a.gtab, a.eps,
-                  a.flag);
+                  a.flag, early);
   if (st != LA_OK) return st;
   return tc_mark(a, 3);
 }
