@@ -328,3 +328,46 @@ def test_tensor_core_path_is_selected_for_the_bf16_workloads():
                                     rope_split=(8, 12, 12))
     assert not la.uses_tensor_cores(1, 2, 24, 64, torch.bfloat16, grid=(2, 3, 4),
                                     rope_split=(20, 22, 22))
+
+
+def _chain(call, x0, n=3):
+    """n calls enqueued back to back on one stream, each reading the previous
+    one's output (as q, and as k where the call takes one), then the same
+    calls one at a time after a synchronize: bitwise equal."""
+    outs = [x0]
+    for _ in range(n):
+        outs.append(call(outs[-1]))
+    torch.cuda.synchronize()
+    for i in range(1, n):
+        ref = call(outs[i].clone())
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i + 1], ref), "call %d of the chain" % (i + 1)
+
+
+def test_chained_calls_read_the_previous_output():
+    # The apply kernel loads its first q (and gate) tiles before its
+    # dependency wait, relying on the state build letting it launch only
+    # after the state build's own wait: everything before the state build in
+    # the stream -- here the previous call's apply kernel, which wrote this
+    # call's q and k -- has completed by then.
+    w = workloads.Workload("chain_d128", B=2, H=3, N=6 * 8 * 10, D=128, dtype="bf16", seed=31,
+                           grid=(6, 8, 10), rope_split=(32, 48, 48), gate=True)
+    t = upload(w, workloads.make_inputs(w))
+    p = la.make_params(w.B, w.H, w.N, w.D, t["q"].dtype, "bidirectional", 0, w.grid,
+                       w.rope_split, w.rope_theta, w.eps)
+    ws = la.workspace_for(p, t["q"].device)
+    _chain(lambda x: la.forward(x, x, t["v"], t["g"], grid=w.grid, rope_split=w.rope_split,
+                                theta=w.rope_theta, eps=w.eps, workspace=ws), t["q"])
+    # D = 64 with RoPE (loads after the wait) and cross-attention (no RoPE,
+    # loads before it)
+    w64 = W["480p_bidir"].scaled(2)
+    t64 = upload(w64, workloads.make_inputs(w64))
+    p64 = la.make_params(w64.B, w64.H, w64.N, w64.D, t64["q"].dtype, "bidirectional", 0,
+                         w64.grid, w64.rope_split, w64.rope_theta, w64.eps)
+    ws64 = la.workspace_for(p64, t64["q"].device)
+    _chain(lambda x: la.forward(x, x, t64["v"], grid=w64.grid, rope_split=w64.rope_split,
+                                theta=w64.rope_theta, eps=w64.eps, workspace=ws64), t64["q"])
+    kv = t64["k"][:, :, :300].contiguous(), t64["v"][:, :, :300].contiguous()
+    pc = la.make_params(w64.B, w64.H, w64.N, w64.D, t64["q"].dtype, eps=w64.eps)
+    wsc = la.Workspace(la._native.lin_attn_cross_workspace_size(pc, 300), t64["q"].device)
+    _chain(lambda x: la.cross_forward(x, kv[0], kv[1], eps=w64.eps, workspace=wsc), t64["q"])
