@@ -933,20 +933,27 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 // one row n of the column-major partials (n = D is z) of one head, for all of
 // the head's segments. The CTA first tabulates the partial count of up to
 // kFinSegs segments in shared memory; threads then take the segments in
-// batches of kFinBatch, issuing the loads of the first two partials of every
+// batches of BATCH, issuing the loads of the first two partials of every
 // segment of a batch before the first add (more than two is rare and loops).
+// With few blocks per head (kFinFewBlocks or fewer) the kernel takes batches
+// of kFinSmallBatch under a cap of 80 registers per thread (MINB = 6), so that
+// the apply kernel's CTAs (608 threads x 64 registers) fit beside two of its
+// CTAs on an SM and start while it runs (480p, 7 blocks: 118.8 -> 117.2 us per
+// forward on B200); with many blocks, batches of 16 and no cap (fewer rounds
+// of loads).
 
 constexpr int kFinThreads = 128;
-constexpr int kFinBatch = 16;
 constexpr int kFinSegs = 1024;
+constexpr int kFinFewBlocks = 8;
+constexpr int kFinSmallBatch = 4;
 
 template <int D>
 __host__ __device__ constexpr int fin_items_per_head() {
   return (D + 1) * (D / 4);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kFinThreads)
+template <int D, int BATCH, int MINB>
+__global__ void __launch_bounds__(kFinThreads, MINB)
 finalize_images(const float* __restrict__ partials, const __grid_constant__ Sched sc,
                 uint8_t* __restrict__ images, float* __restrict__ stS,
                 float* __restrict__ stz, int use_state, int commit) {
@@ -979,18 +986,18 @@ finalize_images(const float* __restrict__ partials, const __grid_constant__ Sche
       s_np[jj] = parts_of(sc, (int)(seg0 + j0 + jj));
     __syncthreads();
     if (valid) {
-      for (int jb = 0; jb < cnt; jb += kFinBatch) {
-        float4 b0[kFinBatch], b1[kFinBatch];
-        int np[kFinBatch];
+      for (int jb = 0; jb < cnt; jb += BATCH) {
+        float4 b0[BATCH], b1[BATCH];
+        int np[BATCH];
 #pragma unroll
-        for (int k = 0; k < kFinBatch; ++k) {
+        for (int k = 0; k < BATCH; ++k) {
           np[k] = jb + k < cnt ? s_np[jb + k] : 0;
           const float* p = pbase + (j0 + jb + k) * pstride;
           if (np[k] > 0) b0[k] = __ldg(reinterpret_cast<const float4*>(p));
           if (np[k] > 1) b1[k] = __ldg(reinterpret_cast<const float4*>(p + DD1));
         }
 #pragma unroll
-        for (int k = 0; k < kFinBatch; ++k) {
+        for (int k = 0; k < BATCH; ++k) {
           if (np[k] > 0) {
             float4 blk = b0[k];
             if (np[k] > 1) blk = add4(blk, b1[k]);
@@ -1584,8 +1591,13 @@ la_status tc_run_d(const TcArgs& a, int sms) {
     // the reduction and the apply kernel are launched programmatically
     // dependent: they start early and wait in griddepcontrol.wait
     const dim3 grid((unsigned)a.heads, (fin_items_per_head<D>() + kFinThreads - 1) / kFinThreads);
-    st = launch_pdl(finalize_images<D>, grid, dim3(kFinThreads), 0, a.stream,
-                    (const float*)a.part, sc, images, a.stS, a.stz, a.use_state, a.commit);
+    st = sc.nblk <= kFinFewBlocks
+             ? launch_pdl(finalize_images<D, kFinSmallBatch, 6>, grid, dim3(kFinThreads), 0,
+                          a.stream, (const float*)a.part, sc, images, a.stS, a.stz,
+                          a.use_state, a.commit)
+             : launch_pdl(finalize_images<D, 16, 1>, grid, dim3(kFinThreads), 0, a.stream,
+                          (const float*)a.part, sc, images, a.stS, a.stz, a.use_state,
+                          a.commit);
     if (st != LA_OK) return st;
   }
   if ((st = tc_mark(a, 2)) != LA_OK) return st;

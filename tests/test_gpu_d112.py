@@ -67,6 +67,18 @@ def test_head_dim_112_block_steps():
     torch.cuda.synchronize()
     ref = oracle.forward(oracle.params_for(w, "block_causal"), x["q"], x["k"], x["v"])
     assert_parity(to64(torch.cat(outs, dim=2)), ref, "bf16", "d112 block steps")
+    # a read-only step (commit off) leaves the state byte for byte as it was
+    # and gives the output the committing step gives
+    S0, z0 = st.S.clone(), st.z.clone()
+    blk = [t[n][:, :, :bt].contiguous() for n in ("q", "k", "v")]
+    kw = dict(t_offset=3, grid=(1, 4, 6), rope_split=w.rope_split, eps=w.eps)
+    a = st.step(*blk, commit=False, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(st.S, S0) and torch.equal(st.z, z0)
+    b = st.step(*blk, commit=True, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert not torch.equal(st.S, S0)
 
 
 def test_head_dim_112_480p_full_size_sampled_rows():
