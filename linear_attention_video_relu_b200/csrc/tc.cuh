@@ -36,6 +36,9 @@ namespace la {
 // dynamic shared memory per CTA on sm_100 (227 KB), less 1 KB for the
 // kernels' static shared variables
 constexpr int kSmemBudget = 227 * 1024 - 1024;
+// per CTA when two share an SM (228 KB, 1 KB reserved per CTA, static shared
+// variables)
+constexpr int kSmemBudgetHalf = 112 * 1024;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 enum : int { kFlagStateTimeout = 1, kFlagApplyTimeout = 2 };
@@ -150,19 +153,20 @@ __host__ __device__ constexpr bool apply_direct_out(int D) { return D == 128; }
 // Two S slots (the next segment's image prefetched while the current one is
 // in use) when at least 4 q stages still fit, else one slot and the most
 // stages.
-inline void pick_apply_plan(int D, int entries, int gate, int* stages, int* sbuf, int* gst) {
+inline void pick_apply_plan(int D, int entries, int gate, int* stages, int* sbuf, int* gst,
+                            int budget = kSmemBudget) {
   *stages = 0;
   *sbuf = 1;
   auto g = [&](int s) { return gate ? (apply_direct_out(D) ? 2 : s) : 0; };
   for (int s = 8; s >= 4; --s)
-    if (apply_plan(D, entries, gate, s, 2, g(s)).total <= (uint32_t)kSmemBudget) {
+    if (apply_plan(D, entries, gate, s, 2, g(s)).total <= (uint32_t)budget) {
       *stages = s;
       *sbuf = 2;
       *gst = g(s);
       return;
     }
   for (int s = 8; s >= 2; --s)
-    if (apply_plan(D, entries, gate, s, 1, g(s)).total <= (uint32_t)kSmemBudget) {
+    if (apply_plan(D, entries, gate, s, 1, g(s)).total <= (uint32_t)budget) {
       *stages = s;
       *gst = g(s);
       return;
@@ -1039,12 +1043,23 @@ finalize_images(const float* __restrict__ partials, const __grid_constant__ Sche
 // warp 0 q (+ gate) tiles and images, 1 MMA, 2-17 math, 18 store or gate loads
 constexpr int kTcThreadsApply = 96 + kMath;
 
+// At D = 64 without RoPE two apply CTAs share an SM where their plans fit in
+// half of its shared memory (4 q stages each instead of 8): the same bytes in
+// flight per SM, and twice the math warps per scheduler to hide the per-tile
+// chain's shared- and tensor-memory latencies (these variants are compiled
+// for 48 registers per thread so that two fit). Cross-attention at 480p x 300
+// text tokens: 59.3 -> 54.8 us on B200. With RoPE (one image slot in half the
+// memory, the table twice per SM) it was slower, so those keep one CTA.
+__host__ __device__ constexpr int apply_min_ctas(int D, bool rope) {
+  return D == 64 && !rope ? 2 : 1;
+}
+
 __host__ __device__ constexpr uint32_t tmem_cols_pow2(uint32_t n) {
   return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : (n <= 256 ? 256 : 512)));
 }
 
 template <int D, bool ROPE, bool GATE>
-__global__ void __launch_bounds__(kTcThreadsApply, 1)
+__global__ void __launch_bounds__(kTcThreadsApply, apply_min_ctas(D, ROPE))
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
          const __grid_constant__ CUtensorMap tm_o, __nv_bfloat16* __restrict__ out, int ocols,
          const __grid_constant__ Rope rope, int L, int nblk,
@@ -1557,6 +1572,11 @@ inline la_status tc_smem_attr(K kernel, uint32_t bytes) {
     cudaGetLastError();
     return LA_ERR_UNSUPPORTED;
   }
+  // the whole unified L1/shared array as shared memory, so that two apply
+  // CTAs of half the budget can share an SM (a hint; nothing else relies on it)
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    cudaGetLastError();
   return LA_OK;
 }
 
@@ -1608,8 +1628,12 @@ la_status tc_run_d(const TcArgs& a, int sms) {
       !make_map(&mo, a.out, a.D, a.Lq, sc.nseg, kApplyTile, scd) ||
       !make_map(&mg, gate ? a.g : a.q, a.D, a.Lq, sc.nseg, kApplyTile, scd))
     return LA_ERR_CUDA;
-  int s3 = 0, sb3 = 1, gs3 = 0;
-  pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3, &gs3);
+  int s3 = 0, sb3 = 1, gs3 = 0, cps = 1;   // cps: apply CTAs per SM
+  if (apply_min_ctas(D, a.rope.on != 0) == 2) {
+    pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3, &gs3, kSmemBudgetHalf);
+    if (s3 >= 3) cps = 2;
+  }
+  if (cps == 1) pick_apply_plan(D, entries, gate ? 1 : 0, &s3, &sb3, &gs3);
   const ApplyPlan p3 = apply_plan(D, entries, gate ? 1 : 0, s3, sb3, gs3);
   const long long U3 = (long long)sc.nseg * ((a.Lq + kApplyTile - 1) / kApplyTile);
   // q (and gate) stages the apply kernel loads before its dependency wait,
@@ -1618,7 +1642,7 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   // behind the separate reduction kernel, where the early traffic slowed the
   // reductions (L2-latency bound) more than it saved
   const int early = a.fused && (D == 128 || !a.rope.on) ? 2 : 0;
-  const int G3 = (int)(U3 < sms ? U3 : sms);
+  const int G3 = (int)(U3 < (long long)sms * cps ? U3 : (long long)sms * cps);
   auto k3 = a.rope.on ? (gate ? apply_tc<D, true, true> : apply_tc<D, true, false>)
                       : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
   if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
