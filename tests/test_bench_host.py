@@ -197,3 +197,28 @@ def test_traffic_of_the_temporal_conv_follows_its_own_source(tmp_path, monkeypat
     assert bench.ncu_traffic("temporal_conv", "480p_hidden_tconv") == 300
     (csrc / "tconv.cu").write_text("int b; int d;\n")    # its own source changes: stale
     assert bench.ncu_traffic("temporal_conv", "480p_hidden_tconv") is None
+
+
+def test_every_committed_traffic_line_names_a_workload_the_bench_reads():
+    # a '# bench-traffic <kernel> <workload> ...' line is only read back if its
+    # workload key is one the bench looks up: the bare name for bidirectional
+    # forwards, name/mode for the other modes, the cross and conv names
+    import glob
+    import os
+    import bench
+    keys = {"480p_bidir"}
+    for name, _ in bench.secondary_jobs(1, None, 1.0, "measured"):
+        if "/" in name:
+            w, mode = name.split("/")
+            keys.add(w if mode in ("bidirectional", "cross") else name)
+        else:
+            keys.add(name)
+    seen = 0
+    for path in glob.glob(os.path.join(bench.ROOT, "profiles", "*.txt")):
+        for line in open(path):
+            parts = line.split()
+            if len(parts) == 6 and parts[:2] == ["#", "bench-traffic"]:
+                seen += 1
+                assert parts[2] in ("state_build", "apply", "temporal_conv"), (path, line)
+                assert parts[3] in keys, (path, parts[3], sorted(keys))
+    assert seen >= 10
