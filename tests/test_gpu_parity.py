@@ -371,3 +371,37 @@ def test_chained_calls_read_the_previous_output():
     pc = la.make_params(w64.B, w64.H, w64.N, w64.D, t64["q"].dtype, eps=w64.eps)
     wsc = la.Workspace(la._native.lin_attn_cross_workspace_size(pc, 300), t64["q"].device)
     _chain(lambda x: la.cross_forward(x, kv[0], kv[1], eps=w64.eps, workspace=wsc), t64["q"])
+
+
+def test_chained_block_steps_read_the_previous_output():
+    # Algorithm 1's per-block call at D = 128 (the apply kernel loads its
+    # first q stages before its dependency wait there): each step's q is the
+    # previous step's output, enqueued back to back; the same steps made one
+    # at a time after a synchronize, from the same starting state, give the
+    # same outputs and the same committed state, bit for bit.
+    w = workloads.Workload("chain_steps", B=1, H=2, N=3 * 6 * 8, D=128, dtype="bf16", seed=32,
+                           grid=(3, 6, 8), rope_split=(32, 48, 48), gate=True)
+    t = upload(w, workloads.make_inputs(w))
+    bt = 6 * 8
+    blk = [{n: t[n][:, :, b * bt:(b + 1) * bt].contiguous() for n in ("q", "k", "v", "g")}
+           for b in range(3)]
+    kw = dict(grid=(1, 6, 8), rope_split=w.rope_split, eps=w.eps)
+
+    def run(sync):
+        st = la.BlockState(w.B, w.H, w.D)
+        x = blk[0]["q"]
+        outs = []
+        for b in range(3):
+            x = st.step(x, blk[b]["k"], blk[b]["v"], blk[b]["g"], t_offset=b, commit=True, **kw)
+            if sync:
+                torch.cuda.synchronize()
+                x = x.clone()
+            outs.append(x)
+        torch.cuda.synchronize()
+        return outs, st
+
+    a, sa = run(False)
+    b, sb = run(True)
+    for i in range(3):
+        assert torch.equal(a[i], b[i]), "step %d" % i
+    assert torch.equal(sa.S, sb.S) and torch.equal(sa.z, sb.z)
