@@ -152,11 +152,14 @@ __host__ __device__ constexpr bool apply_direct_out(int D) { return D == 128; }
 
 // Two S slots (the next segment's image prefetched while the current one is
 // in use) when at least 4 q stages still fit, else one slot and the most
-// stages.
+// stages; a gate ring of its own holds two tiles, or one where a large RoPE
+// table leaves no room for two (the gate load of the next tile then waits for
+// the current tile's epilogue).
 inline void pick_apply_plan(int D, int entries, int gate, int* stages, int* sbuf, int* gst,
                             int budget = kSmemBudget) {
   *stages = 0;
   *sbuf = 1;
+  *gst = 0;
   auto g = [&](int s) { return gate ? (apply_direct_out(D) ? 2 : s) : 0; };
   for (int s = 8; s >= 4; --s)
     if (apply_plan(D, entries, gate, s, 2, g(s)).total <= (uint32_t)budget) {
@@ -169,6 +172,13 @@ inline void pick_apply_plan(int D, int entries, int gate, int* stages, int* sbuf
     if (apply_plan(D, entries, gate, s, 1, g(s)).total <= (uint32_t)budget) {
       *stages = s;
       *gst = g(s);
+      return;
+    }
+  if (!gate || !apply_direct_out(D)) return;
+  for (int s = 8; s >= 2; --s)
+    if (apply_plan(D, entries, gate, s, 1, 1).total <= (uint32_t)budget) {
+      *stages = s;
+      *gst = 1;
       return;
     }
 }

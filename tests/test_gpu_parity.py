@@ -68,6 +68,13 @@ def edge_cases():
         (mk("d128_blocks", B=1, H=3, N=3 * 7 * 13, D=128, dtype="bf16", seed=22,
             grid=(3, 7, 13), rope_split=(32, 48, 48), gate=True, modes=("block_causal",),
             block_tokens=91), "block_causal"),
+        # D = 128 with a gate and a RoPE table too large for a two-tile gate
+        # ring (2 x 3 x 134: 3598 entries): the apply kernel's one-tile ring
+        (mk("d128_wide_table", B=1, H=2, N=2 * 3 * 134, D=128, dtype="bf16", seed=25,
+            grid=(2, 3, 134), rope_split=(32, 48, 48), gate=True), "bidirectional"),
+        (mk("d128_wide_table_blocks", B=1, H=2, N=2 * 3 * 134, D=128, dtype="bf16", seed=26,
+            grid=(2, 3, 134), rope_split=(32, 48, 48), gate=True, modes=("block_causal",),
+            block_tokens=402), "block_causal"),
         # thousands of one-tile heads: a CTA completes more heads than it can
         # leave to its tail and reduces the rest on the spot
         (mk("many_small_heads", B=64, H=128, N=16, D=64, dtype="bf16", seed=23,
@@ -322,6 +329,11 @@ def test_tensor_core_path_is_selected_for_the_bf16_workloads():
     w = W["480p_bidir"]
     assert la.uses_tensor_cores(w.B, w.H, w.N, w.D, torch.bfloat16, mode="token_causal",
                                 grid=w.grid, rope_split=w.rope_split)
+    # D = 128 on the 720p grid (3628 table entries) and the wide-table case
+    for grid in ((21, 45, 80), (2, 3, 134)):
+        n = grid[0] * grid[1] * grid[2]
+        assert la.uses_tensor_cores(1, 2, n, 128, torch.bfloat16, grid=grid,
+                                    rope_split=(32, 48, 48))
     # fp32 I/O, D = 32 and RoPE widths that are not multiples of 8 use CUDA cores
     assert not la.uses_tensor_cores(1, 2, 256, 32, torch.float32)
     assert not la.uses_tensor_cores(1, 4, 60, 32, torch.bfloat16, grid=(3, 4, 5),
