@@ -30,10 +30,11 @@
  *
  * Conventions for every entry point:
  *   - Memory. The caller owns all device memory (inputs, output, state,
- *     workspace); the library allocates and frees nothing. Every entry point
- *     but lin_attn_forward_noalloc keeps no global mutable state, so those
- *     calls are re-entrant; lin_attn_forward_noalloc works in one device
- *     array shared by all its calls (see its comment).
+ *     workspace); the library allocates and frees nothing. Calls are
+ *     re-entrant: the library's process-wide state is a mutex-guarded record
+ *     of the kernels whose shared-memory limit it has set on each device, and
+ *     the one device array shared by all calls of lin_attn_forward_noalloc
+ *     (see its comment).
  *   - Layout. q, k, v, gate, out are contiguous [B, H, N, D] (or [B, N, H, D]
  *     with p->layout = LA_LAYOUT_BNHD) with D innermost, in the I/O dtype.
  *     The state is fp32: S [B, H, D, D] with

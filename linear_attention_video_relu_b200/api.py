@@ -7,6 +7,7 @@ bf16 or fp32; the carried state is fp32 S [B, H, D, D] and z [B, H, D].
 """
 from __future__ import annotations
 
+import contextlib
 from typing import Optional, Sequence
 
 import torch
@@ -56,9 +57,29 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
-def _stream(stream: Optional[torch.cuda.Stream]):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream
+# torch's raw current-stream query, when this torch has it: the handle without
+# building a Stream object (a per-call cost on the host)
+_current_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream: Optional[torch.cuda.Stream], device: Optional[int] = None):
+    """The handle of `stream`, else of the current stream of `device` (an
+    index; None: the current device)."""
+    if stream is not None:
+        return stream.cuda_stream
+    if device is None:
+        device = torch.cuda.current_device()
+    if _current_raw_stream is not None:
+        return _current_raw_stream(device)
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _on_device(t: torch.Tensor):
+    """t's device made current for the call; no switch when it already is."""
+    idx = t.get_device()
+    if idx == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(idx)
 
 
 _DTYPE_OF = {v: k for k, v in _DTYPES.items()}
@@ -74,8 +95,12 @@ def _check_io(p: C.la_params, *ts, require_cuda: bool = True):
     """Contiguous CUDA tensors of shape [B, H, N, D] (or [B, N, H, D]) in the
     params' dtype (require_cuda=False checks the rest on host tensors)."""
     shape = ((p.B, p.H, p.N, p.D) if p.layout == C.LA_LAYOUT_BHND else (p.B, p.N, p.H, p.D))
+    dt = _DTYPE_OF[p.dtype]
     for t in ts:
         if t is None:
+            continue
+        if t.dtype is dt and t.is_contiguous() and t.shape == shape and (t.is_cuda or
+                                                                         not require_cuda):
             continue
         if (require_cuda and not t.is_cuda) or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
@@ -131,10 +156,10 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[to
     _same_device(q, k, v, gate, out, None if workspace is None else workspace.buf)
     if workspace is None:
         workspace = workspace_for(p, q.device)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         C.check(C.lin_attn_forward(p, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(out),
-                                   workspace.ptr, workspace.nbytes, _stream(stream)),
-                "lin_attn_forward")
+                                   workspace.ptr, workspace.nbytes,
+                                   _stream(stream, q.get_device())), "lin_attn_forward")
     return out
 
 
@@ -160,9 +185,10 @@ def cross_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if workspace is None:
         with torch.cuda.device(q.device):
             workspace = Workspace(C.lin_attn_cross_workspace_size(p, M), q.device)
-    with torch.cuda.device(q.device):
+    with _on_device(q):
         C.check(C.lin_attn_cross_forward(p, M, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(out),
-                                         workspace.ptr, workspace.nbytes, _stream(stream)),
+                                         workspace.ptr, workspace.nbytes,
+                                         _stream(stream, q.get_device())),
                 "lin_attn_cross_forward")
     return out
 
@@ -178,6 +204,7 @@ class BlockState:
         C.check(C.lin_attn_state_init(self._st, B, H, D, self.S.data_ptr(), self.z.data_ptr()),
                 "lin_attn_state_init")
         self._ws = {}
+        self._plans = {}
 
     def reset(self, stream=None) -> None:
         with torch.cuda.device(self.S.device):
@@ -192,37 +219,50 @@ class BlockState:
             self._ws[key] = ws
         return ws
 
+    def _plan(self, x, grid, rope_split, theta, eps, layout):
+        """(params, workspace) of a block of x's shape and dtype with these
+        settings, made once per distinct call and kept (params are only read
+        by the library)."""
+        key = (x.shape, x.dtype, None if grid is None else tuple(grid),
+               None if rope_split is None else tuple(rope_split), theta, eps, layout)
+        ent = self._plans.get(key)
+        if ent is None:
+            B, H, N, D = _dims(x, layout)
+            p = make_params(B, H, N, D, x.dtype, "bidirectional", 0, grid, rope_split, theta,
+                            eps, layout)
+            ent = (p, self._workspace(p))
+            self._plans[key] = ent
+        return ent
+
     def step(self, q, k, v, gate=None, *, t_offset: int = 0, commit: bool = True,
              grid=None, rope_split=None, theta: float = 10000.0, eps: float = 1e-6,
              out=None, stream=None, layout: str = "bhnd") -> torch.Tensor:
         """One block of block-causal attention against the carried state."""
-        B, H, N, D = _dims(q, layout)
-        p = make_params(B, H, N, D, q.dtype, "bidirectional", 0, grid, rope_split, theta, eps,
-                        layout)
+        p, ws = self._plan(q, grid, rope_split, theta, eps, layout)
         _check_io(p, q, k, v, gate)
         if out is None:
             out = torch.empty_like(q)
-        _check_io(p, out)
+        else:
+            _check_io(p, out)
         _same_device(self.S, q, k, v, gate, out)
-        ws = self._workspace(p)
-        with torch.cuda.device(q.device):
-            C.check(C.lin_attn_block_step(p, self._st, t_offset, _ptr(q), _ptr(k), _ptr(v),
-                                          _ptr(gate), _ptr(out), 1 if commit else 0, ws.ptr,
-                                          ws.nbytes, _stream(stream)), "lin_attn_block_step")
+        dev = q.get_device()
+        with _on_device(q):
+            C.check(C.lin_attn_block_step(p, self._st, t_offset, q.data_ptr(), k.data_ptr(),
+                                          v.data_ptr(), _ptr(gate), out.data_ptr(),
+                                          1 if commit else 0, ws.ptr, ws.nbytes,
+                                          _stream(stream, dev)), "lin_attn_block_step")
         return out
 
     def update(self, k, v, *, t_offset: int = 0, grid=None, rope_split=None,
                theta: float = 10000.0, stream=None, layout: str = "bhnd") -> None:
         """Fold a block's k, v into the state without producing output."""
-        B, H, N, D = _dims(k, layout)
-        p = make_params(B, H, N, D, k.dtype, "bidirectional", 0, grid, rope_split, theta, 1e-6,
-                        layout)
+        p, ws = self._plan(k, grid, rope_split, theta, 1e-6, layout)
         _check_io(p, k, v)
         _same_device(self.S, k, v)
-        ws = self._workspace(p)
-        with torch.cuda.device(k.device):
-            C.check(C.lin_attn_state_update(p, self._st, t_offset, _ptr(k), _ptr(v), ws.ptr,
-                                            ws.nbytes, _stream(stream)), "lin_attn_state_update")
+        with _on_device(k):
+            C.check(C.lin_attn_state_update(p, self._st, t_offset, k.data_ptr(), v.data_ptr(),
+                                            ws.ptr, ws.nbytes, _stream(stream, k.get_device())),
+                    "lin_attn_state_update")
 
 
 def uses_tensor_cores(B, H, N, D, dtype, **kw) -> bool:

@@ -588,6 +588,72 @@ __device__ void reduce_segment_smem(const float* sp, int np, int seg,
   }
 }
 
+// The carried state of one segment copied to shared memory transposed, row n
+// of T (pitch D + 1 floats) holding column n of S and row D holding z, by
+// 4-byte asynchronous copies: consecutive threads read consecutive floats of
+// S (the per-item reads of carried4 touch one float per 32-byte sector), the
+// pitch spreads their shared-memory writes over all banks, and no register
+// holds a value in flight. Complete once the thread's cp_async_wait_all
+// returns.
+template <int D>
+__device__ void load_carried_transposed(const float* __restrict__ gS,
+                                        const float* __restrict__ gz, float* T, int tid,
+                                        int nthr) {
+  constexpr int TP = D + 1;
+  const uint32_t t0 = ptx::smem_u32(T);
+  for (int i = tid; i < D * D + D; i += nthr) {
+    const int a = i / D, n = i - a * D;   // S[a][n], or z[n] for a = D
+    ptx::cp_async4(t0 + 4u * (uint32_t)(a < D ? n * TP + a : D * TP + n),
+                   a < D ? gS + i : gz + n);
+  }
+}
+
+// reduce_segment_smem with the carried state in T (load_carried_transposed):
+// the same fp32 operations in the same order; when committing, the new state
+// goes back into T for store_carried_transposed.
+template <int D>
+__device__ void reduce_segment_tr(const float* sp, int np, int seg, uint8_t* __restrict__ images,
+                                  float* T, int commit, int tid, int nthr) {
+  constexpr int DD1 = D * (D + 1), QPR = D / 4, ITEMS = (D + 1) * QPR, TP = D + 1;
+  uint8_t* img = images + (long long)seg * image_bytes(D);
+  for (int item = tid; item < ITEMS; item += nthr) {
+    const int n = item / QPR;
+    const int a0 = 4 * (item - n * QPR);
+    const int off = n * D + a0;
+    float4 acc = *reinterpret_cast<const float4*>(sp + off);
+    for (int i = 1; i < np; ++i)
+      acc = add4(acc, *reinterpret_cast<const float4*>(sp + (long long)i * DD1 + off));
+    float* t = T + n * TP + a0;
+    const float4 run = add4(make_float4(t[0], t[1], t[2], t[3]), acc);
+    store_image4<D>(img + image_offset<D>(n, a0), n == D, a0, run);
+    if (commit) {
+      t[0] = run.x;
+      t[1] = run.y;
+      t[2] = run.z;
+      t[3] = run.w;
+    }
+  }
+}
+
+// T back to the carried state in whole float4 rows of S (and z).
+template <int D>
+__device__ void store_carried_transposed(const float* T, float* __restrict__ gS,
+                                         float* __restrict__ gz, int tid, int nthr) {
+  constexpr int QPR = D / 4, TP = D + 1;
+  for (int item = tid; item < (D + 1) * QPR; item += nthr) {
+    const int a = item / QPR;
+    const int n0 = 4 * (item - a * QPR);
+    if (a < D) {
+      *reinterpret_cast<float4*>(gS + a * D + n0) =
+          make_float4(T[(n0 + 0) * TP + a], T[(n0 + 1) * TP + a], T[(n0 + 2) * TP + a],
+                      T[(n0 + 3) * TP + a]);
+    } else {
+      const float* t = T + D * TP + n0;
+      *reinterpret_cast<float4*>(gz + n0) = make_float4(t[0], t[1], t[2], t[3]);
+    }
+  }
+}
+
 // ---- state build ------------------------------------------------------------------
 
 // warp 0 TMA, warp 1 MMA, warps 2-17 math, warps 18-21 epilogue (one per TMEM
@@ -904,6 +970,7 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     // them from shared memory -- one round trip to L2 for all of them instead
     // of one per row group of each thread.
     constexpr uint32_t SLOT = DD1 * 4;
+    constexpr uint32_t TBYTES = (D + 1) * (D + 1) * 4;   // transposed carried state
     const int cap = (int)(P.off_bar / SLOT);
     __threadfence();
     uint32_t tph = 0;
@@ -922,14 +989,30 @@ state_build_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           ptx::bulk_load(base + (uint32_t)i * SLOT,
                          partials + ((long long)seg * sc.maxc + i) * DD1, SLOT, tail_bar);
       }
+      // the carried state goes through shared memory, transposed, behind the
+      // partial slots where it fits
+      float* gS = use_state ? stS + (long long)seg * D * D : nullptr;
+      float* gz = use_state ? stz + (long long)seg * D : nullptr;
+      float* T = reinterpret_cast<float*>(sm + (uint32_t)np * SLOT);
+      const bool tr = use_state && (uint32_t)np * SLOT + TBYTES <= P.off_bar;
       float first[4];
-      carried4<D>(use_state ? stS + (long long)seg * D * D : nullptr,
-                  use_state ? stz + (long long)seg * D : nullptr, use_state, threadIdx.x, first);
+      if (tr) load_carried_transposed<D>(gS, gz, T, threadIdx.x, kTcThreadsState);
+      else carried4<D>(gS, gz, use_state, threadIdx.x, first);
       const bool got = wait_bounded(tail_bar, tph, flag, kFlagStateTimeout, &s_abort);
+      if (tr) ptx::cp_async_wait_all();
       if (!__syncthreads_and(got)) break;   // every thread leaves together
       tph ^= 1u;
-      reduce_segment_smem<D>(reinterpret_cast<const float*>(sm), np, seg, images, stS, stz,
-                             use_state, commit, threadIdx.x, kTcThreadsState, first);
+      if (tr) {
+        reduce_segment_tr<D>(reinterpret_cast<const float*>(sm), np, seg, images, T, commit,
+                             threadIdx.x, kTcThreadsState);
+        if (commit) {
+          __syncthreads();
+          store_carried_transposed<D>(T, gS, gz, threadIdx.x, kTcThreadsState);
+        }
+      } else {
+        reduce_segment_smem<D>(reinterpret_cast<const float*>(sm), np, seg, images, stS, stz,
+                               use_state, commit, threadIdx.x, kTcThreadsState, first);
+      }
       __syncthreads();   // before the next segment's copies overwrite the slots
     }
   }
@@ -1068,13 +1151,13 @@ __host__ __device__ constexpr uint32_t tmem_cols_pow2(uint32_t n) {
   return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : (n <= 256 ? 256 : 512)));
 }
 
-template <int D, bool ROPE, bool GATE>
+template <int D, bool ROPE, bool GATE, bool LATE>
 __global__ void __launch_bounds__(kTcThreadsApply, apply_min_ctas(D, ROPE))
 apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
          const __grid_constant__ CUtensorMap tm_o, __nv_bfloat16* __restrict__ out, int ocols,
          const __grid_constant__ Rope rope, int L, int nblk,
          const __grid_constant__ SegCoords scd, long long U, int stages, int sbuf, int gst, const uint8_t* __restrict__ images,
-         const float2* __restrict__ gtab, float eps, int* flag, int early) {
+         const float2* __restrict__ gtab, float eps, int* flag, int early, int nlate) {
   constexpr int TM = kApplyTile;
   constexpr int HALVES = D / 64;
   constexpr int HALF_BYTES = TM * 128;
@@ -1121,8 +1204,21 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   __shared__ int s_abort;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const long long u0 = (long long)blockIdx.x * U / gridDim.x;
-  const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+  // tile range: an even split, or (LATE) the last `nlate` CTAs of the grid
+  // take half as many tiles as the others (they start last: see the launcher)
+  long long u0, u1;
+  if constexpr (LATE) {
+    auto tile_start = [&](long long c) {
+      const long long e = gridDim.x - nlate;
+      const long long w = 2 * (c < e ? c : e) + (c > e ? c - e : 0);
+      return w * U / (2 * e + nlate);
+    };
+    u0 = tile_start(blockIdx.x);
+    u1 = tile_start(blockIdx.x + 1);
+  } else {
+    u0 = (long long)blockIdx.x * U / gridDim.x;
+    u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+  }
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -1575,9 +1671,60 @@ inline la_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   return LA_OK;
 }
 
+// The tensor-core kernels whose shared-memory attributes are set, as one bit
+// per device (ordinals below 64) for each kernel: a call then costs no
+// attribute calls. Guarded by a mutex, so calls stay re-entrant; a context
+// reset (cudaDeviceReset) drops the attributes but not this record, and the
+// next launch then fails with LA_ERR_CUDA.
+class AttrRegistry {
+ public:
+  bool has(const void* fn, int dev) {
+    std::lock_guard<std::mutex> g(mu_);
+    for (int i = 0; i < n_; ++i)
+      if (fn_[i] == fn) return (mask_[i] >> dev) & 1u;
+    return false;
+  }
+  void add(const void* fn, int dev) {
+    std::lock_guard<std::mutex> g(mu_);
+    for (int i = 0; i < n_; ++i)
+      if (fn_[i] == fn) {
+        mask_[i] |= 1ull << dev;
+        return;
+      }
+    if (n_ < kMax) {
+      fn_[n_] = fn;
+      mask_[n_++] = 1ull << dev;
+    }
+  }
+
+ private:
+  static constexpr int kMax = 64;
+  std::mutex mu_;
+  const void* fn_[kMax] = {};
+  uint64_t mask_[kMax] = {};
+  int n_ = 0;
+};
+
+inline AttrRegistry& attr_registry() {
+  static AttrRegistry r;
+  return r;
+}
+
+// Every plan of a tensor-core kernel fits kSmemBudget, so the dynamic
+// shared-memory limit is set to that once per kernel and device (the launch's
+// own size decides how many CTAs share an SM).
 template <typename K>
 inline la_status tc_smem_attr(K kernel, uint32_t bytes) {
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+  if (bytes > (uint32_t)kSmemBudget) return LA_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
+  }
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  const bool record = dev >= 0 && dev < 64;
+  if (record && attr_registry().has(fn, dev)) return LA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) !=
       cudaSuccess) {
     cudaGetLastError();
     return LA_ERR_UNSUPPORTED;
@@ -1587,6 +1734,7 @@ inline la_status tc_smem_attr(K kernel, uint32_t bytes) {
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                            (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
     cudaGetLastError();
+  if (record) attr_registry().add(fn, dev);
   return LA_OK;
 }
 
@@ -1648,19 +1796,35 @@ la_status tc_run_d(const TcArgs& a, int sms) {
   const long long U3 = (long long)sc.nseg * ((a.Lq + kApplyTile - 1) / kApplyTile);
   // q (and gate) stages the apply kernel loads before its dependency wait,
   // by measure on B200: two behind a state build that reduces its own
-  // segments, at D = 128 and without RoPE; none on the D = 64 RoPE path and
-  // behind the separate reduction kernel, where the early traffic slowed the
-  // reductions (L2-latency bound) more than it saved
-  const int early = a.fused && (D == 128 || !a.rope.on) ? 2 : 0;
+  // segments, at D = 128, without RoPE, and in small calls (up to 8 tiles
+  // per SM, e.g. block steps, where the apply's start is most of its time);
+  // none on large D = 64 RoPE calls and behind the separate reduction kernel,
+  // where the early traffic slowed the reductions (L2-latency bound) more
+  // than it saved
+  const int early = a.fused && (D == 128 || !a.rope.on || U3 <= 8LL * sms) ? 2 : 0;
   const int G3 = (int)(U3 < (long long)sms * cps ? U3 : (long long)sms * cps);
-  auto k3 = a.rope.on ? (gate ? apply_tc<D, true, true> : apply_tc<D, true, false>)
-                      : (gate ? apply_tc<D, false, true> : apply_tc<D, false, false>);
+  // Behind a state build that reduces its own segments, the apply CTAs are
+  // placed in index order on the SMs the state-build CTAs leave, and those
+  // that reduce leave last: in a small call (a few tiles per CTA) the last
+  // CTAs would start too late to finish with the rest, so the last
+  // (one per segment) take half as many tiles
+  const int nlate = a.fused && U3 <= 8LL * sms && U3 >= 2LL * G3 && 4 * sc.nseg <= G3
+                        ? sc.nseg : 0;
+  // (a separate instantiation, so that the even split compiles as before)
+  auto k3 = nlate > 0
+                ? (a.rope.on ? (gate ? apply_tc<D, true, true, true> : apply_tc<D, true, false, true>)
+                             : (gate ? apply_tc<D, false, true, true>
+                                     : apply_tc<D, false, false, true>))
+                : (a.rope.on ? (gate ? apply_tc<D, true, true, false>
+                                     : apply_tc<D, true, false, false>)
+                             : (gate ? apply_tc<D, false, true, false>
+                                     : apply_tc<D, false, false, false>));
   if ((st = tc_smem_attr(k3, p3.total)) != LA_OK) return st;
   st = launch_pdl(k3, dim3(G3), dim3(kTcThreadsApply), p3.total, a.stream, mq, mg, mo,
                   static_cast<__nv_bfloat16*>(a.out), a.D, a.rope, a.Lq, sc.nblk, scd, U3, s3,
                   sb3, gs3,
                   reinterpret_cast<const uint8_t*>(a.apply), (const float2*)a.gtab, a.eps,
-                  a.flag, early);
+                  a.flag, early, nlate);
   if (st != LA_OK) return st;
   return tc_mark(a, 3);
 }
