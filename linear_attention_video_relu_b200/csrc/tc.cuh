@@ -183,6 +183,16 @@ inline void pick_apply_plan(int D, int entries, int gate, int* stages, int* sbuf
     }
 }
 
+// First tile of CTA c (of g) in the apply kernel's weighted split of u tiles:
+// the last `nlate` CTAs weigh 1, the others 2 (nlate = 0 splits evenly). With
+// u >= 2 g every CTA gets at least one tile.
+__host__ __device__ inline long long apply_tile_start(long long c, int g, int nlate,
+                                                      long long u) {
+  const long long e = g - nlate;
+  const long long w = 2 * (c < e ? c : e) + (c > e ? c - e : 0);
+  return w * u / (2 * e + nlate);
+}
+
 inline int pick_apply_stages(int D, int entries, int gate) {
   int st, sb, gs;
   pick_apply_plan(D, entries, gate, &st, &sb, &gs);
@@ -1208,13 +1218,8 @@ apply_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   // take half as many tiles as the others (they start last: see the launcher)
   long long u0, u1;
   if constexpr (LATE) {
-    auto tile_start = [&](long long c) {
-      const long long e = gridDim.x - nlate;
-      const long long w = 2 * (c < e ? c : e) + (c > e ? c - e : 0);
-      return w * U / (2 * e + nlate);
-    };
-    u0 = tile_start(blockIdx.x);
-    u1 = tile_start(blockIdx.x + 1);
+    u0 = apply_tile_start(blockIdx.x, gridDim.x, nlate, U);
+    u1 = apply_tile_start(blockIdx.x + 1, gridDim.x, nlate, U);
   } else {
     u0 = (long long)blockIdx.x * U / gridDim.x;
     u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;

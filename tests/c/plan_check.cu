@@ -4,7 +4,8 @@
 // fits its budget with at least two stages, so every bf16 call the library
 // accepts (tables of up to kMaxRopeEntries) has a tensor-core plan; two apply
 // CTAs of a half-budget plan fit in one SM's 228 KB with their reserved
-// shared memory; and the 480p and 720p grids take the intended plans.
+// shared memory; the 480p and 720p grids take the intended plans; and the
+// apply kernel's weighted tile split covers every tile.
 // Compiled by nvcc as host code and run on the CPU; prints "ok <checks>" or
 // the first failure.
 #include <stdio.h>
@@ -71,6 +72,25 @@ int main() {
   for (int e : {0, 1358, 2510, 3628, kMaxRopeEntries})
     REQUIRE(tc_supported(true, 128, 1, 32, 48, 48, e) && tc_supported(true, 64, 1, 16, 24, 24, e),
             "no tensor-core plan at %d entries", e);
+  // the apply kernel's weighted tile split, as the launcher enables it
+  // (u >= 2 g, nlate <= g / 4): every tile once, in order, at least one per
+  // CTA; nlate = 0 is the even split c * u / g
+  for (int g : {1, 2, 7, 100, 148, 296})
+    for (long long u = 2LL * g; u <= 8LL * 148; u += 13)
+      for (int nl = 0; 4 * nl <= g; ++nl) {
+        REQUIRE(apply_tile_start(0, g, nl, u) == 0 && apply_tile_start(g, g, nl, u) == u,
+                "split g=%d u=%lld nlate=%d does not cover the tiles", g, u, nl);
+        for (int c = 0; c < g; ++c) {
+          const long long a = apply_tile_start(c, g, nl, u), b = apply_tile_start(c + 1, g, nl, u);
+          REQUIRE(b - a >= 1, "split g=%d u=%lld nlate=%d: CTA %d gets %lld tiles", g, u, nl, c,
+                  b - a);
+          if (nl == 0) REQUIRE(a == c * u / g, "even split differs at CTA %d", c);
+        }
+      }
+  // a 720p block step (32 heads x 29 tiles on 148 CTAs, the last 32 light)
+  REQUIRE(apply_tile_start(116, 148, 32, 928) - apply_tile_start(115, 148, 32, 928) >= 7 &&
+              apply_tile_start(148, 148, 32, 928) - apply_tile_start(147, 148, 32, 928) <= 4,
+          "block-step split");
   printf("ok %lld\n", checks);
   return 0;
 }
