@@ -182,19 +182,24 @@ def _block_view(x, b, bt):
     return x[:, :, b * bt:(b + 1) * bt].contiguous()
 
 
-def test_block_steps_d128_gated_match_oracle():
-    # the carried state at D = 128 with the gate: two blocks, committed in turn
-    w = workloads.Workload("d128_steps", B=1, H=2, N=4 * 6 * 8, D=128, dtype="bf16",
-                           seed=25, grid=(4, 6, 8), rope_split=(32, 48, 48), gate=True,
-                           modes=("block_causal",), block_tokens=2 * 6 * 8)
+@pytest.mark.parametrize("grid,fpb", [((4, 6, 8), 2), ((4, 3, 134), 1)],
+                         ids=["4x6x8", "wide_table_4x3x134"])
+def test_block_steps_d128_gated_match_oracle(grid, fpb):
+    # the carried state at D = 128 with the gate, blocks committed in turn; a
+    # 1 x 3 x 134 block has 3580 RoPE table entries, too many for a two-tile
+    # gate ring beside the table (the apply kernel's one-tile ring)
+    T, Hg, Wg = grid
+    w = workloads.Workload("d128_steps", B=1, H=2, N=T * Hg * Wg, D=128, dtype="bf16",
+                           seed=25, grid=grid, rope_split=(32, 48, 48), gate=True,
+                           modes=("block_causal",), block_tokens=fpb * Hg * Wg)
     x = workloads.make_inputs(w)
     t = upload(w, x)
     bt = w.block_tokens
     st = la.BlockState(w.B, w.H, w.D)
     outs = [st.step(_block_view(t["q"], b, bt), _block_view(t["k"], b, bt),
-                    _block_view(t["v"], b, bt), _block_view(t["g"], b, bt), t_offset=2 * b,
-                    commit=True, grid=(2, 6, 8), rope_split=w.rope_split, eps=w.eps)
-            for b in range(2)]
+                    _block_view(t["v"], b, bt), _block_view(t["g"], b, bt), t_offset=fpb * b,
+                    commit=True, grid=(fpb, Hg, Wg), rope_split=w.rope_split, eps=w.eps)
+            for b in range(T // fpb)]
     seq = torch.cat(outs, dim=2)
     torch.cuda.synchronize()
     ref = oracle.forward(oracle.params_for(w, "block_causal"), x["q"], x["k"], x["v"],
