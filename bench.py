@@ -339,7 +339,9 @@ def measure_workload(w, mode, steps, warmup, pg, device, peak, peak_kind, seed):
 
 def measure_block_steps(w, steps, warmup, device, peak, peak_kind, seed):
     """Algorithm 1's per-block call: lin_attn_block_step with commit on every
-    block of the 720p workload, one call per block."""
+    block of the 720p workload, one call per block through BlockState.step.
+    Also the host time to issue one step (issue_us): below us_per_block the
+    GPU bounds the rate, near it the host does."""
     import torch
     import linear_attention_video_relu_b200 as la
     t = device_inputs(w, device, seed)
@@ -365,13 +367,16 @@ def measure_block_steps(w, steps, warmup, device, peak, peak_kind, seed):
     stream = torch.cuda.current_stream(device)
     a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    h0 = time.perf_counter()
     for _ in range(reps):
         run_all()
+    h1 = time.perf_counter()
     b_.record(stream)
     torch.cuda.synchronize(device)
     ms = a.elapsed_time(b_) / (reps * nblk)
     bytes_blk = 4 * w.B * w.H * bt * w.D * 2
     return {"workload": w.name + "_block_step", "block_tokens": bt, "us_per_block": ms * 1e3,
+            "issue_us": (h1 - h0) / (reps * nblk) * 1e6,
             "tokens_per_s": w.B * bt / (ms * 1e-3),
             "hbm_frac": bytes_blk / (ms * 1e-3) / 1e9 / peak}
 
@@ -655,7 +660,7 @@ def compact(r: dict) -> dict:
     if "ms_per_step" in r:
         c["ms"] = round(r["ms_per_step"], 4)
     for key, short in (("us_per_forward", "us"), ("us_per_call", "us"),
-                       ("us_per_block", "us_blk")):
+                       ("us_per_block", "us_blk"), ("issue_us", "issue_us")):
         if key in r:
             c[short] = round(r[key], 2)
     if "tokens_per_s" in r:

@@ -164,9 +164,10 @@ def test_secondary_lines_are_short():
              "us_per_forward": 61.66, "tokens_per_s": 5.3e8, "algorithmic_bytes": 1,
              "hbm_gbs": 4392.1, "hbm_frac": 0.672}
     blk = {"workload": "720p_long_block_step", "block_tokens": 3680, "us_per_block": 30.9,
-           "tokens_per_s": 1.19e8, "hbm_frac": 0.2986}
+           "issue_us": 18.234, "tokens_per_s": 1.19e8, "hbm_frac": 0.2986}
     lines = [bench.compact(r) for r in (full, cross, blk)]
     assert lines[1]["us"] == 61.66 and lines[2]["us_blk"] == 30.9
+    assert lines[2]["issue_us"] == 18.23
     full["kernels"]["apply"] = kern(320.5, 0.8123, 272841984)
     assert bench.compact(full)["ap"] == [320.5, 0.8123, 272.8]
     assert bench.compact(dict(cross, traffic=270900000))["traffic_MB"] == 270.9
