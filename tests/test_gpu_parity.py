@@ -390,26 +390,33 @@ def test_chained_calls_read_the_previous_output():
     _chain(lambda x: la.cross_forward(x, kv[0], kv[1], eps=w64.eps, workspace=wsc), t64["q"])
 
 
-def test_chained_block_steps_read_the_previous_output():
-    # Algorithm 1's per-block call at D = 128 (the apply kernel loads its
-    # first q stages before its dependency wait there): each step's q is the
-    # previous step's output, enqueued back to back; the same steps made one
-    # at a time after a synchronize, from the same starting state, give the
-    # same outputs and the same committed state, bit for bit.
-    w = workloads.Workload("chain_steps", B=1, H=2, N=3 * 6 * 8, D=128, dtype="bf16", seed=32,
-                           grid=(3, 6, 8), rope_split=(32, 48, 48), gate=True)
+@pytest.mark.parametrize("H,D,fgrid,split,gate", [
+    (2, 128, (1, 6, 8), (32, 48, 48), True),
+    # a 720p block: 32 heads x 3680 tokens, whose apply loads q early and
+    # gives its last CTAs half the tiles
+    (32, 64, (4, 23, 40), (16, 24, 24), False)], ids=["d128_gated", "720p_block"])
+def test_chained_block_steps_read_the_previous_output(H, D, fgrid, split, gate):
+    # Algorithm 1's per-block call where the apply kernel loads its first q
+    # stages before its dependency wait: each step's q is the previous step's
+    # output, enqueued back to back; the same steps made one at a time after a
+    # synchronize, from the same starting state, give the same outputs and
+    # the same committed state, bit for bit.
+    fpb, Hg, Wg = fgrid
+    w = workloads.Workload("chain_steps", B=1, H=H, N=3 * fpb * Hg * Wg, D=D, dtype="bf16",
+                           seed=32, grid=(3 * fpb, Hg, Wg), rope_split=split, gate=gate)
     t = upload(w, workloads.make_inputs(w))
-    bt = 6 * 8
-    blk = [{n: t[n][:, :, b * bt:(b + 1) * bt].contiguous() for n in ("q", "k", "v", "g")}
-           for b in range(3)]
-    kw = dict(grid=(1, 6, 8), rope_split=w.rope_split, eps=w.eps)
+    bt = fpb * Hg * Wg
+    names = ("q", "k", "v", "g") if gate else ("q", "k", "v")
+    blk = [{n: t[n][:, :, b * bt:(b + 1) * bt].contiguous() for n in names} for b in range(3)]
+    kw = dict(grid=fgrid, rope_split=w.rope_split, eps=w.eps)
 
     def run(sync):
         st = la.BlockState(w.B, w.H, w.D)
         x = blk[0]["q"]
         outs = []
         for b in range(3):
-            x = st.step(x, blk[b]["k"], blk[b]["v"], blk[b]["g"], t_offset=b, commit=True, **kw)
+            x = st.step(x, blk[b]["k"], blk[b]["v"], blk[b].get("g"), t_offset=b * fpb,
+                        commit=True, **kw)
             if sync:
                 torch.cuda.synchronize()
                 x = x.clone()
