@@ -182,12 +182,15 @@ def _block_view(x, b, bt):
     return x[:, :, b * bt:(b + 1) * bt].contiguous()
 
 
-@pytest.mark.parametrize("grid,fpb", [((4, 6, 8), 2), ((4, 3, 134), 1)],
-                         ids=["4x6x8", "wide_table_4x3x134"])
+@pytest.mark.parametrize("grid,fpb", [((4, 6, 8), 2), ((8, 6, 8), 4), ((4, 3, 134), 1)],
+                         ids=["4x6x8", "8x6x8", "wide_table_4x3x134"])
 def test_block_steps_d128_gated_match_oracle(grid, fpb):
-    # the carried state at D = 128 with the gate, blocks committed in turn; a
-    # 1 x 3 x 134 block has 3580 RoPE table entries, too many for a two-tile
-    # gate ring beside the table (the apply kernel's one-tile ring)
+    # the carried state at D = 128 with the gate, blocks committed in turn.
+    # The state build's tail takes each of its paths: 2 partials per head
+    # (the carried state transposed in shared memory), 3 (the partial slots
+    # fill the room: carried values read per item), 7 (partials read from
+    # L2). A 1 x 3 x 134 block has 3580 RoPE table entries, too many for a
+    # two-tile gate ring beside the table (the apply kernel's one-tile ring).
     T, Hg, Wg = grid
     w = workloads.Workload("d128_steps", B=1, H=2, N=T * Hg * Wg, D=128, dtype="bf16",
                            seed=25, grid=grid, rope_split=(32, 48, 48), gate=True,
