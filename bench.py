@@ -299,10 +299,14 @@ def roofline_entry(name, bytes_per_launch, ms_list, peak, peak_kind, workload):
     avg_ms = sum(ms_list) / len(ms_list)
     gbs = bytes_per_launch / (avg_ms * 1e-3) / 1e9
     traffic = ncu_traffic(name, workload)
-    return {"kernel": name, "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
-            "unit": "GB/s", "frac": round(gbs / peak, 4), "traffic": traffic,
-            "algorithmic_bytes": bytes_per_launch, "avg_us": round(avg_ms * 1e3, 2),
-            "peak_source": peak_kind}
+    e = {"kernel": name, "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+         "unit": "GB/s", "frac": round(gbs / peak, 4), "traffic": traffic,
+         "algorithmic_bytes": bytes_per_launch, "avg_us": round(avg_ms * 1e3, 2),
+         "peak_source": peak_kind}
+    if traffic is None:
+        e["traffic_note"] = ("no ncu capture of %s on %s for the current kernel sources "
+                             "(hash %s)" % (name, workload, kernel_source_hash("tc")))
+    return e
 
 
 def measure_workload(w, mode, steps, warmup, pg, device, peak, peak_kind, seed):

@@ -223,3 +223,14 @@ def test_every_committed_traffic_line_names_a_workload_the_bench_reads():
                 assert parts[2] in ("state_build", "apply", "temporal_conv"), (path, line)
                 assert parts[3] in keys, (path, parts[3], sorted(keys))
     assert seen >= 10
+
+
+def test_roofline_entry_says_why_traffic_is_null(monkeypatch):
+    monkeypatch.setattr(bench, "ncu_traffic", lambda k, w: None)
+    e = bench.roofline_entry("state_build", 268369920, [0.065, 0.066], 6535.7, "measured",
+                             "480p_bidir")
+    assert e["traffic"] is None and bench.kernel_source_hash("tc") in e["traffic_note"]
+    assert abs(e["frac"] - 268369920 / 0.0655e-3 / 1e9 / 6535.7) < 1e-4
+    monkeypatch.setattr(bench, "ncu_traffic", lambda k, w: 273690112)
+    e = bench.roofline_entry("state_build", 268369920, [0.065], 6535.7, "measured", "480p_bidir")
+    assert e["traffic"] == 273690112 and "traffic_note" not in e
