@@ -299,14 +299,19 @@ def roofline_entry(name, bytes_per_launch, ms_list, peak, peak_kind, workload):
     avg_ms = sum(ms_list) / len(ms_list)
     gbs = bytes_per_launch / (avg_ms * 1e-3) / 1e9
     traffic = ncu_traffic(name, workload)
-    e = {"kernel": name, "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
-         "unit": "GB/s", "frac": round(gbs / peak, 4), "traffic": traffic,
-         "algorithmic_bytes": bytes_per_launch, "avg_us": round(avg_ms * 1e3, 2),
-         "peak_source": peak_kind}
-    if traffic is None:
-        e["traffic_note"] = ("no ncu capture of %s on %s for the current kernel sources "
-                             "(hash %s)" % (name, workload, kernel_source_hash("tc")))
-    return e
+    return {"kernel": name, "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(gbs / peak, 4), "traffic": traffic,
+            "algorithmic_bytes": bytes_per_launch, "avg_us": round(avg_ms * 1e3, 2),
+            "peak_source": peak_kind}
+
+
+def traffic_note(line: dict):
+    """One short reason, for the whole line, when the roofline's traffic is
+    null: no committed ncu capture was taken on the current kernel sources."""
+    rf = line.get("roofline") or {}
+    if rf.get("traffic") is None and "kernel" in rf:
+        return "no ncu capture on kernel sources %s" % kernel_source_hash("tc")
+    return None
 
 
 def measure_workload(w, mode, steps, warmup, pg, device, peak, peak_kind, seed):
@@ -773,6 +778,9 @@ def main():
     }
     if args.workload != MAIN or mode != "bidirectional":
         line["metric"] = "linear-attn fwd tokens/s (profiling run: %s, %s)" % (w.name, mode)
+    note = traffic_note(line)
+    if note:
+        line["traffic_note"] = note
     if rank == 0 and args.e2e_steps > 0:
         line["e2e"] = measure_e2e(w, args.e2e_steps, device, w.seed)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -225,12 +225,14 @@ def test_every_committed_traffic_line_names_a_workload_the_bench_reads():
     assert seen >= 10
 
 
-def test_roofline_entry_says_why_traffic_is_null(monkeypatch):
+def test_null_roofline_traffic_is_explained_once(monkeypatch):
     monkeypatch.setattr(bench, "ncu_traffic", lambda k, w: None)
     e = bench.roofline_entry("state_build", 268369920, [0.065, 0.066], 6535.7, "measured",
                              "480p_bidir")
-    assert e["traffic"] is None and bench.kernel_source_hash("tc") in e["traffic_note"]
+    assert e["traffic"] is None
     assert abs(e["frac"] - 268369920 / 0.0655e-3 / 1e9 / 6535.7) < 1e-4
+    note = bench.traffic_note({"roofline": e})
+    assert bench.kernel_source_hash("tc") in note and len(note) < 60
     monkeypatch.setattr(bench, "ncu_traffic", lambda k, w: 273690112)
     e = bench.roofline_entry("state_build", 268369920, [0.065], 6535.7, "measured", "480p_bidir")
-    assert e["traffic"] == 273690112 and "traffic_note" not in e
+    assert e["traffic"] == 273690112 and bench.traffic_note({"roofline": e}) is None
